@@ -1,0 +1,322 @@
+"""Pins for the fp64 oracle (CPU only).
+
+Every oracle function is tied to something other than itself: hand-worked
+examples from the pages' definitions (tests/golden), closed forms, library
+routines (torch SDPA, torch.logsumexp, scipy's KS test), invariants, and brute
+force on tiny inputs. The last tests plant mistakes in the oracle and check
+that a pin catches each of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from oracle import margins as M
+from token_pruned_sparse_b200 import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _num(v):
+    return {"inf": math.inf, "ln3": math.log(3.0), "ln4": math.log(4.0)}.get(v, v) if isinstance(v, str) else v
+
+
+# ----------------------------------------------------------------- score ---
+def test_score_worked_examples():
+    g = _gold("score_worked.json")
+    for c in g["cases"]:
+        s = O.lipar_score(np.array([[c["cur"]]], float), np.array([[c["ref"]]], float))
+        assert s[0] == _num(c["score"])
+    fr = g["interframe"]
+    x = np.array(fr["x"], float)
+    assert list(O.lipar_score(x)) == [_num(v) for v in fr["score_no_prev"]]
+    assert list(O.lipar_score(x, x_prev_frame=np.array(fr["x_prev_frame"], float))) == \
+        [_num(v) for v in fr["score_with_prev"]]
+
+
+def test_score_linearity_and_zero_change():
+    rng = np.random.default_rng(0)
+    ref = rng.integers(-128, 129, (50, 1, 16)).astype(float) / 16
+    delta = rng.integers(-64, 65, (50, 1, 16)).astype(float) / 16
+    s1 = O.lipar_score(ref + delta, ref)
+    for lam in (0.25, 2.0, 8.0):
+        np.testing.assert_array_equal(O.lipar_score(ref + lam * delta, ref), lam * s1)
+    assert not O.lipar_score(ref, ref).any()
+    # zero change -> empty active set at any tau > 0 (inter-step and inter-frame)
+    assert len(O.select_threshold(O.lipar_score(ref, ref), 1e-6)) == 0
+    video = np.repeat(ref[:8].reshape(1, 8, 16), 5, axis=0)
+    s = O.lipar_score(video, x_prev_frame=video[0])
+    assert len(O.select_threshold(s, 1e-6)) == 0
+    # without a previous frame, frame 0 is always active
+    assert list(O.select_threshold(O.lipar_score(video), 1e-6)) == list(range(8))
+
+
+def test_score_matches_torch_norms():
+    """Relative L1 equals torch's vector 1-norm ratio (library witness)."""
+    x = synth.gaussian_bf16((6, 40, 32), 3)
+    r = synth.gaussian_bf16((6, 40, 32), 4)
+    xt, rt = x.double().reshape(-1, 32), r.double().reshape(-1, 32)
+    ref = (torch.linalg.vector_norm(xt - rt, ord=1, dim=1) / torch.linalg.vector_norm(rt, ord=1, dim=1)).numpy()
+    np.testing.assert_allclose(O.lipar_score(x, r), ref, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- select ---
+def test_topk_bruteforce_tiny():
+    """The selected set is the unique k-subset whose every member beats every
+    non-member by (score desc, index asc); checked by enumerating subsets."""
+    rng = np.random.default_rng(1)
+    for trial in range(60):
+        n = int(rng.integers(1, 9))
+        s = rng.integers(0, 4, n).astype(float)          # many ties
+        if trial % 3 == 0:
+            s[rng.integers(0, n)] = math.inf
+        for k in range(n + 1):
+            winners = [S for S in itertools.combinations(range(n), k)
+                       if all((s[a] > s[b]) or (s[a] == s[b] and a < b)
+                              for a in S for b in set(range(n)) - set(S))]
+            assert len(winners) == 1
+            assert list(O.select_topk(s, k)) == list(winners[0])
+
+
+def test_topk_equals_threshold_at_kth_score():
+    rng = np.random.default_rng(2)
+    s = rng.exponential(size=1000)
+    for k in (1, 10, 500, 999):
+        kth = np.sort(s)[::-1][k - 1]
+        assert list(O.select_topk(s, k)) == list(O.select_threshold(s, kth))
+    assert list(O.select_topk(s, 1000)) == list(range(1000))
+    assert len(O.select_topk(s, 0)) == 0
+
+
+def test_topk_golden_and_specials():
+    g = _gold("schedule_worked.json")
+    s = np.array(g["group_split"]["scores"])
+    assert list(O.select_topk(s, g["topk"]["k"])) == g["topk"]["idx"]
+    s2 = np.array([math.nan, -0.0, 0.0, 1.0, -math.inf])
+    assert list(O.select_topk(s2, 3)) == [1, 2, 3]         # -0 == +0, tie to lower index; NaN lowest
+    assert list(O.select_topk(s2, 4)) == [1, 2, 3, 4]
+    assert list(O.select_threshold(s2, 0.0)) == [1, 2, 3]
+
+
+def test_group_split_golden_and_invariants():
+    g = _gold("schedule_worked.json")["group_split"]
+    assert list(O.group_split(np.array(g["scores"]), 3)) == g["groups"]
+    rng = np.random.default_rng(3)
+    for N, K in ((30, 3), (31, 3), (100, 4), (7, 7)):
+        s = rng.integers(0, 5, N).astype(float)
+        grp = O.group_split(s, K)
+        sizes = np.bincount(grp, minlength=K)
+        assert list(sizes[:-1]) == [N // K] * (K - 1) and sizes[-1] == N - (K - 1) * (N // K)
+        for a in range(K - 1):                           # earlier groups change faster
+            assert s[grp == a].min() >= s[grp == a + 1].max()
+        # brute force: a token's group is fixed by how many tokens outrank it
+        for n in range(N):
+            rank = sum((s[m] > s[n]) or (s[m] == s[n] and m < n) for m in range(N))
+            assert grp[n] == min(rank // (N // K), K - 1)
+
+
+def test_schedule_golden_and_enumeration():
+    g = _gold("schedule_worked.json")
+    for m, key in ((0, "active_groups_m0"), (1, "active_groups_m1")):
+        for i in range(g["T"]):
+            assert list(O.schedule_groups(3, g["budgets"], g["T"], i, m).astype(int)) == g[key][i]
+    # the configured HSA schedule: T=40, budgets (40, 20, 10), thirds of 118800
+    T, budgets, N = 40, (40, 20, 10), 118800
+    grp = np.repeat(np.arange(3, dtype=np.int8), N // 3)
+    counts = np.zeros(3, int)
+    total = 0
+    for i in range(T):
+        act = O.schedule_groups(3, budgets, T, i, 0)
+        counts += act
+        A = len(O.schedule_active(grp, 3, budgets, T, i, 0))
+        total += A
+        assert A == {0: N, 2: 2 * N // 3}.get(i % 4, N // 3)
+    assert list(counts) == list(budgets)                 # each group runs exactly s_k steps
+    assert total * 3 == 70 * N                           # sum |A_i| = 23 1/3 N
+    for i in list(range(3)) + list(range(T - 3, T)):
+        assert len(O.schedule_active(grp, 3, budgets, T, i, 3)) == N
+
+
+# ---------------------------------------------------------- kv sync / RNG ---
+def test_kv_sync_rows_and_identity_renoise():
+    N, H, d, A = 50, 2, 8, 17
+    kc, vc = synth.gaussian_bf16((N, H, d), 1), synth.gaussian_bf16((N, H, d), 2)
+    kf, vf = synth.gaussian_bf16((A, H, d), 3), synth.gaussian_bf16((A, H, d), 4)
+    idx = np.sort(np.random.default_rng(5).choice(N, A, replace=False)).astype(np.int32)
+    k2, v2, ke, ve = O.kv_sync(kc, vc, kf, vf, idx, renoise=(1.0, 0.0, 9, 3))
+    pruned = np.setdiff1d(np.arange(N), idx)
+    assert torch.equal(k2[idx], kf) and torch.equal(v2[idx], vf)
+    assert torch.equal(k2[pruned], kc[pruned]) and torch.equal(v2[pruned], vc[pruned])
+    np.testing.assert_array_equal(ke, k2.double().numpy())   # a=1, b=0 -> bit-identical
+    np.testing.assert_array_equal(ve, v2.double().numpy())
+
+
+def test_renoise_statistics():
+    """z = (eff - a*c)/b over pruned rows is i.i.d. N(0,1): moments, KS test
+    (scipy), and K/V and step independence."""
+    from scipy import stats
+    N, H, d = 600, 4, 64
+    kc = synth.gaussian_bf16((N, H, d), 11)
+    vc = synth.gaussian_bf16((N, H, d), 12)
+    idx = np.arange(0, N, 3, dtype=np.int32)
+    a, b = 0.3, 0.7
+    _, _, ke, ve = O.kv_sync(kc, vc, kc[idx], vc[idx], idx, renoise=(a, b, 1234, 5))
+    pruned = np.setdiff1d(np.arange(N), idx)
+    zk = ((ke[pruned] - a * kc[pruned].double().numpy()) / b).ravel()
+    zv = ((ve[pruned] - a * vc[pruned].double().numpy()) / b).ravel()
+    n = zk.size
+    for z in (zk, zv):
+        assert abs(z.mean()) < 5 / math.sqrt(n)
+        assert abs(z.var() - 1) < 5 * math.sqrt(2 / n)
+        assert stats.kstest(z, "norm").pvalue > 1e-4
+    assert abs(np.corrcoef(zk, zv)[0, 1]) < 5 / math.sqrt(n)
+    e = np.arange(4096)
+    z5, z6 = O.renoise_normals(1234, 5, 0, e), O.renoise_normals(1234, 6, 0, e)
+    assert abs(np.corrcoef(z5, z6)[0, 1]) < 5 / math.sqrt(4096)
+    # active rows are the fresh rows, untouched by noise
+    np.testing.assert_array_equal(ke[idx], kc[idx].double().numpy())
+
+
+def test_philox_words_uniform_and_distinct():
+    """Raw stream: parity unpinned (no known-answer vectors offline); only
+    uniformity of the bytes and distinctness across counters are checked."""
+    from scipy import stats
+    w = O.philox_words(42, 0, 0, np.arange(1 << 14))
+    assert len(np.unique(w.reshape(-1))) > 0.999 * w.size
+    top = (w >> 24).ravel()
+    assert stats.chisquare(np.bincount(top, minlength=256)).pvalue > 1e-4
+    assert not np.array_equal(w, O.philox_words(42, 1, 0, np.arange(1 << 14)))
+    assert not np.array_equal(w, O.philox_words(42, 0, 1, np.arange(1 << 14)))
+    assert not np.array_equal(w, O.philox_words(43, 0, 0, np.arange(1 << 14)))
+
+
+# -------------------------------------------------------------- attention ---
+def _sdpa(q, k, v, scale, allowed=None):
+    """torch SDPA in fp64 on CPU, one head at a time: [A,H,d] x [N,H,d]."""
+    out = []
+    for h in range(q.shape[1]):
+        qq = q[:, h].double()[None, None]
+        kk = k[:, h].double()[None, None]
+        vv = v[:, h].double()[None, None]
+        m = None if allowed is None else torch.from_numpy(allowed)[None, None]
+        out.append(torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=m, scale=scale)[0, 0])
+    return torch.stack(out, 1).numpy()
+
+
+def test_attn_worked_example():
+    g = _gold("attn_worked.json")
+    q = torch.tensor([[[_num(g["q"])]]], dtype=torch.float64)
+    k = torch.tensor([[[_num(x)]] for x in g["k"]], dtype=torch.float64)
+    v = torch.tensor([[[x]] for x in g["v"]], dtype=torch.float64)
+    o, lse = O.pruned_attn(q, k, v, [0], 1.0)
+    assert abs(o[0, 0, 0] - g["o"]) < 1e-12 and abs(lse[0, 0] - _num(g["lse"])) < 1e-12
+
+
+@pytest.mark.parametrize("N,A,H,d", [(300, 300, 2, 64), (517, 131, 3, 128)])
+def test_attn_dense_matches_sdpa(N, A, H, d):
+    """All-active (k = N) equals textbook dense softmax attention."""
+    q = synth.gaussian_bf16((A, H, d), 21)
+    k = synth.gaussian_bf16((N, H, d), 22)
+    v = synth.gaussian_bf16((N, H, d), 23)
+    idx = np.sort(np.random.default_rng(0).choice(N, A, replace=False))
+    for scale in (1 / math.sqrt(d), 0.5):
+        o, lse = O.pruned_attn(q, k, v, idx, scale)
+        np.testing.assert_allclose(o, _sdpa(q, k, v, scale), rtol=1e-9, atol=1e-11)
+        s = torch.einsum("ahd,nhd->ahn", q.double(), k.double()) * scale
+        np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=1e-12)
+
+
+def test_attn_blockmask_matches_sdpa():
+    N, H, d, blk = 700, 2, 64, 128
+    A = 300
+    q = synth.gaussian_bf16((A, H, d), 31)
+    k = synth.gaussian_bf16((N, H, d), 32)
+    v = synth.gaussian_bf16((N, H, d), 33)
+    idx = np.sort(np.random.default_rng(1).choice(N, A, replace=False))
+    nb = -(-N // blk)
+    bm = (np.random.default_rng(2).random((nb, nb)) < 0.4).astype(np.uint8)
+    bm[np.arange(nb), np.arange(nb)] = 1
+    allowed = np.array([[bm[i // blk, n // blk] for n in range(N)] for i in idx], bool)
+    o, _ = O.pruned_attn(q, k, v, idx, 0.125, blockmask=bm, block=blk)
+    np.testing.assert_allclose(o, _sdpa(q, k, v, 0.125, allowed), rtol=1e-9, atol=1e-11)
+    # a query whose mask row keeps nothing gets o = 0, lse = -inf
+    bm2 = bm.copy()
+    bm2[idx[0] // blk] = 0
+    o2, l2 = O.pruned_attn(q, k, v, idx, 0.125, blockmask=bm2, block=blk, rows=[0])
+    assert not o2.any() and np.all(np.isneginf(l2))
+
+
+def test_attn_constant_keys_give_mean_of_v():
+    N, H, d = 333, 2, 64
+    k = synth.gaussian_bf16((1, H, d), 41).expand(N, H, d).contiguous()
+    v = synth.gaussian_bf16((N, H, d), 42)
+    q = synth.gaussian_bf16((20, H, d), 43)
+    o, lse = O.pruned_attn(q, k, v, np.arange(20), 0.3)
+    np.testing.assert_allclose(o, np.broadcast_to(v.double().mean(0).numpy(), o.shape), rtol=1e-12, atol=1e-13)
+    blk = 128
+    bm = np.zeros((3, 3), np.uint8)
+    bm[:, 1] = 1
+    o, _ = O.pruned_attn(q, k, v, np.arange(20), 0.3, blockmask=bm, block=blk)
+    np.testing.assert_allclose(o, np.broadcast_to(v[128:256].double().mean(0).numpy(), o.shape), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- scatter ---
+def test_scatter_and_gather_rows():
+    full = synth.gaussian_bf16((40, 2, 8), 51)
+    act = synth.gaussian_bf16((9, 2, 8), 52)
+    idx = np.array([0, 3, 4, 10, 11, 20, 30, 38, 39], np.int32)
+    out = O.scatter_out(full, act, idx)
+    assert torch.equal(out[idx], act)
+    rest = np.setdiff1d(np.arange(40), idx)
+    assert torch.equal(out[rest], full[rest])
+    assert torch.equal(O.gather_rows(out, idx), act)
+    assert torch.equal(O.scatter_out(full, act[:0], idx[:0]), full)
+
+
+# ------------------------------------------------------------- margins ---
+def test_margin_enforcement_keeps_selection_gap():
+    spec = synth.VideoSpec(5, 10, 12, 32, 2, 3, True, 9)
+    x, _ = synth.latent_video(spec)
+    xb = M.enforce_frame_margin(synth.to_bf16(x), ranks=(300,))
+    s = O.lipar_score(xb)
+    srt = np.sort(s)[::-1]
+    assert srt[299] >= srt[300] * (1 + M.MARGIN)
+    vp, dl = synth.velocity_pair(spec)
+    vpb = synth.to_bf16(vp)
+    vc = M.enforce_step_margin(vpb, dl, ranks=(200, 400))
+    s = np.sort(O.lipar_score(vc[None], vpb[None]))[::-1]
+    assert s[199] >= s[200] * (1 + M.MARGIN) and s[399] >= s[400] * (1 + M.MARGIN)
+
+
+# ------------------------------------------------------- planted mistakes ---
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """Each plausible slip in the oracle fails at least one pin."""
+    g = _gold("score_worked.json")["cases"][0]
+    cur, ref = np.array([[g["cur"]]], float), np.array([[g["ref"]]], float)
+    # dropped |.| in the denominator
+    bad = lambda x, r: np.abs(x - r).sum(-1) / r.sum(-1)
+    assert bad(cur, ref)[0, 0] != g["score"]
+    # transposed operands (score against the current token instead of the reference)
+    assert O.lipar_score(ref, cur)[0] != g["score"]
+    # attention without the scale, or with keys/values swapped, breaks the SDPA pin
+    q = synth.gaussian_bf16((8, 1, 64), 1)
+    k = synth.gaussian_bf16((50, 1, 64), 2)
+    v = synth.gaussian_bf16((50, 1, 64), 3)
+    ref_o = _sdpa(q, k, v, 0.125)
+    assert np.abs(O.pruned_attn(q, k, v, np.arange(8), 1.0)[0] - ref_o).max() > 1e-3
+    assert np.abs(O.pruned_attn(q, v, k, np.arange(8), 0.125)[0] - ref_o).max() > 1e-3
+    # ties to the HIGHER index would break the brute-force top-k pin
+    s = np.array([1.0, 1.0, 0.0])
+    assert list(O.select_topk(s, 1)) == [0]
+    # a strict '>' threshold would select k-1 at tau = s_(k)
+    assert len(O.select_threshold(np.array([3.0, 2.0, 1.0]), 2.0)) == 2
