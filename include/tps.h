@@ -1,0 +1,210 @@
+/*
+ * tps.h -- C ABI of libtps.so: token-pruned attention for video diffusion
+ * transformers on NVIDIA B200 (sm_100a).
+ *
+ * The path, per denoising step and layer:
+ *   lipar_score   -> per-token relative-L1 change             (float32 [N])
+ *   lipar_select  -> ascending active index list idx + count  (int32, device)
+ *   lipar_group / lipar_schedule -> HSA step groups and per-step active list
+ *   tps_gather_rows -> the active tokens' rows (input of the QKV projection)
+ *   kv_sync       -> fresh K/V rows into the layer cache (+ noise-aware re-noise)
+ *   pruned_attn   -> active queries attend all N cached keys (optional key-block mask)
+ *   scatter_out   -> active outputs written back over the cached outputs
+ *
+ * Sources (gist.science technical summaries):
+ *   [LIPAR] "Training-free Latent Inter-Frame Pruning with Attention Recovery"
+ *   [HSA]   "Resumen Tecnico: Asignacion de Pasos Heterogenea (HSA) para la
+ *            Generacion Eficiente de Video"
+ *   [SVOO]  "Training-Free Sparse Attention for Fast Video Generation via Offline
+ *            Layer-Wise Sparsity Profiling and Online Bidirectional Co-Clustering"
+ *   [TR]    "Timeripple: Accelerating vDiTs by Understanding the Spatio-Temporal
+ *            Correlations in Latent Space"
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates device memory and keeps no pointer after the call returns.
+ *     Exceptions are marked HOST.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns (tps_bf16), row-major.
+ *     Token-major layouts: a K/V/Q/O row of token n is the H*d contiguous
+ *     values of [N, H, d].
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream). Argument errors are detected on the host before any
+ *     launch and leave all outputs untouched.
+ *   - The active count lives in device memory (`count`, int32), so no host
+ *     synchronisation is needed between stages; `cap` is the host-known upper
+ *     bound of the count used to size grids. Rows j >= min(*count, cap) are
+ *     ignored.
+ *   - Index entries outside [0, N) are skipped by the kernels and recorded in
+ *     a device status word (TPS_ERR_BOUNDS); tps_check() reports it.
+ *   - Return value: one of the TPS_* status codes; tps_last_error() gives a
+ *     message for the calling host thread.
+ */
+#ifndef TPS_H_
+#define TPS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TPS_API __attribute__((visibility("default")))
+#else
+#define TPS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes --------------------------------------------------------- */
+#define TPS_OK               0
+#define TPS_ERR_INVALID_ARG  1  /* null pointer, bad mode, k > N, d not 64/128, ... */
+#define TPS_ERR_SHAPE        2  /* sizes out of the supported range               */
+#define TPS_ERR_ALIGN        3  /* a pointer is not 16-byte aligned               */
+#define TPS_ERR_CUDA         4  /* a CUDA runtime/driver call failed (message)    */
+#define TPS_ERR_TIMEOUT      5  /* a bounded device wait gave up (tps_check)      */
+#define TPS_ERR_BOUNDS       6  /* an index outside [0, N) was skipped (tps_check)*/
+#define TPS_ERR_WORKSPACE    7  /* workspace null or smaller than required        */
+
+typedef uint16_t tps_bf16;   /* bfloat16 bit pattern                  */
+typedef void*    tps_stream; /* cudaStream_t                          */
+
+/* ---- step 1: token score ([LIPAR] 2.B; [HSA] 2.1) ---------------------------
+ * Relative L1 change per token:  s = sum_c |cur_c - ref_c| / sum_c |ref_c|,
+ * computed in fp32 from bf16. den = 0 gives 0 when num = 0, else +inf.
+ *   x            [F, HW, C] bf16, the current latent tokens (N = F*HW).
+ *   x_ref        NULL: inter-frame mode, token (f,p) against (f-1,p).
+ *                non-NULL: inter-step mode, [F, HW, C] bf16, token n against
+ *                x_ref[n] (e.g. the previous step's velocity prediction).
+ *   x_prev_frame inter-frame only: [HW, C] bf16 reference for frame 0; NULL
+ *                makes every frame-0 score +inf (always active).
+ *   score        [F*HW] float32 output.
+ * Requires C % 8 == 0, 8 <= C <= 4096, F*HW < 2^31, 16-byte aligned pointers. */
+TPS_API int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame,
+                int64_t F, int64_t HW, int64_t C, float* score, tps_stream stream);
+
+/* ---- steps 2-3: active set and compaction ([LIPAR] 2.B; [HSA] 2.1) ---------
+ * mode TPS_SELECT_THRESHOLD: active iff score >= tau (a token below tau is
+ *   redundant and pruned). NaN is never active.
+ * mode TPS_SELECT_TOPK: the k highest scores; equal scores go to the lower
+ *   index; NaN ranks below -inf; -0 equals +0. 0 <= k <= N.
+ * Output: idx[0 .. *count) ascending int32 token indices (idx must hold N
+ *   entries for threshold mode, k for top-k), *count written on the device.
+ * ws: device workspace of at least tps_workspace_size(TPS_OP_SELECT, N, 0)
+ *   bytes, 16-byte aligned; its contents need no initialisation. Calls that
+ *   share one workspace must be ordered on the GPU (same stream). */
+#define TPS_SELECT_THRESHOLD 0
+#define TPS_SELECT_TOPK      1
+TPS_API int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
+                 int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, tps_stream stream);
+
+/* ---- HSA group assignment ([HSA] 2.1, dynamic token selection) -------------
+ * Ranks tokens by score descending (ties to the lower index, NaN last) and
+ * splits the ranks into K contiguous groups of N/K (the remainder joins the
+ * last group). group[n] = 0 for the fastest-changing third (the reference
+ * group G_1 with the full budget), K-1 for the slowest. 1 <= K <= 8, K <= N.
+ * ws: tps_workspace_size(TPS_OP_GROUP, N, K) bytes. */
+TPS_API int lipar_group(const float* score, int64_t N, int K, int8_t* group,
+                void* ws, size_t ws_bytes, tps_stream stream);
+
+/* ---- HSA per-step active set ([HSA] 2.1 schedule, 2.4 phase window) --------
+ * Group k is active at global step `step` iff step mod (T / budgets[k]) == 0;
+ * every group is active when step < m or step >= T - m.
+ *   budgets  HOST int32[K], each a divisor of T (budgets[0] = T for G_1).
+ *   group    [N] int8 from lipar_group (values outside [0, K) are never active).
+ *   idx, count as for lipar_select (idx holds N entries).
+ * ws: tps_workspace_size(TPS_OP_SCHEDULE, N, K) bytes. */
+TPS_API int lipar_schedule(const int8_t* group, int64_t N, int K, const int32_t* budgets, int T,
+                   int step, int m, int32_t* idx, int32_t* count,
+                   void* ws, size_t ws_bytes, tps_stream stream);
+
+/* ---- gather of active rows ([HSA] 2.2 (1): only active tokens enter the
+ * QKV projection) --------------------------------------------------------------
+ * dst[j] = src[idx[j]] for j < min(*count, cap); rows of row_bytes bytes
+ * (row_bytes % 16 == 0); src has N rows, dst cap rows. */
+TPS_API int tps_gather_rows(void* dst, const void* src, const int32_t* idx, const int32_t* count,
+                    int64_t cap, int64_t N, int64_t row_bytes, tps_stream stream);
+
+/* ---- step 4: KV-cache synchronisation ([HSA] 2.2 (2); [LIPAR] 2.C) ---------
+ * k_cache[idx[j]] = k_fresh[j] and v_cache[idx[j]] = v_fresh[j] for
+ * j < min(*count, cap) (bit copies), caches [N, H, d], fresh [cap, H, d].
+ * rn == NULL: nothing else; k_eff / v_eff are not touched (may be NULL).
+ * rn != NULL (noise-aware duplication): additionally writes the attention
+ *   inputs k_eff, v_eff [N, H, d]: active rows = the fresh rows; pruned rows
+ *   n = bf16_rne(a * cache[n] + b * eps), eps ~ N(0,1) from Philox4x32-10
+ *   (Salmon et al., SC'11) with counter (q mod 2^32, q div 2^32, step,
+ *   tensor: 0 = K, 1 = V), key (seed mod 2^32, seed div 2^32), q = e div 4 for
+ *   flat element e = (n*H + h)*d + c, word e mod 4 mapped to
+ *   u = (floor(w/2^9) + 1/2) * 2^-23, Box-Muller over words (0,1) and (2,3).
+ *   The cache is not overwritten by noised rows. idx must be ascending.
+ * d in {64, 128}; H*d <= 16384; N < 2^31. */
+typedef struct tps_renoise {
+  float    a;     /* weight of the clean cached row   */
+  float    b;     /* weight of the fresh noise        */
+  uint64_t seed;  /* Philox key                       */
+  uint32_t step;  /* denoising step (counter word 2)  */
+  uint32_t pad_;
+} tps_renoise;
+
+TPS_API int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_fresh,
+            const tps_bf16* v_fresh, const int32_t* idx, const int32_t* count, int64_t cap,
+            int64_t N, int H, int d, const tps_renoise* rn /* HOST, may be NULL */,
+            tps_bf16* k_eff, tps_bf16* v_eff, tps_stream stream);
+
+/* ---- step 5: pruned attention ([HSA] 2.2 (3)-(4); [SVOO] part 2; [TR]) ------
+ * For every active row j < min(*count, cap) and head h:
+ *   o_act[j,h] = sum_n softmax_n(scale * q_act[j,h] . k[n,h]) v[n,h]
+ * over all n < N, or, with a key-block mask, only over keys n whose block
+ * n / block has blockmask[(idx[j] / block) * nb + n / block] != 0, where
+ * nb = ceil(N / block): the mask row is the query's ORIGINAL token block.
+ *   q_act  [cap, H, d] bf16; k, v [N, H, d] bf16; o_act [cap, H, d] bf16 (RNE).
+ *   blockmask NULL (dense) or uint8 [nb, nb] (block must be 128, nb <= 4096).
+ *   lse    NULL or float32 [cap, H]: natural-log sum of exp of the scaled
+ *          logits. A row with no allowed key gets o = 0 and lse = -inf.
+ * bf16 inputs, fp32 accumulation and softmax, tcgen05 tensor cores.
+ * d in {64, 128}; 1 <= H <= 256; N < 2^31; pointers 16-byte aligned. */
+TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
+                const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
+                float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
+                tps_stream stream);
+
+/* Same contract as pruned_attn, computed with the legacy warp-level
+ * mma.sync tensor-core path (kept as the baseline the tcgen05 kernel is
+ * measured against). */
+TPS_API int pruned_attn_mma(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
+                    const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H,
+                    int d, float scale, const uint8_t* blockmask, int block, tps_bf16* o_act,
+                    float* lse, tps_stream stream);
+
+/* ---- step 6: restoration ([LIPAR] Dutch summary 2.D) -------------------------
+ * o_full[idx[j]] = o_act[j] for j < min(*count, cap); every other row of
+ * o_full [N, H, d] keeps its cached output bit for bit. */
+TPS_API int scatter_out(tps_bf16* o_full, const tps_bf16* o_act, const int32_t* idx,
+                const int32_t* count, int64_t cap, int64_t N, int H, int d, tps_stream stream);
+
+/* ---- support --------------------------------------------------------------- */
+#define TPS_OP_SELECT   0
+#define TPS_OP_GROUP    1
+#define TPS_OP_SCHEDULE 2
+/* Workspace bytes for lipar_select / lipar_group / lipar_schedule (0 on bad op). */
+TPS_API size_t tps_workspace_size(int op, int64_t N, int K);
+
+/* Message of the last failing call on this host thread ("" if none). */
+TPS_API const char* tps_last_error(void);
+
+/* Synchronises `stream`, then reads and clears this device's status word:
+ * TPS_OK, TPS_ERR_BOUNDS (an index was skipped) or TPS_ERR_TIMEOUT (a bounded
+ * device wait gave up), or TPS_ERR_CUDA if the synchronisation failed. */
+TPS_API int tps_check(tps_stream stream);
+
+/* Debug export: the raw Philox4x32-10 words used by kv_sync's re-noise, for
+ * counter blocks q0 .. q0+nq-1: out[4*i + w] = word w of block q0 + i. */
+TPS_API int tps_philox_fill(uint32_t* out, uint64_t q0, int64_t nq, uint64_t seed, uint32_t step,
+                    uint32_t tensor, tps_stream stream);
+
+/* Library version string. */
+TPS_API const char* tps_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TPS_H_ */

@@ -201,14 +201,14 @@ def renoise_normals(seed: int, step: int, tensor: int, e) -> np.ndarray:
     """N(0,1) deviate for flat element index e (float64).
 
     Element e uses word (e mod 4) of counter block q = e div 4. Each word w
-    maps to u = (floor(w / 2^8) + 1/2) * 2^-24 in (0, 1). Words (0, 1) and
-    (2, 3) form Box-Muller pairs: r = sqrt(-2 ln u_a), z_a = r cos(2 pi u_b),
-    z_b = r sin(2 pi u_b)."""
+    maps to u = (floor(w / 2^9) + 1/2) * 2^-23 in (0, 1), a value that is
+    exact in fp32 as well as fp64. Words (0, 1) and (2, 3) form Box-Muller
+    pairs: r = sqrt(-2 ln u_a), z_a = r cos(2 pi u_b), z_b = r sin(2 pi u_b)."""
     e = np.asarray(e, np.int64)
     q = (e >> 2).astype(np.uint64)
     j = e & 3
     w = philox_words(seed, step, tensor, q).astype(np.float64)
-    u = (np.floor(w / 256.0) + 0.5) * 2.0 ** -24
+    u = (np.floor(w / 512.0) + 0.5) * 2.0 ** -23
     pair = (j >> 1) * 2                       # 0 for words 0/1, 2 for words 2/3
     ua = np.take_along_axis(u, pair[:, None], 1)[:, 0]
     ub = np.take_along_axis(u, (pair + 1)[:, None], 1)[:, 0]
@@ -219,7 +219,7 @@ def renoise_normals(seed: int, step: int, tensor: int, e) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Step 4: KV-cache synchronisation (+ noise-aware duplication)
 # ---------------------------------------------------------------------------
-def kv_sync(k_cache, v_cache, k_fresh, v_fresh, idx, renoise=None):
+def kv_sync(k_cache, v_cache, k_fresh, v_fresh, idx, renoise=None, heads=None):
     """[HSA] 2.2: only active tokens produce fresh K/V; those rows overwrite the
     per-layer cache, the other rows stay stale but valid. Returns the updated
     caches (bf16, bit copies) and, when ``renoise`` is given, float64 K_eff /
@@ -230,6 +230,9 @@ def kv_sync(k_cache, v_cache, k_fresh, v_fresh, idx, renoise=None):
     eff[n] = a * cache[n] + b * eps(n), eps drawn independently for K (tensor
     0) and V (tensor 1) at flat element (n*H + h)*d + c; active rows take the
     fresh row. The noised rows are not written back into the cache.
+
+    ``heads`` restricts K_eff / V_eff to a subset of heads (shape [N, len(heads),
+    d]) for sampled checks at full size.
     """
     kc = k_cache.clone()
     vc = v_cache.clone()
@@ -241,14 +244,17 @@ def kv_sync(k_cache, v_cache, k_fresh, v_fresh, idx, renoise=None):
         return kc, vc, None, None
     a, b, seed, step = renoise
     N, H, d = kc.shape
+    heads = np.arange(H) if heads is None else np.asarray(heads, np.int64)
     pruned = np.setdiff1d(np.arange(N), np.asarray(idx, np.int64))
+    cols = (heads[:, None] * d + np.arange(d)[None, :]).reshape(-1)      # flat (h, c) offsets
     out = []
     for t, cache in ((0, kc), (1, vc)):
-        eff = f64(cache)
-        if len(pruned):
-            e = (pruned[:, None] * (H * d) + np.arange(H * d)[None, :]).reshape(-1)
-            z = renoise_normals(seed, step, t, e).reshape(len(pruned), H, d)
-            eff[pruned] = a * eff[pruned] + b * z
+        eff = f64(cache[:, torch.as_tensor(heads)])
+        for p0 in range(0, len(pruned), 4096):
+            rows = pruned[p0:p0 + 4096]
+            e = (rows[:, None] * (H * d) + cols[None, :]).reshape(-1)
+            z = renoise_normals(seed, step, t, e).reshape(len(rows), len(heads), d)
+            eff[rows] = a * eff[rows] + b * z
         out.append(eff)
     return kc, vc, out[0], out[1]
 
@@ -273,11 +279,8 @@ def pruned_attn(q_act, k, v, idx, scale: float, blockmask=None, block: int = 128
     size); ``heads`` to a subset of heads. Returns float64 (o [R, Hs, d],
     lse [R, Hs]).
     """
-    Q = f64(q_act)
-    Kf = f64(k)
-    Vf = f64(v)
-    A, H, d = Q.shape
-    N = Kf.shape[0]
+    A, H, d = q_act.shape
+    N = k.shape[0]
     idx = np.asarray(idx, np.int64)
     rows = np.arange(A) if rows is None else np.asarray(rows, np.int64)
     heads = np.arange(H) if heads is None else np.asarray(heads, np.int64)
@@ -289,20 +292,19 @@ def pruned_attn(q_act, k, v, idx, scale: float, blockmask=None, block: int = 128
         bm = np.asarray(blockmask.cpu().numpy() if isinstance(blockmask, torch.Tensor) else blockmask) != 0
         key_block = np.arange(N) // block
     chunk = max(1, min(len(rows), (1 << 24) // max(N, 1)))
-    for c0 in range(0, len(rows), chunk):
-        r = rows[c0:c0 + chunk]
-        if blockmask is not None:
-            allowed = bm[idx[r] // block][:, key_block]            # [c, N]
-        for hi, h in enumerate(heads):
-            S = (Q[r, h] @ Kf[:, h].T) * scale                     # [c, N]
+    for hi, h in enumerate(heads):
+        Kh, Vh = f64(k[:, h]), f64(v[:, h])                        # one head in fp64
+        for c0 in range(0, len(rows), chunk):
+            r = rows[c0:c0 + chunk]
+            S = (f64(q_act[r, h]) @ Kh.T) * scale                  # [c, N]
             if blockmask is not None:
-                S = np.where(allowed, S, -np.inf)
+                S = np.where(bm[idx[r] // block][:, key_block], S, -np.inf)
             mx = S.max(axis=1)
             ok = np.isfinite(mx)
             P = np.exp(S - np.where(ok, mx, 0.0)[:, None])
             P[~ok] = 0.0
             l = P.sum(axis=1)
-            O = P @ Vf[:, h]
+            O = P @ Vh
             o[c0:c0 + len(r), hi] = np.where(ok[:, None], O / np.where(ok, l, 1.0)[:, None], 0.0)
             lse[c0:c0 + len(r), hi] = np.where(ok, mx + np.log(np.where(ok, l, 1.0)), -np.inf)
     return o, lse

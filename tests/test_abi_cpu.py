@@ -1,0 +1,99 @@
+"""C ABI checks that need no GPU: the library loads, exports every function
+include/tps.h declares, and rejects bad arguments on the host (before any CUDA
+call) with the documented status codes and a message."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from token_pruned_sparse_b200 import tps
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tps.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^TPS_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared()
+    for n in ("lipar_score", "lipar_select", "lipar_group", "lipar_schedule", "kv_sync", "pruned_attn",
+              "scatter_out", "tps_gather_rows", "tps_workspace_size", "tps_last_error", "tps_check"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tps.lib()
+    missing = [n for n in declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(tps.SIGNATURES) >= set(declared())
+    assert "sm_100a" in tps.version()
+
+
+F = C.c_void_p(0x1000)        # fake, 16-byte aligned, never dereferenced
+MIS = C.c_void_p(0x1001)      # misaligned
+NULL = None
+
+
+def _err(code):
+    return code, tps.lib().tps_last_error().decode()
+
+
+def test_score_validation():
+    l = tps.lib()
+    assert _err(l.lipar_score(NULL, NULL, NULL, 2, 4, 64, F, NULL))[0] == tps.INVALID_ARG
+    code, msg = _err(l.lipar_score(F, NULL, NULL, 2, 4, 60, F, NULL))
+    assert code == tps.SHAPE and "C=60" in msg
+    assert l.lipar_score(MIS, NULL, NULL, 2, 4, 64, F, NULL) == tps.ALIGN
+    assert l.lipar_score(F, F, F, 2, 4, 64, F, NULL) == tps.INVALID_ARG
+    assert l.lipar_score(F, NULL, NULL, 0, 4, 64, F, NULL) == tps.SHAPE
+
+
+def test_select_validation_and_workspace():
+    l = tps.lib()
+    assert l.lipar_select(F, 10, 5, 0.0, 0, F, F, F, 1 << 20, NULL) == tps.INVALID_ARG
+    code, msg = _err(l.lipar_select(F, 10, tps.SELECT_TOPK, 0.0, 11, F, F, F, 1 << 20, NULL))
+    assert code == tps.INVALID_ARG and "k=11" in msg
+    need = tps.workspace_size(tps.OP_SELECT, 100000)
+    assert need > 0 and tps.workspace_size(tps.OP_SELECT, 200000) > need
+    code, msg = _err(l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, F, need - 1, NULL))
+    assert code == tps.WORKSPACE and "required" in msg
+    assert l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, NULL, need, NULL) == tps.WORKSPACE
+    assert l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, MIS, need, NULL) == tps.ALIGN
+    assert tps.workspace_size(9, 10) == 0
+    assert l.lipar_group(F, 10, 9, F, F, 1 << 20, NULL) == tps.INVALID_ARG
+    assert l.lipar_group(F, 2, 3, F, F, 1 << 20, NULL) == tps.INVALID_ARG
+    bad = (C.c_int32 * 3)(40, 20, 7)                     # 7 does not divide 40
+    code, msg = _err(l.lipar_schedule(F, 10, 3, C.cast(bad, C.c_void_p), 40, 0, 0, F, F, F, 1 << 20, NULL))
+    assert code == tps.INVALID_ARG and "divide" in msg
+    good = (C.c_int32 * 3)(40, 20, 10)
+    assert l.lipar_schedule(F, 10, 3, C.cast(good, C.c_void_p), 40, 40, 0, F, F, F, 1 << 20, NULL) == tps.INVALID_ARG
+
+
+def test_rows_and_attention_validation():
+    l = tps.lib()
+    assert l.kv_sync(F, F, F, F, F, F, 10, 100, 2, 96, NULL, NULL, NULL, NULL) == tps.INVALID_ARG
+    assert l.kv_sync(F, F, F, F, NULL, F, 10, 100, 2, 64, NULL, NULL, NULL, NULL) == tps.INVALID_ARG
+    rn = tps.Renoise(0.5, 0.5, 1, 0, 0)
+    assert l.kv_sync(F, F, F, F, F, F, 10, 100, 2, 64, C.cast(C.byref(rn), C.c_void_p), NULL, NULL, NULL) == \
+        tps.INVALID_ARG
+    assert l.kv_sync(MIS, F, F, F, F, F, 10, 100, 2, 64, NULL, NULL, NULL, NULL) == tps.ALIGN
+    assert l.scatter_out(F, F, F, F, 10, 0, 2, 64, NULL) == tps.SHAPE
+    assert l.tps_gather_rows(F, F, F, F, 10, 100, 24, NULL) == tps.SHAPE
+    for fn in (l.pruned_attn, l.pruned_attn_mma):
+        assert fn(F, F, F, F, F, 10, 100, 2, 80, 0.1, NULL, 128, F, NULL, NULL) == tps.INVALID_ARG
+        assert fn(F, F, F, F, F, 10, 100, 0, 64, 0.1, NULL, 128, F, NULL, NULL) == tps.SHAPE
+        assert fn(F, F, F, F, F, 10, 100, 2, 64, 0.1, F, 64, F, NULL, NULL) == tps.INVALID_ARG
+        assert fn(F, F, F, F, F, 10, 4097 * 128, 2, 64, 0.1, F, 128, F, NULL, NULL) == tps.SHAPE
+        assert fn(MIS, F, F, F, F, 10, 100, 2, 64, 0.1, NULL, 128, F, NULL, NULL) == tps.ALIGN
+        assert fn(F, F, F, F, F, 10, 100, 2, 64, float("nan"), NULL, 128, F, NULL, NULL) == tps.INVALID_ARG
+    assert l.tps_philox_fill(MIS, 0, 4, 1, 0, 0, NULL) == tps.ALIGN
+
+
+def test_binding_raises_with_message():
+    with pytest.raises(tps.TPSError) as e:
+        tps._chk(tps.lib().lipar_score(NULL, NULL, NULL, 2, 4, 64, F, NULL))
+    assert e.value.code == tps.INVALID_ARG and "non-null" in str(e.value)

@@ -1,0 +1,249 @@
+"""GPU parity: pruned attention (tcgen05 kernel and the legacy mma.sync
+baseline) vs the fp64 oracle, through the C ABI; plus the whole per-layer path
+on the configs, at full size with sampled rows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from token_pruned_sparse_b200 import synth
+from token_pruned_sparse_b200 import tps
+
+from workloads import attn_tolerance_ok, frame_case, oracle_idx, qkv, step_case
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+IMPLS = ["pruned_attn", "pruned_attn_mma"]
+
+
+def _run(impl, q, k, v, idx, scale, bm=None, with_lse=True, count=None, cap=None):
+    fn = getattr(tps, impl)
+    qd = q.to(DEV)
+    di = torch.from_numpy(np.asarray(idx, np.int32)).to(DEV) if len(idx) else torch.zeros(1, dtype=torch.int32, device=DEV)
+    dc = torch.tensor([len(idx) if count is None else count], dtype=torch.int32, device=DEV)
+    cap = q.shape[0] if cap is None else cap
+    o = torch.full_like(qd, 7.0)
+    lse = torch.full((max(q.shape[0], 1), q.shape[1]), 7.0, device=DEV) if with_lse else None
+    fn(qd, k.to(DEV), v.to(DEV), di, dc, scale, blockmask=None if bm is None else bm.to(DEV),
+       o_act=o, lse=lse, cap=cap)
+    tps.tps_check()
+    return o.cpu(), (lse.cpu().numpy() if with_lse else None)
+
+
+def _check(o_gpu, lse_gpu, o_ref, lse_ref, rows=None):
+    g = o_gpu.double().numpy()
+    if rows is not None:
+        g = g[rows]
+        lse_gpu = None if lse_gpu is None else lse_gpu[rows]
+    ok, info = attn_tolerance_ok(g, o_ref)
+    assert ok, info
+    if lse_gpu is not None:
+        fin = np.isfinite(lse_ref)
+        assert np.array_equal(np.isneginf(lse_gpu), np.isneginf(lse_ref))
+        np.testing.assert_allclose(lse_gpu[fin], lse_ref[fin], rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("N,A,H,d", [(256, 256, 2, 64), (300, 113, 2, 64), (517, 131, 3, 128), (1000, 1, 1, 128),
+                                     (129, 129, 4, 128), (4099, 700, 2, 64), (2000, 1999, 1, 128)])
+@pytest.mark.parametrize("sharp", [False, True])
+def test_attn_random_dense(impl, N, A, H, d, sharp):
+    q = synth.gaussian_bf16((A, H, d), N + A)
+    k = synth.gaussian_bf16((N, H, d), N + A + 1)
+    v = synth.gaussian_bf16((N, H, d), N + A + 2)
+    idx = np.sort(np.random.default_rng(A).choice(N, A, replace=False))
+    scale = (0.35 if sharp else 1.0 / math.sqrt(d))
+    o, lse = _run(impl, q, k, v, idx, scale)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
+    _check(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_attn_constant_keys_mean_of_v(impl):
+    N, H, d = 1500, 2, 128
+    k = synth.gaussian_bf16((1, H, d), 1).expand(N, H, d).contiguous()
+    v = synth.gaussian_bf16((N, H, d), 2)
+    q = synth.gaussian_bf16((200, H, d), 3)
+    o, _ = _run(impl, q, k, v, np.arange(200), 0.2)
+    mean_v = v.double().mean(0).numpy()
+    ok, info = attn_tolerance_ok(o.double().numpy(), np.broadcast_to(mean_v, (200, H, d)))
+    assert ok, info
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("N,A", [(1000, 400), (1100, 1100), (129, 60)])
+def test_attn_blockmask(impl, N, A):
+    H, d = 2, 128
+    q = synth.gaussian_bf16((A, H, d), 10)
+    k = synth.gaussian_bf16((N, H, d), 11)
+    v = synth.gaussian_bf16((N, H, d), 12)
+    idx = np.sort(np.random.default_rng(13).choice(N, A, replace=False))
+    nb = -(-N // 128)
+    bm = torch.from_numpy((np.random.default_rng(14).random((nb, nb)) < 0.35).astype(np.uint8))
+    bm[np.arange(nb), np.arange(nb)] = 1
+    bm[idx[A // 2] // 128] = 0                     # one query block keeps nothing
+    o, lse = _run(impl, q, k, v, idx, 0.3, bm=bm)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 0.3, blockmask=bm)
+    _check(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_attn_count_below_cap_leaves_tail(impl):
+    N, A, H, d = 700, 300, 2, 64
+    q = synth.gaussian_bf16((A, H, d), 20)
+    k = synth.gaussian_bf16((N, H, d), 21)
+    v = synth.gaussian_bf16((N, H, d), 22)
+    idx = np.arange(0, 600, 2)
+    o, lse = _run(impl, q, k, v, idx, 0.125, count=150)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 0.125, rows=np.arange(150))
+    _check(o[:150], lse[:150], o_ref, lse_ref)
+    assert torch.all(o[150:].float() == 7.0) and np.all(lse[150:] == 7.0)
+    o0, _ = _run(impl, q, k, v, idx, 0.125, count=0)
+    assert torch.all(o0.float() == 7.0)
+
+
+# ------------------------------------------------------ whole per-layer path ---
+def _layer(impl, k_cache, v_cache, q_full, k_full, v_full, o_cache, idx_d, cnt_d, cap, scale, bm=None, renoise=None):
+    """gather -> kv_sync -> attention -> scatter on the device."""
+    H, d = q_full.shape[1], q_full.shape[2]
+    q_act = torch.empty((cap, H, d), dtype=torch.bfloat16, device=DEV)
+    k_new = torch.empty_like(q_act)
+    v_new = torch.empty_like(q_act)
+    tps.tps_gather_rows(q_act, q_full, idx_d, cnt_d, cap=cap)
+    tps.tps_gather_rows(k_new, k_full, idx_d, cnt_d, cap=cap)
+    tps.tps_gather_rows(v_new, v_full, idx_d, cnt_d, cap=cap)
+    ke, ve = tps.kv_sync(k_cache, v_cache, k_new, v_new, idx_d, cnt_d, cap=cap, renoise=renoise)
+    kk, vv = (k_cache, v_cache) if renoise is None else (ke, ve)
+    o_act = torch.empty_like(q_act)
+    lse = torch.empty((cap, H), dtype=torch.float32, device=DEV)
+    getattr(tps, impl)(q_act, kk, vv, idx_d, cnt_d, scale, blockmask=bm, o_act=o_act, lse=lse, cap=cap)
+    tps.scatter_out(o_cache, o_act, idx_d, cnt_d, cap=cap)
+    tps.tps_check()
+    return o_act, lse, kk, vv
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_path_tiny_full(impl):
+    """tiny: threshold 0.2 on inter-frame scores, every output row checked."""
+    cfg, xb, _ = frame_case("tiny")
+    Q, K, V = qkv("tiny")
+    N, H, d = Q.shape
+    kc = synth.gaussian_bf16((N, H, d), 90)
+    vc = synth.gaussian_bf16((N, H, d), 91)
+    oc = synth.gaussian_bf16((N, H, d), 92)
+    s = tps.lipar_score(xb.to(DEV))
+    idx_d, cnt_d = tps.lipar_select(s, tps.SELECT_THRESHOLD, tau=cfg.tau)
+    A = int(cnt_d.item())
+    idx = oracle_idx("tiny")
+    assert A == len(idx) and np.array_equal(idx_d[:A].cpu().numpy(), idx)
+    kcd, vcd, ocd = kc.to(DEV), vc.to(DEV), oc.to(DEV)
+    o_act, lse, _, _ = _layer(impl, kcd, vcd, Q.to(DEV), K.to(DEV), V.to(DEV), ocd, idx_d, cnt_d, N, 1 / math.sqrt(d))
+    k2, v2, _, _ = O.kv_sync(kc, vc, K[idx], V[idx], idx)
+    assert torch.equal(kcd.cpu(), k2) and torch.equal(vcd.cpu(), v2)
+    o_ref, lse_ref = O.pruned_attn(Q[idx], k2, v2, idx, 1 / math.sqrt(d))
+    _check(o_act[:A].cpu(), lse[:A].cpu().numpy(), o_ref, lse_ref)
+    out = ocd.cpu()
+    rest = np.setdiff1d(np.arange(N), idx)
+    assert torch.equal(out[rest], oc[rest]) and torch.equal(out[idx], o_act[:A].cpu())
+
+
+def _sample(A, n, seed):
+    r = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, A - 1], r.choice(A, min(n, A), replace=False)]))
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_path_mid_topk_sampled(impl):
+    """mid: top-k 30% of inter-frame scores; cached K/V = previous frame's
+    projection; 384 sampled active rows x all heads vs the oracle."""
+    cfg, xb, k = frame_case("mid")
+    Q, K, V = qkv("mid")
+    N, H, d = Q.shape
+    HW = cfg.video.HW
+    kc = torch.cat([K[:HW], K[:-HW]])            # previous frame's projection
+    vc = torch.cat([V[:HW], V[:-HW]])
+    oc = synth.gaussian_bf16((N, H, d), 93)
+    s = tps.lipar_score(xb.to(DEV))
+    idx_d, cnt_d = tps.lipar_select(s, tps.SELECT_TOPK, k=k)
+    idx = oracle_idx("mid")
+    assert np.array_equal(idx_d[:k].cpu().numpy(), idx)
+    kcd, vcd, ocd = kc.to(DEV), vc.to(DEV), oc.to(DEV)
+    o_act, lse, kk, vv = _layer(impl, kcd, vcd, Q.to(DEV), K.to(DEV), V.to(DEV), ocd, idx_d, cnt_d, k, 1 / math.sqrt(d))
+    k2, v2, _, _ = O.kv_sync(kc, vc, K[idx], V[idx], idx)
+    assert torch.equal(kcd.cpu(), k2) and torch.equal(vcd.cpu(), v2)
+    rows = _sample(k, 384, 1)
+    o_ref, lse_ref = O.pruned_attn(Q[idx], k2, v2, idx, 1 / math.sqrt(d), rows=rows)
+    _check(o_act.cpu(), lse.cpu().numpy(), o_ref, lse_ref, rows=rows)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_wan_keep100_is_dense_sampled(impl):
+    """Wan-like layer at keep 100%: pruned attention == dense attention."""
+    Q, K, V = qkv("wan")
+    N, H, d = Q.shape
+    idx = np.arange(N)
+    o, lse = _run(impl, Q, K, V, idx, 1 / math.sqrt(d))
+    rows = _sample(N, 256, 2)
+    o_ref, lse_ref = O.pruned_attn(Q, K, V, idx, 1 / math.sqrt(d), rows=rows)
+    _check(o, lse, o_ref, lse_ref, rows=rows)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_block_sparse_config_sampled(impl):
+    """block-sparse: 118800 tokens, 40% active queries, 139/929 key blocks
+    kept per query block; sampled rows vs the oracle."""
+    cfg, xb, k = frame_case("block")
+    Q, K, V = qkv("block")
+    N, H, d = Q.shape
+    bm = synth.block_mask_band_random(cfg.video, 128, cfg.extra["kept_per_row"], cfg.video.seed)
+    assert int(bm.sum(1).min()) == int(bm.sum(1).max()) == 139
+    idx = oracle_idx("block")
+    assert len(idx) == 47520
+    o, lse = _run(impl, Q[idx], K, V, idx, 1 / math.sqrt(d), bm=bm)
+    rows = _sample(len(idx), 160, 3)
+    o_ref, lse_ref = O.pruned_attn(Q[idx], K, V, idx, 1 / math.sqrt(d), blockmask=bm, rows=rows)
+    _check(o, lse, o_ref, lse_ref, rows=rows)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_hsa_steps_with_renoise_sampled(impl):
+    """HSA at full size: groups from the inter-step score, per-step active sets
+    (steps 0, 1, 2 give |A| = N, N/3, 2N/3), re-noised pruned rows
+    (a = 1 - sigma, b = sigma). Checked: bit-exact caches and index lists, the
+    re-noised K/V of three heads over all rows, and sampled attention rows of
+    those heads against the oracle's own fp64 K_eff / V_eff."""
+    cfg, vpb, vc, _ = step_case("hsa")
+    F, HW, C = cfg.video.F, cfg.video.HW, cfg.video.C
+    K_, T, budgets = cfg.extra["K"], cfg.extra["T"], cfg.extra["budgets"]
+    Q, Kp, Vp = qkv("hsa")
+    N, H, d = Q.shape
+    heads = np.array([0, 11, 23])
+    s = tps.lipar_score(vc.reshape(F, HW, C).to(DEV), vpb.reshape(F, HW, C).to(DEV))
+    g = tps.lipar_group(s, K_)
+    g_ref = O.group_split(O.lipar_score(vc[None], vpb[None]), K_)
+    assert np.array_equal(g.cpu().numpy(), g_ref)
+    kcd, vcd = Kp.to(DEV), Vp.to(DEV)          # step 0 fills the cache
+    kc, vc_ = Kp.clone(), Vp.clone()
+    ocd = torch.zeros((N, H, d), dtype=torch.bfloat16, device=DEV)
+    Qd, Kd, Vd = Q.to(DEV), Kp.to(DEV), Vp.to(DEV)
+    for step in (0, 1, 2):
+        sigma = 1.0 - step / T
+        idx_d, cnt_d = tps.lipar_schedule(g, K_, budgets, T, step, 0)
+        idx = O.schedule_active(g_ref, K_, budgets, T, step, 0)
+        A = int(cnt_d.item())
+        assert A == len(idx) and np.array_equal(idx_d[:A].cpu().numpy(), idx)
+        rn = (1.0 - sigma, sigma, cfg.video.seed, step)
+        o_act, lse, ke, ve = _layer(impl, kcd, vcd, Qd, Kd, Vd, ocd, idx_d, cnt_d, A, 1 / math.sqrt(d), renoise=rn)
+        kc, vc_, ke_ref, ve_ref = O.kv_sync(kc, vc_, Kp[idx], Vp[idx], idx, renoise=rn, heads=heads)
+        assert torch.equal(kcd.cpu(), kc) and torch.equal(vcd.cpu(), vc_)
+        for got, ref in ((ke, ke_ref), (ve, ve_ref)):
+            err = np.abs(got[:, torch.from_numpy(heads)].cpu().double().numpy() - ref)
+            ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+            assert np.all(err <= ulp + 1e-5 * sigma + 1e-30)
+        rows = _sample(A, 48, step)
+        o_ref, lse_ref = O.pruned_attn(Q[idx][:, torch.from_numpy(heads)], ke_ref, ve_ref, idx,
+                                       1 / math.sqrt(d), rows=rows)
+        _check(o_act[:, torch.from_numpy(heads)].cpu(), lse[:, torch.from_numpy(heads)].cpu().numpy(),
+               o_ref, lse_ref, rows=rows)

@@ -1,0 +1,110 @@
+"""GPU parity: kv_sync (plain and re-noised), scatter_out, tps_gather_rows and
+the raw Philox stream vs the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from token_pruned_sparse_b200 import synth
+from token_pruned_sparse_b200 import tps
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _case(N, H, d, A, seed):
+    kc = synth.gaussian_bf16((N, H, d), seed)
+    vc = synth.gaussian_bf16((N, H, d), seed + 1)
+    kf = synth.gaussian_bf16((max(A, 1), H, d), seed + 2)[:A]
+    vf = synth.gaussian_bf16((max(A, 1), H, d), seed + 3)[:A]
+    idx = np.sort(np.random.default_rng(seed).choice(N, A, replace=False)).astype(np.int32)
+    return kc, vc, kf, vf, idx
+
+
+def _dev_idx(idx, cap=None):
+    cap = len(idx) if cap is None else cap
+    buf = torch.zeros(max(cap, 1), dtype=torch.int32)
+    buf[: len(idx)] = torch.from_numpy(idx)
+    return buf.to(DEV), torch.tensor([len(idx)], dtype=torch.int32, device=DEV)
+
+
+@pytest.mark.parametrize("N,H,d,A", [(256, 2, 64, 100), (1000, 3, 128, 1000), (20280, 12, 128, 6084),
+                                     (517, 24, 128, 0), (9, 1, 64, 1)])
+def test_kv_sync_plain_bit_exact(N, H, d, A):
+    kc, vc, kf, vf, idx = _case(N, H, d, A, N + A)
+    kcd, vcd = kc.to(DEV), vc.to(DEV)
+    di, dc = _dev_idx(idx)
+    kfd = kf.to(DEV) if A else torch.empty((1, H, d), dtype=torch.bfloat16, device=DEV)
+    vfd = vf.to(DEV) if A else torch.empty((1, H, d), dtype=torch.bfloat16, device=DEV)
+    tps.kv_sync(kcd, vcd, kfd, vfd, di, dc, cap=A)
+    k2, v2, _, _ = O.kv_sync(kc, vc, kf, vf, idx)
+    assert torch.equal(kcd.cpu(), k2) and torch.equal(vcd.cpu(), v2)
+    tps.tps_check()
+
+
+def _renoise_tol(ref, b):
+    # one bf16 rounding of the result (half an ulp each side, so one ulp of
+    # slack) plus the fp32 Box-Muller error (|z| <= 6, log/sincos ~1e-6 abs)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+    return ulp + abs(b) * 1e-5 + 1e-30
+
+
+@pytest.mark.parametrize("N,H,d,A,a,b", [(256, 2, 64, 100, 0.3, 0.7), (3001, 3, 128, 1234, 0.9, 0.1),
+                                         (5000, 24, 128, 5000, 0.5, 0.5), (777, 4, 64, 0, 0.0, 1.0),
+                                         (777, 4, 64, 300, 1.0, 0.0)])
+def test_kv_sync_renoise(N, H, d, A, a, b):
+    kc, vc, kf, vf, idx = _case(N, H, d, A, 3 * N + A)
+    kcd, vcd = kc.to(DEV), vc.to(DEV)
+    di, dc = _dev_idx(idx)
+    kfd = kf.to(DEV) if A else torch.empty((1, H, d), dtype=torch.bfloat16, device=DEV)
+    vfd = vf.to(DEV) if A else torch.empty((1, H, d), dtype=torch.bfloat16, device=DEV)
+    seed, step = 0x123456789ABC, 17
+    ke, ve = tps.kv_sync(kcd, vcd, kfd, vfd, di, dc, cap=A, renoise=(a, b, seed, step))
+    k2, v2, ke_ref, ve_ref = O.kv_sync(kc, vc, kf, vf, idx, renoise=(a, b, seed, step))
+    assert torch.equal(kcd.cpu(), k2) and torch.equal(vcd.cpu(), v2)       # cache: bit copies only
+    for got, ref in ((ke, ke_ref), (ve, ve_ref)):
+        g = got.cpu().double().numpy()
+        assert np.array_equal(g[idx], ref[idx])                             # active rows: fresh, exact
+        err = np.abs(g - ref)
+        assert np.all(err <= _renoise_tol(ref, b)), float(err.max())
+    if a == 1.0 and b == 0.0:
+        assert torch.equal(ke.cpu(), k2) and torch.equal(ve.cpu(), v2)
+    tps.tps_check()
+
+
+def test_philox_stream_bit_exact():
+    for seed, step, t, q0 in ((0, 0, 0, 0), (0xFFFFFFFFFFFFFFFF, 39, 1, 2 ** 32 - 5), (42, 7, 0, 123456789)):
+        got = tps.tps_philox_fill(q0, 4099, seed, step, t).cpu().numpy().view(np.uint32).reshape(-1, 4)
+        ref = O.philox_words(seed, step, t, np.arange(q0, q0 + 4099, dtype=np.uint64))
+        assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("N,H,d,A", [(256, 2, 64, 100), (20280, 12, 128, 6084), (1000, 1, 64, 0), (130, 24, 128, 130)])
+def test_scatter_and_gather_bit_exact(N, H, d, A):
+    full = synth.gaussian_bf16((N, H, d), N)
+    act = synth.gaussian_bf16((max(A, 1), H, d), N + 1)[:max(A, 1)]
+    idx = np.sort(np.random.default_rng(A).choice(N, A, replace=False)).astype(np.int32)
+    di, dc = _dev_idx(idx)
+    fd = full.to(DEV)
+    tps.scatter_out(fd, act.to(DEV), di, dc, cap=A)
+    assert torch.equal(fd.cpu(), O.scatter_out(full, act[:A], idx))
+    g = torch.empty((max(A, 1), H, d), dtype=torch.bfloat16, device=DEV)
+    tps.tps_gather_rows(g, fd, di, dc, cap=A)
+    assert torch.equal(g[:A].cpu(), O.gather_rows(fd.cpu(), idx))
+    tps.tps_check()
+
+
+def test_count_below_cap_and_bounds_flag():
+    N, H, d = 100, 2, 64
+    full = synth.gaussian_bf16((N, H, d), 5)
+    act = synth.gaussian_bf16((10, H, d), 6)
+    idx = torch.tensor([1, 5, 9, 200, 11, 0, 0, 0, 0, 0], dtype=torch.int32)   # 200 is out of range
+    fd = full.to(DEV)
+    cnt = torch.tensor([5], dtype=torch.int32, device=DEV)
+    tps.scatter_out(fd, act.to(DEV), idx.to(DEV), cnt, cap=10)
+    with pytest.raises(tps.TPSError) as e:
+        tps.tps_check()
+    assert e.value.code == tps.BOUNDS
+    ref = O.scatter_out(full, act[[0, 1, 2, 4]], np.array([1, 5, 9, 11]))
+    assert torch.equal(fd.cpu(), ref)
+    tps.tps_check()                                                         # flag was cleared

@@ -1,0 +1,510 @@
+// Active-set selection and stream compaction:
+//   lipar_select   (threshold / top-k)     [LIPAR] 2.B: a token whose change is
+//                                          below tau is redundant and pruned.
+//   lipar_group    (HSA rank split)        [HSA] 2.1: tokens partitioned into K
+//                                          groups by relative-L1 velocity change.
+//   lipar_schedule (HSA per-step set)      [HSA] 2.1: group k active iff
+//                                          i mod (T/s_k) == 0; 2.4: first/last
+//                                          m steps run every token.
+//
+// Design (HBM/latency-bound, N ~ 1e4..1e6):
+//   * Scores map to order-preserving uint32 keys (NaN lowest, -0 == +0).
+//   * Top-k / rank cuts use an MSB-first radix select, 8-bit digits, one
+//     launch per digit. Each block builds a shared-memory histogram and adds it
+//     to a global one; the last block to finish (atomic ticket, no spinning)
+//     picks the digit bucket and resets the histogram for the next pass. After
+//     four passes the exact k-th key K* and the number of ties at K* still to
+//     take (krem) are known.
+//   * Compaction: a count kernel writes per-block counts and its last block
+//     turns them into exclusive offsets (and the device-side total); a write
+//     kernel recomputes each element's class, ranks it with warp ballots and
+//     popc, and writes the ascending index list. Ties at K* are taken in index
+//     order, so the result is unique.
+#include "tps_internal.cuh"
+
+namespace tps {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kItems = 4;
+constexpr int kTile = kThreads * kItems;  // elements per compaction block
+constexpr int kMaxBound = 7;              // rank cuts (K <= 8 groups)
+
+struct SelHdr {
+  unsigned int ticket;     // last-block ticket of the count kernels
+  unsigned int ticket_r;   // last-block ticket of the radix passes
+  unsigned int pad[2];
+  unsigned int prefix[8];  // radix prefix, finally K*, per cut
+  unsigned int krem[8];    // ties at K* still to take, per cut
+  unsigned int hist[kMaxBound][256];
+};
+constexpr size_t kHdrBytes = (sizeof(SelHdr) + 255) / 256 * 256;
+
+struct Cuts {
+  unsigned int k[kMaxBound];
+};
+
+inline int64_t n_blocks(int64_t N) { return (N + kTile - 1) / kTile; }
+
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  if ((b & 0x7fffffffu) > 0x7f800000u) return 0u;  // NaN ranks below everything
+  if (b == 0x80000000u) b = 0u;                    // -0 equals +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Inclusive scan of one value per thread over the 256-thread block.
+__device__ __forceinline__ unsigned int block_incl_scan(unsigned int v, unsigned int* total) {
+  __shared__ unsigned int wsum[kWarps];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[w] = x;
+  __syncthreads();
+  unsigned int add = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) {
+    const unsigned int s = wsum[i];
+    add += (i < w) ? s : 0u;
+    tot += s;
+  }
+  __syncthreads();
+  *total = tot;
+  return x + add;
+}
+
+__device__ __forceinline__ unsigned int block_sum(unsigned int v) {
+  unsigned int tot;
+  block_incl_scan(v, &tot);
+  return tot;
+}
+
+// True in every thread of the block that finished last (after all others
+// published their results with a fence). No thread ever waits on another block.
+__device__ __forceinline__ bool last_block(unsigned int* ticket) {
+  __shared__ bool s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (s_last) __threadfence();
+  return s_last;
+}
+
+// ---- radix select -------------------------------------------------------------
+__global__ void sel_init(SelHdr* h, int nbound, Cuts cuts) {
+  for (int i = threadIdx.x; i < kMaxBound * 256; i += blockDim.x) (&h->hist[0][0])[i] = 0u;
+  if (threadIdx.x < 8) {
+    h->prefix[threadIdx.x] = 0u;
+    h->krem[threadIdx.x] = threadIdx.x < nbound ? cuts.k[threadIdx.x] : 0u;
+  }
+  if (threadIdx.x == 0) {
+    h->ticket = 0u;
+    h->ticket_r = 0u;
+  }
+}
+
+// One 8-bit digit (bits [shift, shift+8)) for every cut at once.
+__global__ void __launch_bounds__(kThreads) radix_pass(const float* __restrict__ s, int64_t N,
+                                                       SelHdr* h, int nbound, int shift) {
+  __shared__ unsigned int sh[kMaxBound][256];
+  for (int i = threadIdx.x; i < nbound * 256; i += kThreads) (&sh[0][0])[i] = 0u;
+  const unsigned int himask = shift >= 24 ? 0u : (0xffffffffu << (shift + 8));
+  unsigned int pre[kMaxBound];
+#pragma unroll
+  for (int b = 0; b < kMaxBound; ++b) pre[b] = b < nbound ? h->prefix[b] : 0u;
+  __syncthreads();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; n < N; n += stride) {
+    const unsigned int key = score_key(s[n]);
+    const unsigned int dig = (key >> shift) & 255u;
+#pragma unroll
+    for (int b = 0; b < kMaxBound; ++b)
+      if (b < nbound && (key & himask) == pre[b]) atomicAdd(&sh[b][dig], 1u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nbound * 256; i += kThreads) {
+    const unsigned int v = (&sh[0][0])[i];
+    if (v) atomicAdd(&(&h->hist[0][0])[i], v);
+  }
+  if (!last_block(&h->ticket_r)) return;
+  // Last block: for each cut, thread t looks at bucket 255 - t (descending).
+  for (int b = 0; b < nbound; ++b) {
+    const unsigned int need = __ldcg(&h->krem[b]);
+    const int bin = 255 - threadIdx.x;
+    const unsigned int c = __ldcg(&h->hist[b][bin]);
+    unsigned int tot;
+    const unsigned int incl = block_incl_scan(c, &tot);
+    const unsigned int excl = incl - c;
+    if (need > 0 && excl < need && incl >= need) {
+      h->prefix[b] = pre[b] | (static_cast<unsigned int>(bin) << shift);
+      h->krem[b] = need - excl;
+    }
+    h->hist[b][bin] = 0u;
+  }
+  if (threadIdx.x == 0) h->ticket_r = 0u;
+}
+
+// ---- element classes ----------------------------------------------------------
+// 0 = not selected, 1 = selected, 2 = tie at K* (selected in index order while
+// fewer than krem ties have been taken).
+struct ThreshCls {
+  const float* s;
+  float tau;
+  __device__ __forceinline__ int operator()(int64_t n, const SelHdr*) const {
+    return s[n] >= tau ? 1 : 0;
+  }
+};
+struct TopkCls {
+  const float* s;
+  __device__ __forceinline__ int operator()(int64_t n, const SelHdr* h) const {
+    const unsigned int key = score_key(s[n]);
+    const unsigned int ks = h->prefix[0];
+    return key > ks ? 1 : (key == ks ? 2 : 0);
+  }
+};
+struct SchedCls {
+  const int8_t* g;
+  unsigned int act;  // bit k set: group k active this step
+  int K;
+  __device__ __forceinline__ int operator()(int64_t n, const SelHdr*) const {
+    const int v = g[n];
+    return (v >= 0 && v < K && ((act >> v) & 1u)) ? 1 : 0;
+  }
+};
+
+// Per-block counts (column 0: selected, column 1: ties), then in the last
+// block: exclusive offsets per column and the device-side total.
+template <class Cls>
+__global__ void __launch_bounds__(kThreads) compact_count(Cls cls, int64_t N, SelHdr* h,
+                                                          unsigned int* cnt, unsigned int* off,
+                                                          int ncol, int32_t* count_out) {
+  const int64_t nb = gridDim.x;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTile;
+  unsigned int sel = 0, tie = 0;
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * kThreads + threadIdx.x;
+    if (n < N) {
+      const int c = cls(n, h);
+      sel += c == 1;
+      tie += c == 2;
+    }
+  }
+  sel = block_sum(sel);
+  if (ncol > 1) tie = block_sum(tie);
+  if (threadIdx.x == 0) {
+    cnt[blockIdx.x] = sel;
+    if (ncol > 1) cnt[nb + blockIdx.x] = tie;
+  }
+  if (!last_block(&h->ticket)) return;
+  unsigned int totals[2] = {0u, 0u};
+  for (int col = 0; col < ncol; ++col) {
+    unsigned int run = 0;
+    for (int64_t i0 = 0; i0 < nb; i0 += kThreads) {
+      const int64_t i = i0 + threadIdx.x;
+      const unsigned int v = i < nb ? __ldcg(&cnt[col * nb + i]) : 0u;
+      unsigned int tot;
+      const unsigned int incl = block_incl_scan(v, &tot);
+      if (i < nb) off[col * nb + i] = run + incl - v;
+      run += tot;
+    }
+    totals[col] = run;
+  }
+  if (threadIdx.x == 0) {
+    unsigned int total = totals[0];
+    if (ncol > 1) {
+      const unsigned int kr = __ldcg(&h->krem[0]);
+      total += totals[1] < kr ? totals[1] : kr;
+    }
+    if (count_out) *count_out = static_cast<int32_t>(total);
+    h->ticket = 0u;
+  }
+}
+
+template <class Cls>
+__global__ void __launch_bounds__(kThreads) compact_write(Cls cls, int64_t N, const SelHdr* h,
+                                                          const unsigned int* off, int ncol,
+                                                          int32_t* __restrict__ idx) {
+  __shared__ unsigned int s_sel[kWarps], s_tie[kWarps];
+  const int64_t nb = gridDim.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTile + w * (32 * kItems);
+  unsigned int msel[kItems], mtie[kItems];
+  unsigned int wsel = 0, wtie = 0;
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    const int c = n < N ? cls(n, h) : 0;
+    msel[it] = __ballot_sync(0xffffffffu, c == 1);
+    mtie[it] = __ballot_sync(0xffffffffu, c == 2);
+    wsel += __popc(msel[it]);
+    wtie += __popc(mtie[it]);
+  }
+  if (lane == 0) {
+    s_sel[w] = wsel;
+    s_tie[w] = wtie;
+  }
+  __syncthreads();
+  unsigned int sb = off[blockIdx.x], tb = ncol > 1 ? off[nb + blockIdx.x] : 0u;
+  for (int i = 0; i < w; ++i) {
+    sb += s_sel[i];
+    tb += s_tie[i];
+  }
+  const unsigned int krem = ncol > 1 ? h->krem[0] : 0u;
+  const unsigned int lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    const unsigned int sr = sb + __popc(msel[it] & lt);
+    const unsigned int tr = tb + __popc(mtie[it] & lt);
+    if ((msel[it] >> lane) & 1u) idx[sr + (tr < krem ? tr : krem)] = static_cast<int32_t>(n);
+    else if (((mtie[it] >> lane) & 1u) && tr < krem) idx[sr + tr] = static_cast<int32_t>(n);
+    sb += __popc(msel[it]);
+    tb += __popc(mtie[it]);
+  }
+}
+
+// ---- HSA group split -----------------------------------------------------------
+// Per-block tie counts for every cut; the last block turns them into offsets.
+__global__ void __launch_bounds__(kThreads) group_count(const float* __restrict__ s, int64_t N,
+                                                        SelHdr* h, int nbound, unsigned int* cnt,
+                                                        unsigned int* off) {
+  const int64_t nb = gridDim.x;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTile;
+  unsigned int ks[kMaxBound];
+  unsigned int eq[kMaxBound];
+#pragma unroll
+  for (int b = 0; b < kMaxBound; ++b) {
+    ks[b] = b < nbound ? h->prefix[b] : 0u;
+    eq[b] = 0u;
+  }
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * kThreads + threadIdx.x;
+    if (n < N) {
+      const unsigned int key = score_key(s[n]);
+#pragma unroll
+      for (int b = 0; b < kMaxBound; ++b) eq[b] += (b < nbound && key == ks[b]) ? 1u : 0u;
+    }
+  }
+  for (int b = 0; b < nbound; ++b) {
+    const unsigned int t = block_sum(eq[b]);
+    if (threadIdx.x == 0) cnt[b * nb + blockIdx.x] = t;
+  }
+  if (!last_block(&h->ticket)) return;
+  for (int b = 0; b < nbound; ++b) {
+    unsigned int run = 0;
+    for (int64_t i0 = 0; i0 < nb; i0 += kThreads) {
+      const int64_t i = i0 + threadIdx.x;
+      const unsigned int v = i < nb ? __ldcg(&cnt[b * nb + i]) : 0u;
+      unsigned int tot;
+      const unsigned int incl = block_incl_scan(v, &tot);
+      if (i < nb) off[b * nb + i] = run + incl - v;
+      run += tot;
+    }
+  }
+  if (threadIdx.x == 0) h->ticket = 0u;
+}
+
+// group[n] = number of cuts the token does not make it above.
+__global__ void __launch_bounds__(kThreads) group_write(const float* __restrict__ s, int64_t N,
+                                                        const SelHdr* h, int nbound,
+                                                        const unsigned int* off,
+                                                        int8_t* __restrict__ group) {
+  __shared__ unsigned int s_eq[kMaxBound][kWarps];
+  const int64_t nb = gridDim.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTile + w * (32 * kItems);
+  unsigned int key[kItems];
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    key[it] = n < N ? score_key(s[n]) : 0u;
+  }
+  int grp[kItems] = {0, 0, 0, 0};
+  const unsigned int lt = (1u << lane) - 1u;
+  for (int b = 0; b < nbound; ++b) {
+    const unsigned int ks = h->prefix[b];
+    const unsigned int kr = h->krem[b];
+    unsigned int m[kItems];
+    unsigned int weq = 0;
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int64_t n = base + it * 32 + lane;
+      m[it] = __ballot_sync(0xffffffffu, n < N && key[it] == ks);
+      weq += __popc(m[it]);
+    }
+    if (lane == 0) s_eq[b][w] = weq;
+    __syncthreads();
+    unsigned int eb = off[b * nb + blockIdx.x];
+    for (int i = 0; i < w; ++i) eb += s_eq[b][i];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const unsigned int r = eb + __popc(m[it] & lt);
+      const bool above = key[it] > ks || (key[it] == ks && r < kr);
+      grp[it] += above ? 0 : 1;
+      eb += __popc(m[it]);
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    if (n < N) group[n] = static_cast<int8_t>(grp[it]);
+  }
+}
+
+// ---- host helpers ------------------------------------------------------------------
+struct WsView {
+  SelHdr* hdr;
+  unsigned int* cnt;
+  unsigned int* off;
+};
+
+inline int ncols_for(int op, int K) {
+  if (op == TPS_OP_SELECT) return 2;
+  if (op == TPS_OP_GROUP) return K > 1 ? K - 1 : 1;
+  return 1;
+}
+
+size_t ws_bytes_for(int op, int64_t N, int K) {
+  const int64_t nb = n_blocks(N > 0 ? N : 1);
+  return kHdrBytes + 2 * static_cast<size_t>(ncols_for(op, K)) * nb * sizeof(unsigned int);
+}
+
+int check_ws(void* ws, size_t bytes, int op, int64_t N, int K, WsView* v, const char* who) {
+  if (!ws) return fail(TPS_ERR_WORKSPACE, "%s: workspace is null", who);
+  if (!aligned16(ws)) return fail(TPS_ERR_ALIGN, "%s: workspace must be 16-byte aligned", who);
+  const size_t need = ws_bytes_for(op, N, K);
+  if (bytes < need)
+    return fail(TPS_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", who, bytes, need);
+  const int64_t nb = n_blocks(N);
+  v->hdr = static_cast<SelHdr*>(ws);
+  v->cnt = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + kHdrBytes);
+  v->off = v->cnt + static_cast<size_t>(ncols_for(op, K)) * nb;
+  return TPS_OK;
+}
+
+unsigned int radix_grid(int64_t N) {
+  int64_t g = (N + 4 * kThreads - 1) / (4 * kThreads);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 4;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<unsigned int>(g);
+}
+
+int run_radix(const float* s, int64_t N, SelHdr* h, int nbound, const Cuts& cuts, cudaStream_t st) {
+  sel_init<<<1, kThreads, 0, st>>>(h, nbound, cuts);
+  const unsigned int g = radix_grid(N);
+  for (int shift = 24; shift >= 0; shift -= 8) radix_pass<<<g, kThreads, 0, st>>>(s, N, h, nbound, shift);
+  return launch_status("radix select");
+}
+
+template <class Cls>
+int run_compact(const Cls& cls, int64_t N, const WsView& v, int ncol, int32_t* idx, int32_t* count,
+                cudaStream_t st, bool need_init) {
+  if (need_init) sel_init<<<1, kThreads, 0, st>>>(v.hdr, 0, Cuts{});
+  const unsigned int nb = static_cast<unsigned int>(n_blocks(N));
+  compact_count<Cls><<<nb, kThreads, 0, st>>>(cls, N, v.hdr, v.cnt, v.off, ncol, count);
+  compact_write<Cls><<<nb, kThreads, 0, st>>>(cls, N, v.hdr, v.off, ncol, idx);
+  return launch_status("compaction");
+}
+
+}  // namespace
+}  // namespace tps
+
+extern "C" size_t tps_workspace_size(int op, int64_t N, int K) {
+  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
+  if (N < 0) return 0;
+  return tps::ws_bytes_for(op, N, K);
+}
+
+extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
+                            int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                            tps_stream stream) {
+  using namespace tps;
+  if (mode != TPS_SELECT_THRESHOLD && mode != TPS_SELECT_TOPK)
+    return fail(TPS_ERR_INVALID_ARG, "lipar_select: mode %d is not 0 (threshold) or 1 (top-k)", mode);
+  if (!count) return fail(TPS_ERR_INVALID_ARG, "lipar_select: count must be non-null");
+  if (N < 0 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "lipar_select: N=%lld out of [0, 2^31)", (long long)N);
+  if (mode == TPS_SELECT_TOPK && (k < 0 || k > N))
+    return fail(TPS_ERR_INVALID_ARG, "lipar_select: k=%lld not in [0, N=%lld]", (long long)k, (long long)N);
+  if (N > 0 && (!score || !idx)) return fail(TPS_ERR_INVALID_ARG, "lipar_select: score and idx must be non-null");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (N == 0 || (mode == TPS_SELECT_TOPK && k == 0)) {
+    if (int e = cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), st), "lipar_select: clear count")) return e;
+    return ok();
+  }
+  WsView v;
+  if (int e = check_ws(ws, ws_bytes, TPS_OP_SELECT, N, 0, &v, "lipar_select")) return e;
+  int e;
+  if (mode == TPS_SELECT_THRESHOLD) {
+    e = run_compact(ThreshCls{score, tau}, N, v, 1, idx, count, st, true);
+  } else {
+    Cuts c{};
+    c.k[0] = static_cast<unsigned int>(k);
+    if ((e = run_radix(score, N, v.hdr, 1, c, st))) return e;
+    e = run_compact(TopkCls{score}, N, v, 2, idx, count, st, false);
+  }
+  return e ? e : ok();
+}
+
+extern "C" int lipar_group(const float* score, int64_t N, int K, int8_t* group, void* ws,
+                           size_t ws_bytes, tps_stream stream) {
+  using namespace tps;
+  if (!score || !group) return fail(TPS_ERR_INVALID_ARG, "lipar_group: score and group must be non-null");
+  if (N < 1 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "lipar_group: N=%lld out of [1, 2^31)", (long long)N);
+  if (K < 1 || K > kMaxBound + 1 || K > N)
+    return fail(TPS_ERR_INVALID_ARG, "lipar_group: K=%d must be in [1, 8] and <= N", K);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (K == 1) {
+    if (int e = cuda_status(cudaMemsetAsync(group, 0, static_cast<size_t>(N), st), "lipar_group: fill")) return e;
+    return ok();
+  }
+  WsView v;
+  if (int e = check_ws(ws, ws_bytes, TPS_OP_GROUP, N, K, &v, "lipar_group")) return e;
+  const int nbound = K - 1;
+  Cuts c{};
+  const int64_t size = N / K;
+  for (int b = 0; b < nbound; ++b) c.k[b] = static_cast<unsigned int>((b + 1) * size);
+  if (int e = run_radix(score, N, v.hdr, nbound, c, st)) return e;
+  const unsigned int nb = static_cast<unsigned int>(n_blocks(N));
+  group_count<<<nb, kThreads, 0, st>>>(score, N, v.hdr, nbound, v.cnt, v.off);
+  group_write<<<nb, kThreads, 0, st>>>(score, N, v.hdr, nbound, v.off, group);
+  if (int e = launch_status("lipar_group")) return e;
+  return ok();
+}
+
+extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32_t* budgets, int T,
+                              int step, int m, int32_t* idx, int32_t* count, void* ws,
+                              size_t ws_bytes, tps_stream stream) {
+  using namespace tps;
+  if (!count || !budgets) return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: count and budgets must be non-null");
+  if (N < 0 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "lipar_schedule: N=%lld out of [0, 2^31)", (long long)N);
+  if (K < 1 || K > 8) return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: K=%d must be in [1, 8]", K);
+  if (T < 1 || step < 0 || step >= T || m < 0)
+    return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: need T >= 1, 0 <= step < T, m >= 0");
+  unsigned int act = 0;
+  for (int g = 0; g < K; ++g) {
+    const int s = budgets[g];
+    if (s < 1 || s > T || T % s)
+      return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: budget[%d]=%d must divide T=%d", g, s, T);
+    const bool full = step < m || step >= T - m;
+    if (full || step % (T / s) == 0) act |= 1u << g;
+  }
+  if (N > 0 && (!group || !idx)) return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: group and idx must be non-null");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    if (int e = cuda_status(cudaMemsetAsync(count, 0, sizeof(int32_t), st), "lipar_schedule: clear count")) return e;
+    return ok();
+  }
+  WsView v;
+  if (int e = check_ws(ws, ws_bytes, TPS_OP_SCHEDULE, N, K, &v, "lipar_schedule")) return e;
+  if (int e = run_compact(SchedCls{group, act, K}, N, v, 1, idx, count, st, true)) return e;
+  return ok();
+}
