@@ -324,6 +324,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--attn", choices=["tc", "mma"], default="tc", help="attention kernel (mma = legacy baseline)")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--oracle-rows", type=int, default=256)
     a = ap.parse_args()
@@ -379,7 +380,7 @@ def main():
     tok_s = world * st.k * a.steps / (total_ms * 1e-3)
 
     # ---- end to end through the public API: pinned host inputs -> result on host
-    e2e = e2e_leg(st, dev, max(3, min(a.steps, 50)), world)
+    e2e = None if a.no_e2e else e2e_leg(st, dev, max(3, min(a.steps, 50)), world)
 
     sweep = None if a.no_sweep else keep_sweep(dev, a.attn)
     pk, pk_kind = peaks()
