@@ -97,6 +97,21 @@ TPS_API int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16
 TPS_API int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
                  int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, tps_stream stream);
 
+/* Allocation-free variant of lipar_select (the pages have no counterpart; it
+ * exists for callers that cannot allocate a workspace, e.g. a host running the
+ * step inside a fixed device-memory plan, or a denoising loop that must not
+ * call cudaMalloc because it synchronises the device). Same contract as
+ * lipar_select, but the selection scratch is a file-scope device array inside
+ * libtps.so sized for N <= 4,194,304 tokens (about 73 KB, held by every GPU
+ * that loads the library until exit); larger N returns TPS_ERR_SHAPE. It
+ * allocates nothing. The first call on each device looks up the array's
+ * device address (with that device current), so make that first call before
+ * any stream capture. All calls on a device share the one array: calls that
+ * overlap on the GPU (e.g. on two streams without ordering) race; the scratch
+ * keeps the last call's contents and is re-initialised by every call. */
+TPS_API int lipar_select_static(const float* score, int64_t N, int mode, float tau, int64_t k,
+                                int32_t* idx, int32_t* count, tps_stream stream);
+
 /* ---- HSA group assignment ([HSA] 2.1, dynamic token selection) -------------
  * Ranks tokens by score descending (ties to the lower index, NaN last) and
  * splits the ranks into K contiguous groups of N/K (the remainder joins the

@@ -20,6 +20,8 @@
 //     kernel recomputes each element's class, ranks it with warp ballots and
 //     popc, and writes the ascending index list. Ties at K* are taken in index
 //     order, so the result is unique.
+#include <mutex>
+
 #include "tps_internal.cuh"
 
 namespace tps {
@@ -507,4 +509,53 @@ extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32
   if (int e = check_ws(ws, ws_bytes, TPS_OP_SCHEDULE, N, K, &v, "lipar_schedule")) return e;
   if (int e = run_compact(SchedCls{group, act, K}, N, v, 1, idx, count, st, true)) return e;
   return ok();
+}
+
+// ---- allocation-free variant of lipar_select ------------------------------------------
+// Some callers cannot hand the library a workspace: a C host that runs the
+// step inside a fixed device-memory plan (every buffer owned by the model
+// runtime, none spare), or a latency-critical denoising loop that must not call
+// cudaMalloc, which synchronises the device. For them the selection scratch
+// lives in a file-scope device array sized for at most kStaticMaxN tokens.
+// Every GPU that loads the library holds this array (about 73 KB) until the
+// process exits.
+namespace tps {
+namespace {
+constexpr int64_t kStaticMaxN = INT64_C(1) << 22;   // 4,194,304 tokens
+constexpr size_t kStaticBytes =
+    kHdrBytes + 2 * 2 * static_cast<size_t>((kStaticMaxN + kTile - 1) / kTile) * sizeof(unsigned int);
+static __device__ __align__(256) unsigned char g_select_scratch[kStaticBytes];
+
+// Device address of g_select_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+int static_scratch(void** out) {
+  static void* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "lipar_select_static: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(TPS_ERR_CUDA, "lipar_select_static: device %d out of range", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "lipar_select_static: cudaGetSymbolAddress");
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return TPS_OK;
+}
+}  // namespace
+}  // namespace tps
+
+extern "C" int lipar_select_static(const float* score, int64_t N, int mode, float tau, int64_t k,
+                                   int32_t* idx, int32_t* count, tps_stream stream) {
+  using namespace tps;
+  if (N > kStaticMaxN)
+    return fail(TPS_ERR_SHAPE, "lipar_select_static: N=%lld exceeds the static scratch limit of %lld tokens "
+                "(use lipar_select with a caller-provided workspace)", (long long)N, (long long)kStaticMaxN);
+  void* ws = nullptr;
+  if (int e = static_scratch(&ws)) return e;
+  return lipar_select(score, N, mode, tau, k, idx, count, ws, kStaticBytes, stream);
 }

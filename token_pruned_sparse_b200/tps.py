@@ -28,6 +28,7 @@ _INT = C.c_int
 SIGNATURES = {
     "lipar_score": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "lipar_select": (_INT, [_P, _I64, _INT, C.c_float, _I64, _P, _P, _P, C.c_size_t, _P]),
+    "lipar_select_static": (_INT, [_P, _I64, _INT, C.c_float, _I64, _P, _P, _P]),
     "lipar_group": (_INT, [_P, _I64, _INT, _P, _P, C.c_size_t, _P]),
     "lipar_schedule": (_INT, [_P, _I64, _INT, _P, _INT, _INT, _INT, _P, _P, _P, C.c_size_t, _P]),
     "tps_gather_rows": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -117,6 +118,19 @@ def lipar_select(score, mode, tau=0.0, k=0, idx=None, count=None, ws=None, strea
         ws = workspace(OP_SELECT, N, 0, score.device)
     _chk(lib().lipar_select(_ptr(score), N, mode, float(tau), int(k), _ptr(idx), _ptr(count),
                             _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, count
+
+
+def lipar_select_static(score, mode, tau=0.0, k=0, idx=None, count=None, stream=None):
+    """lipar_select without a workspace: the library's own static scratch
+    (N <= 4,194,304; calls on one device must not overlap on the GPU)."""
+    N = score.numel()
+    if idx is None:
+        idx = torch.empty(max(N if mode == SELECT_THRESHOLD else k, 1), dtype=torch.int32, device=score.device)
+    if count is None:
+        count = torch.empty(1, dtype=torch.int32, device=score.device)
+    _chk(lib().lipar_select_static(_ptr(score), N, mode, float(tau), int(k), _ptr(idx), _ptr(count),
+                                   _stream(stream)))
     return idx, count
 
 
