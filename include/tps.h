@@ -175,6 +175,7 @@ TPS_API int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_fres
  *   blockmask NULL (dense) or uint8 [nb, nb] (block must be 128, nb <= 4096).
  *   lse    NULL or float32 [cap, H]: natural-log sum of exp of the scaled
  *          logits. A row with no allowed key gets o = 0 and lse = -inf.
+ * scale must be finite and > 0 (typically 1/sqrt(d)).
  * bf16 inputs, fp32 accumulation and softmax, tcgen05 tensor cores.
  * d in {64, 128}; 1 <= H <= 256; N < 2^31; pointers 16-byte aligned. */
 TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,

@@ -32,7 +32,7 @@ inline int attn_validate(const char* who, const tps_bf16* q_act, const tps_bf16*
   if (H < 1 || H > 256) return fail(TPS_ERR_SHAPE, "%s: H=%d must be in [1, 256]", who, H);
   if (N < 1 || N >= (INT64_C(1) << 31) || cap < 0 || cap >= (INT64_C(1) << 31))
     return fail(TPS_ERR_SHAPE, "%s: need 1 <= N < 2^31 and 0 <= cap < 2^31", who);
-  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return fail(TPS_ERR_INVALID_ARG, "%s: scale must be finite", who);
+  if (!(scale > 0.f) || scale == INFINITY) return fail(TPS_ERR_INVALID_ARG, "%s: scale must be finite and > 0", who);
   int nb = 0;
   if (blockmask) {
     if (block != 128) return fail(TPS_ERR_INVALID_ARG, "%s: block=%d, only 128 is supported", who, block);

@@ -9,18 +9,22 @@
 // 128-key blocks its ORIGINAL 128-token block keeps; whole key tiles that no
 // query of a CTA needs are never loaded.
 //
-// Kernel layout (one CTA = 128 compacted active queries x one head):
-//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r). Reads S from
-//              TMEM, applies scale / masks / online softmax in the log2 domain,
-//              rescales O in TMEM when the running max grows, writes P (bf16) to
-//              shared memory, and finally normalises O and stores it.
-//   warp 4     TMA producer: Q once, then K and V tiles (128 keys each) into a
-//              two-stage ring, 128-byte swizzled.
-//   warp 5     MMA issuer and TMEM owner: S_j = Q K_j^T into one of two TMEM S
-//              buffers, O += P_j V_j into the TMEM O accumulator; completion is
-//              signalled with tcgen05.commit on mbarriers.
-// S_{j+1} is issued as soon as its buffer is free, so the tensor cores compute
-// S_{j+1} and P_j V_j while the softmax warps work on tile j+1.
+// One CTA = 256 compacted active queries of one head, as two 128-row tiles
+// (t = 0, 1) that share every K/V tile and take turns on the tensor cores:
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r of
+//              its tile (= TMEM lane r). Loads S from TMEM, online softmax in
+//              the log2 domain, writes P (bf16) back over the first half of
+//              its S columns, and rescales O in TMEM only when the running
+//              maximum grew by more than 2^8 (exact: the final normalisation
+//              uses the same reference maximum as every P).
+//   warp 8     TMA producer: Q (both tiles) once, then K and V tiles of 128
+//              keys into a two-stage ring, 128-byte swizzled.
+//   warp 9     MMA issuer and TMEM owner. Per key tile j and tile t:
+//              O_t += P_t(j) V_j (A operand read from TMEM), then
+//              S_t(j+1) = Q_t K_{j+1}^T; completion via tcgen05.commit.
+// While softmax t works on S_t(j+1), the tensor cores run the other tile's
+// P V and Q K^T, so MMA and softmax overlap.
+// TMEM: tile t owns columns [256t, 256t+128) for S/P and [256t+128, +D) for O.
 // Every mbarrier wait is bounded: on expiry the CTA sets an abort flag and the
 // device status word (TPS_ERR_TIMEOUT via tps_check), drains what it issued,
 // frees TMEM and returns.
@@ -34,44 +38,70 @@ namespace {
 
 using namespace tc;
 
-constexpr int kBM = 128;        // queries per CTA (MMA M)
+constexpr int kBM = 128;        // query rows per tile (MMA M)
+constexpr int kQT = 2;          // query tiles per CTA
 constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
-constexpr int kThreads = 192;   // 4 softmax warps + TMA warp + MMA warp
-constexpr int kTmemCols = 512;  // S0 | S1 | O
-constexpr int kSubBytes = kBN * 128;   // one [128 rows x 64 bf16] swizzled sub-tile
+constexpr int kSoftmaxThreads = kQT * kBM;
+constexpr int kThreads = kSoftmaxThreads + 64;   // + TMA warp + MMA warp
+constexpr int kWarps = kThreads / 32;
+constexpr int kTmaWarp = kSoftmaxThreads / 32;
+constexpr int kMmaWarp = kTmaWarp + 1;
+constexpr int kTmemCols = 512;
+constexpr int kSubBytes = 128 * 128;   // one [128 rows x 64 bf16] swizzled sub-tile
+constexpr float kRescaleLog2 = 8.f;    // rescale O only when the max grows by > 2^8
 
 template <int D>
 struct Layout {
   static constexpr int kSub = D / 64;                    // 64-wide sub-tiles per row of Q/K/V
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kSub * kSubBytes;       // [stage][sub]
+  static constexpr int kQ = 0;                           // [tile][sub]
+  static constexpr int kK = kQ + kQT * kSub * kSubBytes; // [stage][sub]
   static constexpr int kV = kK + kStages * kSub * kSubBytes;
-  static constexpr int kP = kV + kStages * kSub * kSubBytes;   // 2 sub-tiles (128 keys)
-  static constexpr int kList = kP + 2 * kSubBytes;       // uint16 kept key blocks
+  static constexpr int kList = kV + kStages * kSub * kSubBytes;   // uint16 kept key blocks
   static constexpr int kListMax = 4096;
   static constexpr int kBar = kList + kListMax * 2;      // mbarriers (Bars)
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
 };
 
-struct Bars {  // mbarrier offsets inside the barrier block (8 bytes each)
-  static constexpr int q_full = 0;
-  static constexpr int k_full = 1;            // + stage
-  static constexpr int v_full = 1 + kStages;  // + stage
-  static constexpr int kv_empty = 1 + 2 * kStages;
-  static constexpr int s_full = 1 + 3 * kStages;   // + buffer (2)
-  static constexpr int s_free = 3 + 3 * kStages;   // + buffer (2)
-  static constexpr int p_full = 5 + 3 * kStages;
-  static constexpr int pv_done = 6 + 3 * kStages;
-  static constexpr int drain = 7 + 3 * kStages;    // last commit of the MMA thread
+struct Bars {  // mbarrier indices inside the barrier block (8 bytes each)
+  static constexpr int q_full = 0;                     // + tile
+  static constexpr int k_full = q_full + kQT;          // + stage
+  static constexpr int v_full = k_full + kStages;      // + stage
+  static constexpr int kv_empty = v_full + kStages;    // + stage
+  static constexpr int s_full = kv_empty + kStages;    // + tile
+  static constexpr int p_full = s_full + kQT;          // + tile
+  static constexpr int pv_done = p_full + kQT;         // + tile
+  static constexpr int drain = pv_done + kQT;          // last commit of the MMA thread
+  static constexpr int count = drain + 1;
 };
+static_assert(Bars::count * 8 <= 256, "barrier block");
 
 struct TcParams {
   AttnArgs a;
   float scale_log2;
   unsigned int* status;
 };
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi) in one packed instruction
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -82,13 +112,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __shared__ uint32_t s_tmem;
   __shared__ int s_ntiles;
   __shared__ volatile int s_abort;
-  __shared__ unsigned int s_wcnt[kThreads / 32];
+  __shared__ unsigned int s_wcnt[kWarps];
 
   const AttnArgs& p = prm.a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int64_t rows = active_count(p.count, p.cap);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
   if (row0 >= rows) return;   // whole CTA exits before touching TMEM or barriers
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -101,29 +131,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // ---- setup: barriers, TMEM, key-tile list ---------------------------------------------
   if (tid == 0) {
     s_abort = 0;
-    mbar_init(bar(Bars::q_full), 1);
+    for (int t = 0; t < kQT; ++t) {
+      mbar_init(bar(Bars::q_full + t), 1);
+      mbar_init(bar(Bars::s_full + t), 1);
+      mbar_init(bar(Bars::p_full + t), kBM);
+      mbar_init(bar(Bars::pv_done + t), 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(Bars::k_full + s), 1);
       mbar_init(bar(Bars::v_full + s), 1);
       mbar_init(bar(Bars::kv_empty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(Bars::s_full + b), 1);
-      mbar_init(bar(Bars::s_free + b), kBM);
-    }
-    mbar_init(bar(Bars::p_full), kBM);
-    mbar_init(bar(Bars::pv_done), 1);
     mbar_init(bar(Bars::drain), 1);
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc<kTmemCols>(smem_u32(&s_tmem));
-  if (warp == 4 && lane == 0) {
+  if (warp == kMmaWarp) tmem_alloc<kTmemCols>(smem_u32(&s_tmem));
+  if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
   if (p.bm) {
-    const int64_t rlast = row0 + kBM - 1 < rows ? row0 + kBM - 1 : rows - 1;
+    const int64_t rlast = row0 + kQT * kBM - 1 < rows ? row0 + kQT * kBM - 1 : rows - 1;
     int qb0 = p.idx[row0] / 128, qb1 = p.idx[rlast] / 128;
     qb0 = qb0 < 0 ? 0 : (qb0 >= p.nb ? p.nb - 1 : qb0);
     qb1 = qb1 < qb0 ? qb0 : (qb1 >= p.nb ? p.nb - 1 : qb1);
@@ -137,7 +166,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (lane == 0) s_wcnt[warp] = __popc(m);
       __syncthreads();
       int off = base, tot = 0;
-      for (int i = 0; i < kThreads / 32; ++i) {
+      for (int i = 0; i < kWarps; ++i) {
         off += i < warp ? s_wcnt[i] : 0;
         tot += s_wcnt[i];
       }
@@ -154,17 +183,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const int ntiles = s_ntiles;
   const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem;            // S buffer b at column 128 * b
-  const uint32_t tO = tmem + 256;      // O accumulator, D columns
+  auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
+  auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
   auto tile_kb = [&](int j) -> int { return p.bm ? static_cast<int>(sList[j]) : j; };
 
-  if (warp == 4) {
+  if (warp == kTmaWarp) {
     // ================================ TMA producer =====================================
     if (lane == 0) {
       int issued = 0;
-      mbar_expect_tx(bar(Bars::q_full), L::kSub * kSubBytes);
-      for (int s = 0; s < L::kSub; ++s)
-        tma_load_3d(sbase + L::kQ + s * kSubBytes, &tmQ, 64 * s, h, static_cast<int>(row0), bar(Bars::q_full));
+      for (int t = 0; t < kQT; ++t) {
+        mbar_expect_tx(bar(Bars::q_full + t), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kQ + (t * L::kSub + s) * kSubBytes, &tmQ, 64 * s, h,
+                      static_cast<int>(row0 + t * kBM), bar(Bars::q_full + t));
+      }
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % kStages;
         if (j >= kStages && !mbar_wait(bar(Bars::kv_empty + st), ((j / kStages) - 1) & 1, &s_abort, prm.status))
@@ -179,162 +211,172 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         issued = j + 1;
       }
       // drain: every load issued above must land before the CTA may exit
-      drain_wait(bar(Bars::q_full), 0);
+      for (int t = 0; t < kQT; ++t) drain_wait(bar(Bars::q_full + t), 0);
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j) {
         drain_wait(bar(Bars::k_full + j % kStages), (j / kStages) & 1);
         drain_wait(bar(Bars::v_full + j % kStages), (j / kStages) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ================================ MMA issuer =======================================
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, false, false);  // Q K^T: both K-major
       constexpr uint32_t kIdescO = idesc_bf16(kBM, D, false, true);     // P V: V is MN-major
-      bool ok = mbar_wait(bar(Bars::q_full), 0, &s_abort, prm.status);
-      tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kStages, b = j & 1;
-        if (!mbar_wait(bar(Bars::k_full + st), (j / kStages) & 1, &s_abort, prm.status)) return false;
-        tc_fence_after();
+      auto issue_s = [&](int t, int j) {
+        const int st = j % kStages;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;   // 16 bf16 along d
-          const uint64_t da = sdesc_sw128(sbase + L::kQ + off, 16, 1024);
+          const uint64_t da = sdesc_sw128(sbase + L::kQ + t * L::kSub * kSubBytes + off, 16, 1024);
           const uint64_t db = sdesc_sw128(sbase + L::kK + st * L::kSub * kSubBytes + off, 16, 1024);
-          mma_f16_ss(tS + 128 * b, da, db, kIdescS, kk > 0);
+          mma_f16_ss(tS(t), da, db, kIdescS, kk > 0);
         }
-        mma_commit(bar(Bars::s_full + b));
-        return true;
+        mma_commit(bar(Bars::s_full + t));
       };
-      if (ok && ntiles > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles) {
-          if (j + 1 >= 2) {
-            ok = mbar_wait(bar(Bars::s_free + ((j + 1) & 1)), (((j + 1) >> 1) - 1) & 1, &s_abort, prm.status);
-            tc_fence_after();
-          }
-          if (ok) ok = issue_s(j + 1);
-          if (!ok) break;
-        }
-        const int st = j % kStages;
-        if (!mbar_wait(bar(Bars::p_full), j & 1, &s_abort, prm.status)) break;
-        if (!mbar_wait(bar(Bars::v_full + st), (j / kStages) & 1, &s_abort, prm.status)) break;
+      bool ok = ntiles > 0;
+      if (ok) ok = mbar_wait(bar(Bars::k_full), 0, &s_abort, prm.status);
+      for (int t = 0; ok && t < kQT; ++t) {
+        ok = mbar_wait(bar(Bars::q_full + t), 0, &s_abort, prm.status);
         tc_fence_after();
+        if (ok) issue_s(t, 0);
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int st = j % kStages;
+        for (int t = 0; ok && t < kQT; ++t) {
+          ok = mbar_wait(bar(Bars::p_full + t), j & 1, &s_abort, prm.status);
+          if (ok && t == 0) ok = mbar_wait(bar(Bars::v_full + st), (j / kStages) & 1, &s_abort, prm.status);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // A = P [128 q x 128 keys], K-major (keys contiguous): 16 keys per step
-          const uint64_t da = sdesc_sw128(sbase + L::kP + (kk >> 2) * kSubBytes + (kk & 3) * 32, 16, 1024);
-          // B = V [128 keys x D], MN-major: 16 keys = 2 swizzle atoms of 8 rows;
-          // LBO = next 64-wide d sub-tile, SBO = next 8 keys
-          const uint64_t db = sdesc_sw128(sbase + L::kV + st * L::kSub * kSubBytes + kk * 16 * 128, kSubBytes, 1024);
-          mma_f16_ss(tO, da, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // B = V [128 keys x D], MN-major: 16 keys = 2 swizzle atoms of 8 rows;
+            // LBO = next 64-wide d sub-tile, SBO = next 8 keys. A = P_t from TMEM,
+            // 16 keys = 8 columns of bf16 pairs.
+            const uint64_t db = sdesc_sw128(sbase + L::kV + st * L::kSub * kSubBytes + kk * 16 * 128, kSubBytes, 1024);
+            mma_f16_ts(tO(t), tS(t) + 8 * kk, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(Bars::pv_done + t));
+          if (t == kQT - 1) mma_commit(bar(Bars::kv_empty + st));
+          if (j + 1 < ntiles) {
+            // S_t(j+1) overwrites the columns P_t(j) was read from: tcgen05.mma
+            // operations of one thread execute in issue order.
+            if (t == 0) {
+              ok = mbar_wait(bar(Bars::k_full + (j + 1) % kStages), ((j + 1) / kStages) & 1, &s_abort, prm.status);
+              tc_fence_after();
+            }
+            if (ok) issue_s(t, j + 1);
+          }
         }
-        mma_commit(bar(Bars::pv_done));
-        mma_commit(bar(Bars::kv_empty + st));
       }
       mma_commit(bar(Bars::drain));   // fires once every MMA issued above has completed
     }
   } else {
     // ================================ softmax warps ====================================
-    const int r = tid;                            // query row within the tile == TMEM lane
-    const int64_t row = row0 + r;
+    const int t = warp >> 2;                      // query tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
+    const int64_t row = row0 + t * kBM + r;
     const bool valid = row < rows;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int qb = 0;
     if (p.bm) {
       qb = p.idx[valid ? row : rows - 1] / 128;
       qb = qb < 0 ? 0 : (qb >= p.nb ? p.nb - 1 : qb);
     }
     const float sl2 = prm.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_run = -INFINITY, l_run = 0.f;
-    uint8_t* sP = gbase + L::kP;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int b = j & 1;
       // every wait result is made warp-uniform: tcgen05.ld/st are .sync.aligned
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + b), (j >> 1) & 1, &s_abort, prm.status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + t), j & 1, &s_abort, prm.status))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + 128 * b + 32 * c + lane_off, s + 32 * c);
-      tc_fence_before();
-      mbar_arrive(bar(Bars::s_free + b));
+      uint32_t sr[kBN];
+      tmem_ld128(tS(t) + lane_off, sr);
 
       const int kb = tile_kb(j);
       const int64_t key0 = static_cast<int64_t>(kb) * kBN;
       const bool row_ok = !p.bm || p.bm[static_cast<int64_t>(qb) * p.nb + kb] != 0;
       const int nvalid = row_ok ? static_cast<int>(p.N - key0 < kBN ? p.N - key0 : kBN) : 0;
-      float tmax = -INFINITY;
+      if (nvalid < kBN) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        const float x = c < nvalid ? s[c] * sl2 : -INFINITY;
-        s[c] = x;
-        tmax = fmaxf(tmax, x);
+        for (int c = 0; c < kBN; ++c)
+          if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
       }
-      const float m_new = fmaxf(m_run, tmax);
-      const float base = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = m_run == -INFINITY ? (j == 0 ? 1.f : 0.f) : fast_exp2(m_run - m_new);
-      float psum = 0.f;
-      uint32_t pk[kBN / 2];
+      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = fast_exp2(s[c] - base), p1 = fast_exp2(s[c + 1] - base);
-        psum += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+      for (int c = 4; c < kBN; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
       }
-      l_run = l_run * alpha + psum;
-      m_run = m_new;
-
-      if (j > 0) {
-        // PV_{j-1} must be complete before O is rescaled and before P is overwritten
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::pv_done), (j - 1) & 1, &s_abort, prm.status))) {
+      const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      if (j == 0) {
+        m_run = m_new;
+      } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleLog2)) {
+        // the warp moves its reference maxima; O (complete up to tile j-1) is rescaled
+        const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(tO + 32 * c + lane_off, o);
+        for (int c = 0; c < D; c += 32) {           // 32 columns at a time: S stays in registers
+          float o[32];
+          tmem_ld32(tO(t) + lane_off + c, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO + 32 * c + lane_off, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO(t) + lane_off + c, o);
         }
+        l_run *= alpha;
+        m_run = m_new;
       }
-      // P row r -> two K-major swizzled sub-tiles (keys 0-63, 64-127)
+      const float base = m_run == -INFINITY ? 0.f : m_run;
+      const uint64_t nbase = f2_pack(-base, -base);
+      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+      uint32_t pk[kBN / 2];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int sub = c >> 3, cc = c & 7;
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(sP + sub * kSubBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+      for (int c = 0; c < kBN; c += 4) {
+        float a0, a1, a2, a3;
+        f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
+        f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
+        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+        acc0 = fadd2(acc0, f2_pack(p0, p1));
+        acc1 = fadd2(acc1, f2_pack(p2, p3));
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+        pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
       }
-      fence_proxy_async_smem();
+      float s0, s1, s2, s3;
+      f2_unpack(acc0, s0, s1);
+      f2_unpack(acc1, s2, s3);
+      l_run += (s0 + s1) + (s2 + s3);
+      tmem_st64(tS(t) + lane_off, pk);            // P_t(j) over the first 64 columns of S_t
       tc_fence_before();
-      mbar_arrive(bar(Bars::p_full));
+      mbar_arrive(bar(Bars::p_full + t));
     }
     // ---- epilogue ------------------------------------------------------------------------
-    if (ok && ntiles > 0) ok = mbar_wait(bar(Bars::pv_done), (ntiles - 1) & 1, &s_abort, prm.status);
+    if (ok && ntiles > 0) ok = mbar_wait(bar(Bars::pv_done + t), (ntiles - 1) & 1, &s_abort, prm.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D; c += 32) {
         float o[32];
-        if (ntiles > 0) tmem_ld32(tO + 32 * c + lane_off, o);
+        if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
         else
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         if (valid) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            orow[4 * c + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
+            orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
                                          pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
                                          pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
                                          pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
@@ -345,11 +387,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 
   // ---- teardown ------------------------------------------------------------------------
-  if (warp == 5 && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
+  if (warp == kMmaWarp && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tmem_dealloc<kTmemCols>(tmem);
   }
@@ -412,7 +454,7 @@ int launch(const AttnArgs& a, cudaStream_t st) {
     attr_done[dev] = true;
   }
   TcParams prm{a, a.scale * kLog2e, status};
-  dim3 grid(static_cast<unsigned int>((a.cap + kBM - 1) / kBM), static_cast<unsigned int>(a.H));
+  dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H));
   attn_tc_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   return launch_status("pruned_attn");
 }
