@@ -53,7 +53,7 @@ def peaks():
 
 def attn_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("attn_tc.cu", "attn_common.cuh", "tps_internal.cuh"):
+    for name in ("attn_tc.cu", "attn_common.cuh", "tc_ptx.cuh", "tps_internal.cuh"):
         p = os.path.join(ROOT, "token_pruned_sparse_b200", "csrc", name)
         if os.path.exists(p):
             with open(p, "rb") as f:
@@ -176,6 +176,27 @@ class MidStep:
         if ev_attn:
             ev_attn[1].record()
         t.scatter_out(self.o_full, self.o_act, self.idx, self.cnt)
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank runs an independent layer: rank r shifts the video seed by r."""
+    return rank
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's
+    time); a no-op at world size 1. Works with any initialised backend."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(per_rank_units: float, world: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job rate: the units every rank processed over the max-over-ranks time."""
+    return world * per_rank_units * steps / (total_ms_max * 1e-3)
 
 
 def flush_l2(buf):
@@ -303,16 +324,145 @@ class OracleStep:
                 f"costs fitted from 64- and 256-row samples)")
 
 
-def oracle_baseline(rows: int):
-    """cpu_baseline of the GPU arm: one linear pass + one attention sample."""
+def oracle_baseline():
+    """cpu_baseline of the GPU arm: one complete mid step through the fp64
+    oracle (every active row, every head), timed on the host cores."""
     o = OracleStep()
     t_lin = o.linear()
-    o.fit()
-    t_att = o.attn(rows)
-    full = o.full_step(t_lin, t_att, rows)
+    t_att = o.attn(o.k)
+    full = t_lin + t_att
     return {"value": round(o.flops / full / 1e12, 6), "unit": "TFLOP/s", "cores": o.threads, "kind": "oracle",
-            "sample": o.describe(rows), "seconds_spent": round(t_lin + t_att, 2),
-            "seconds_per_step_extrapolated": round(full, 2)}
+            "sample": f"one complete mid step (score/select/gather/kv_sync/scatter over {o.N} tokens, attention "
+                      f"of all {o.k} active rows x {o.H} heads in fp64 numpy/BLAS)",
+            "seconds": round(full, 2)}
+
+
+# ------------------------------------------------------- per-config sweep ------
+def _time(fn, flush, reps=5, warm=2):
+    ms = []
+    for i in range(warm + reps):
+        flush_l2(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= warm:
+            ms.append(a.elapsed_time(b))
+    return float(np.median(ms))
+
+
+def executed_key_tiles(idx: np.ndarray, N: int, nb_mask=None, rows_per_cta=256):
+    """Key tiles the attention kernel runs per CTA (dense: all; masked: the
+    union of the mask rows of the query blocks a CTA spans)."""
+    nkt = -(-N // 128)
+    A = len(idx)
+    ctas = -(-A // rows_per_cta)
+    if nb_mask is None:
+        return ctas * nkt, ctas
+    tot = 0
+    for c in range(ctas):
+        r0, r1 = c * rows_per_cta, min(A, (c + 1) * rows_per_cta) - 1
+        qb0, qb1 = idx[r0] // 128, idx[r1] // 128
+        tot += int(np.any(nb_mask[qb0:qb1 + 1] != 0, axis=0).sum())
+    return tot, ctas
+
+
+def config_sweep(dev, peak_tflops, hbm_gbs):
+    """Kernel-level numbers on the larger configs (inputs resident in HBM, L2
+    flushed before every timed call). Attention: algorithmic FLOPs (4*d per
+    query-key-head pair over allowed keys) and executed FLOPs (padded 256-row
+    query tiles x whole 128-key tiles that the kernel runs). Memory-bound
+    stages: algorithmic bytes / time against the measured HBM copy peak."""
+    from token_pruned_sparse_b200 import tps
+    g = torch.Generator(device=dev)
+    g.manual_seed(4)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    out = {}
+    # ---- HSA: 33 x 45x80 = 118800 tokens, 24 heads, d = 128 -----------------------------
+    cfg = synth.CONFIGS["hsa"]
+    N, H, d, C = cfg.video.N, cfg.H, cfg.d, cfg.video.C
+    R = H * d * 2                       # bytes of one K/V/Q/O row
+    rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    v_prev, v_cur = rnd(cfg.video.F, cfg.video.HW, C), rnd(cfg.video.F, cfg.video.HW, C)
+    score = torch.empty(N, dtype=torch.float32, device=dev)
+    stages = {}
+    t = _time(lambda: tps.lipar_score(v_cur, v_prev, out=score), flush)
+    stages["score_interstep"] = (t, N * (4 * C + 4))
+    x_frames = rnd(cfg.video.F, cfg.video.HW, C)
+    t = _time(lambda: tps.lipar_score(x_frames, out=score), flush)
+    stages["score_interframe"] = (t, N * (2 * C + 4))
+    ws = tps.workspace(tps.OP_SELECT, N, 0, dev)
+    idx_all = torch.empty(N, dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    k3 = N // 3
+    t = _time(lambda: tps.lipar_select(score, tps.SELECT_TOPK, k=k3, idx=idx_all, count=cnt, ws=ws), flush)
+    stages["select_topk"] = (t, N * 4 + k3 * 4)
+    t = _time(lambda: tps.lipar_select(score, tps.SELECT_THRESHOLD, tau=1.0, idx=idx_all, count=cnt, ws=ws), flush)
+    stages["select_threshold"] = (t, N * 4 + int(cnt.item()) * 4)
+    K = cfg.extra["K"]
+    wsg = tps.workspace(tps.OP_GROUP, N, K, dev)
+    grp = torch.empty(N, dtype=torch.int8, device=dev)
+    t = _time(lambda: tps.lipar_group(score, K, group=grp, ws=wsg), flush)
+    stages["group"] = (t, N * 4 + N)
+    wss = tps.workspace(tps.OP_SCHEDULE, N, K, dev)
+    t = _time(lambda: tps.lipar_schedule(grp, K, cfg.extra["budgets"], cfg.extra["T"], 1, 0, idx=idx_all, count=cnt,
+                                         ws=wss), flush)
+    A = int(cnt.item())
+    stages["schedule"] = (t, N + A * 4)
+    idx = idx_all[:A].clone()
+    kc, vc = rnd(N, H, d), rnd(N, H, d)
+    kf, vf = rnd(A, H, d), rnd(A, H, d)
+    ke, ve = torch.empty_like(kc), torch.empty_like(vc)
+    t = _time(lambda: tps.tps_gather_rows(kf, kc, idx, cnt), flush)
+    stages["gather"] = (t, 2 * R * A)
+    t = _time(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt), flush)
+    stages["kv_sync"] = (t, 4 * R * A + 4 * A)
+    t = _time(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve), flush)
+    stages["kv_sync_renoise"] = (t, 6 * R * A + 4 * R * (N - A) + 4 * A)
+    o_full, o_act = rnd(N, H, d), rnd(A, H, d)
+    t = _time(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
+    stages["scatter_out"] = (t, 2 * R * A)
+    out["stages_hsa"] = {k: {"ms": round(v[0], 4), "bytes": int(v[1]), "GBps": round(v[1] / v[0] / 1e6, 1),
+                             "frac_hbm": round(v[1] / v[0] / 1e6 / hbm_gbs, 3)} for k, v in stages.items()}
+    # ---- HSA attention per step size --------------------------------------------------
+    att = {}
+    scale = 1 / math.sqrt(d)
+    for name, Aq in (("hsa_A_N/3", N // 3), ("hsa_A_2N/3", 2 * N // 3), ("hsa_A_N", N)):
+        q = rnd(Aq, H, d)
+        ii = torch.arange(0, N, N // Aq if Aq < N else 1, device=dev, dtype=torch.int32)[:Aq].contiguous()
+        cc = torch.tensor([Aq], dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        t = _time(lambda: tps.pruned_attn(q, ke, ve, ii, cc, scale, o_act=o), flush, reps=3, warm=1)
+        alg = 4.0 * d * H * Aq * N
+        tiles, ctas = executed_key_tiles(np.arange(Aq), N)
+        exe = 4.0 * d * H * 256 * 128 * tiles
+        att[name] = {"ms": round(t, 3), "tflops_alg": round(alg / t / 1e9, 1), "tflops_exec": round(exe / t / 1e9, 1),
+                     "frac_peak_exec": round(exe / t / 1e9 / peak_tflops, 3)}
+        del q, o
+    # ---- block-sparse: 40% active queries, 139 of 929 key blocks per query block --------
+    bcfg = synth.CONFIGS["block"]
+    xv, _ = synth.latent_video(bcfg.video)
+    xb = synth.to_bf16(xv).to(dev)
+    sc = tps.lipar_score(xb)
+    kb_ = synth.keep_count(N, bcfg.keep[0])
+    bidx, bcnt = tps.lipar_select(sc, tps.SELECT_TOPK, k=kb_)
+    bm = synth.block_mask_band_random(bcfg.video, 128, bcfg.extra["kept_per_row"], bcfg.video.seed)
+    bmd = bm.to(dev)
+    q = rnd(kb_, H, d)
+    o = torch.empty_like(q)
+    t = _time(lambda: tps.pruned_attn(q, kc, vc, bidx, bcnt, scale, blockmask=bmd, o_act=o), flush, reps=3, warm=1)
+    bidx_h = bidx.cpu().numpy()
+    bm_h = bm.numpy()
+    alg = 4.0 * d * H * 128 * float(bm_h[bidx_h // 128].sum())
+    alg -= 4.0 * d * H * float(np.sum(bm_h[bidx_h // 128][:, -1])) * (128 - (N - (bm_h.shape[0] - 1) * 128))
+    tiles, ctas = executed_key_tiles(bidx_h, N, bm_h)
+    exe = 4.0 * d * H * 256 * 128 * tiles
+    att["block_sparse"] = {"ms": round(t, 3), "tflops_alg": round(alg / t / 1e9, 1),
+                           "tflops_exec": round(exe / t / 1e9, 1), "frac_peak_exec": round(exe / t / 1e9 / peak_tflops, 3),
+                           "exec_over_alg": round(exe / alg, 2)}
+    out["attention"] = att
+    return out
 
 
 # ------------------------------------------------------------------ main ------
@@ -326,7 +476,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
-    ap.add_argument("--oracle-rows", type=int, default=256)
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     a = ap.parse_args()
     if a.warmup < 3:
         a.warmup = 3
@@ -346,7 +496,7 @@ def main():
 
     from token_pruned_sparse_b200 import tps
     tps.lib()
-    st = MidStep(rank, dev, a.attn)
+    st = MidStep(rank_seed_offset(rank), dev, a.attn)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(a.warmup):
         st.step()
@@ -369,15 +519,10 @@ def main():
     clocks = sampler.stop()
     tps.tps_check()
 
-    total_ms = float(np.sum(step_ms))
-    attn_avg = float(np.mean(attn_ms))
-    if world > 1:
-        t = torch.tensor([total_ms, attn_avg], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, attn_avg = float(t[0]), float(t[1])
+    total_ms, attn_avg = max_over_ranks([np.sum(step_ms), np.mean(attn_ms)], world, dev)
     ms_per_step = total_ms / a.steps
-    value = world * st.flops * a.steps / (total_ms * 1e-3) / 1e12
-    tok_s = world * st.k * a.steps / (total_ms * 1e-3)
+    value = job_throughput(st.flops, world, a.steps, total_ms) / 1e12
+    tok_s = job_throughput(st.k, world, a.steps, total_ms)
 
     # ---- end to end through the public API: pinned host inputs -> result on host
     e2e = None if a.no_e2e else e2e_leg(st, dev, max(3, min(a.steps, 50)), world)
@@ -392,9 +537,10 @@ def main():
                 "kernel": "pruned_attn" if a.attn == "tc" else "pruned_attn_mma",
                 "flops_per_launch": st.flops, "avg_launch_ms": round(attn_avg, 4)}
 
+    configs = None if (a.no_configs or world > 1) else config_sweep(dev, peak, float(pk["hbm_gbs"]))
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu:
-        cpu = oracle_baseline(a.oracle_rows)
+        cpu = oracle_baseline()
 
     if world > 1:
         dist.barrier()
@@ -415,7 +561,7 @@ def main():
         "active_tokens_per_s": round(tok_s, 1),
         "gpu_launches": st.launches * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
-        "keep_sweep_wan": sweep,
+        "keep_sweep_wan": sweep, "configs": configs,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -447,13 +593,8 @@ def e2e_leg(st, dev, steps, world):
         one()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
-    return {"value": round(world * st.flops * steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    ms = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
+    return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 4)}
 
