@@ -35,7 +35,7 @@ __all__ = [
     "f64", "round_bf16", "lipar_score", "select_threshold", "select_topk", "group_split",
     "schedule_groups", "schedule_active", "compact", "kv_sync", "philox4x32_10",
     "philox_words", "renoise_normals", "pruned_attn", "scatter_out", "gather_rows",
-    "attn_flops",
+    "attn_flops", "euler_update",
 ]
 
 
@@ -329,6 +329,22 @@ def scatter_out(o_full, o_act, idx):
     if len(idx_t):
         out[idx_t] = o_act[: len(idx_t)]
     return out
+
+
+def euler_update(x, v_cache, v_fresh, idx, dsigma: float):
+    """[HSA] 2.3 cached Euler update: every token keeps the velocity predicted at
+    its most recent active step; at each global step ALL tokens advance by the
+    same Euler increment (sigma_{i+1} - sigma_i) -- active tokens with their
+    fresh velocity, skipped tokens with the cached one -- as one operation over
+    the N tokens. Reading: the sampler state x is float32, velocities bf16.
+
+    Returns (x_new float64 [N, C], v_cache_new bf16 [N, C]) with
+    v_cache_new[idx] = v_fresh (bit copies) and x_new = x + dsigma * v_cache_new."""
+    vc = v_cache.clone()
+    idx_t = torch.as_tensor(np.asarray(idx, np.int64))
+    if len(idx_t):
+        vc[idx_t] = v_fresh[: len(idx_t)]
+    return f64(x) + float(dsigma) * f64(vc), vc
 
 
 def gather_rows(src, idx):

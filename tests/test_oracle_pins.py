@@ -320,3 +320,39 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     assert list(O.select_topk(s, 1)) == [0]
     # a strict '>' threshold would select k-1 at tau = s_(k)
     assert len(O.select_threshold(np.array([3.0, 2.0, 1.0]), 2.0)) == 2
+
+
+# ------------------------------------------------------- HSA cached Euler ---
+def test_euler_worked_example():
+    g = _gold("euler_worked.json")
+    x = torch.tensor(g["x"], dtype=torch.float32)
+    vc = torch.tensor(g["v_cache"], dtype=torch.bfloat16)
+    vf = torch.tensor(g["v_fresh"], dtype=torch.bfloat16)
+    xn, vcn = O.euler_update(x, vc, vf, g["idx"], g["dsigma"])
+    assert xn.tolist() == g["x_new"]
+    assert vcn.float().tolist() == g["v_cache_new"]
+
+
+def test_euler_closed_forms():
+    """dsigma = 0 leaves x unchanged; all-active is the plain Euler step with the
+    fresh velocity; constant velocities telescope over a schedule:
+    x_T = x_0 + (sigma_T - sigma_0) * v exactly (dyadic values)."""
+    rng = np.random.default_rng(7)
+    N, C = 40, 16
+    x0 = torch.from_numpy(rng.integers(-64, 64, (N, C)).astype(np.float32) / 8)
+    v = torch.from_numpy(rng.integers(-16, 16, (N, C)).astype(np.float32) / 4).to(torch.bfloat16)
+    idx = np.array([3, 9, 20], np.int32)
+    xn, vcn = O.euler_update(x0, v, v[idx] * 2, idx, 0.0)
+    np.testing.assert_array_equal(xn, x0.double().numpy())
+    assert torch.equal(vcn[idx], v[idx] * 2)
+    xa, _ = O.euler_update(x0, v * 0, v, np.arange(N), -0.125)
+    np.testing.assert_array_equal(xa, x0.double().numpy() - 0.125 * v.double().numpy())
+    T = 8
+    sig = [1 - i / T for i in range(T + 1)]
+    x = x0.double()
+    vc = v.clone()
+    for i in range(T):
+        act = np.arange(N)[np.arange(N) % (1 + i % 3) == 0]     # a varying active set
+        xi, vc = O.euler_update(x, vc, v[act], act, sig[i + 1] - sig[i])
+        x = torch.from_numpy(xi)
+    np.testing.assert_array_equal(x.numpy(), x0.double().numpy() + (sig[T] - sig[0]) * v.double().numpy())
