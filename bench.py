@@ -423,6 +423,12 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     o_full, o_act = rnd(N, H, d), rnd(A, H, d)
     t = _time(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
     stages["scatter_out"] = (t, 2 * R * A)
+    # cached Euler update (HSA 2.3): fp32 state [N, C], bf16 velocity cache
+    xs = torch.randn(N, C, generator=g, device=dev, dtype=torch.float32)
+    vcache = rnd(N, C)
+    vfresh = rnd(A, C)
+    t = _time(lambda: tps.hsa_euler_update(xs, vcache, vfresh, idx, cnt, -0.025), flush)
+    stages["euler_update"] = (t, A * (2 * C + 2 * C + 8 * C) + (N - A) * (2 * C + 8 * C) + 4 * A)
     out["stages_hsa"] = {k: {"ms": round(v[0], 4), "bytes": int(v[1]), "GBps": round(v[1] / v[0] / 1e6, 1),
                              "frac_hbm": round(v[1] / v[0] / 1e6 / hbm_gbs, 3)} for k, v in stages.items()}
     # ---- HSA attention per step size --------------------------------------------------

@@ -89,9 +89,12 @@ TPS_API int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16
  *   index; NaN ranks below -inf; -0 equals +0. 0 <= k <= N.
  * Output: idx[0 .. *count) ascending int32 token indices (idx must hold N
  *   entries for threshold mode, k for top-k), *count written on the device.
- * ws: device workspace of at least tps_workspace_size(TPS_OP_SELECT, N, 0)
- *   bytes, 16-byte aligned; its contents need no initialisation. Calls that
- *   share one workspace must be ordered on the GPU (same stream). */
+ * ws: device workspace, 16-byte aligned, of tps_workspace_size(TPS_OP_SELECT,
+ *   N, 0) bytes; its contents need no initialisation. With that size a call of
+ *   N <= 524,288 runs as one cooperative launch; a smaller workspace (down to
+ *   the multi-launch minimum, else TPS_ERR_WORKSPACE) selects the multi-launch
+ *   path, with identical results. Calls that share one workspace must be
+ *   ordered on the GPU (same stream). */
 #define TPS_SELECT_THRESHOLD 0
 #define TPS_SELECT_TOPK      1
 TPS_API int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
@@ -196,6 +199,20 @@ TPS_API int pruned_attn_mma(const tps_bf16* q_act, const tps_bf16* k, const tps_
  * o_full [N, H, d] keeps its cached output bit for bit. */
 TPS_API int scatter_out(tps_bf16* o_full, const tps_bf16* o_act, const int32_t* idx,
                 const int32_t* count, int64_t cap, int64_t N, int H, int d, tps_stream stream);
+
+/* ---- HSA cached Euler update ([HSA] 2.3) -------------------------------------
+ * Every token keeps the velocity of its most recent active step; each global
+ * step advances ALL tokens by the same increment dsigma = sigma_{i+1} - sigma_i:
+ *   v_cache[idx[j]] = v_fresh[j]        for j < min(*count, cap)  (bit copies)
+ *   x[n] = fmaf(dsigma, v_cache[n], x[n]) for every n < N (one rounding)
+ *   x        float32 [N, C], the sampler state (updated in place)
+ *   v_cache  bf16 [N, C], velocity of each token's last active step (in place)
+ *   v_fresh  bf16 [cap, C], velocities just predicted for the active tokens
+ * idx must be ascending and unique; duplicates or entries outside [0, N) are
+ * skipped and flagged (TPS_ERR_BOUNDS via tps_check). C % 8 == 0, C <= 4096. */
+TPS_API int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_fresh, const int32_t* idx,
+                             const int32_t* count, int64_t cap, int64_t N, int64_t C, float dsigma,
+                             tps_stream stream);
 
 /* ---- support --------------------------------------------------------------- */
 #define TPS_OP_SELECT   0

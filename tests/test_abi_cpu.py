@@ -59,7 +59,7 @@ def test_select_validation_and_workspace():
     assert code == tps.INVALID_ARG and "k=11" in msg
     need = tps.workspace_size(tps.OP_SELECT, 100000)
     assert need > 0 and tps.workspace_size(tps.OP_SELECT, 200000) > need
-    code, msg = _err(l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, F, need - 1, NULL))
+    code, msg = _err(l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, F, 1024, NULL))
     assert code == tps.WORKSPACE and "required" in msg
     assert l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, NULL, need, NULL) == tps.WORKSPACE
     assert l.lipar_select(F, 100000, tps.SELECT_THRESHOLD, 0.0, 0, F, F, MIS, need, NULL) == tps.ALIGN

@@ -108,3 +108,41 @@ def test_count_below_cap_and_bounds_flag():
     ref = O.scatter_out(full, act[[0, 1, 2, 4]], np.array([1, 5, 9, 11]))
     assert torch.equal(fd.cpu(), ref)
     tps.tps_check()                                                         # flag was cleared
+
+
+# ------------------------------------------------------- HSA cached Euler ---
+def _ulp32(a):
+    return np.spacing(np.abs(a).astype(np.float32)).astype(np.float64)
+
+
+@pytest.mark.parametrize("N,C,A", [(256, 64, 100), (1001, 128, 333), (118800, 128, 39600), (50, 8, 50), (77, 16, 0)])
+def test_euler_update_parity(N, C, A):
+    rng = np.random.default_rng(N + C + A)
+    x = torch.from_numpy(rng.standard_normal((N, C)).astype(np.float32))
+    vc = synth.gaussian_bf16((N, C), N + 1)
+    vf = synth.gaussian_bf16((max(A, 1), C), N + 2)[:max(A, 1)]
+    idx = np.sort(rng.choice(N, A, replace=False)).astype(np.int32)
+    di, dc = _dev_idx(idx)
+    xd, vcd = x.to(DEV), vc.to(DEV)
+    dsigma = -2.0 ** -5                                         # exact in fp32 and fp64
+    x_ref, vc_ref = x, vc
+    for step in range(1, 3):                                    # two steps in a row
+        tps.hsa_euler_update(xd, vcd, vf.to(DEV), di, dc, dsigma, cap=A)
+        x_ref, vc_ref = O.euler_update(x_ref, vc_ref, vf[:A], idx, dsigma)   # the oracle's own state
+        assert torch.equal(vcd.cpu(), vc_ref)
+        got = xd.cpu().double().numpy()
+        # one fp32 rounding (fmaf) per step on the device, none in the fp64 oracle
+        assert np.all(np.abs(got - x_ref) <= step * _ulp32(x_ref) + 1e-45)
+    tps.tps_check()
+
+
+def test_euler_update_flags_bad_index():
+    N, C = 64, 8
+    x = torch.zeros((N, C), device=DEV)
+    vc = torch.zeros((N, C), dtype=torch.bfloat16, device=DEV)
+    vf = torch.ones((3, C), dtype=torch.bfloat16, device=DEV)
+    idx = torch.tensor([5, 5, 9], dtype=torch.int32, device=DEV)   # duplicate
+    tps.hsa_euler_update(x, vc, vf, idx, torch.tensor([3], dtype=torch.int32, device=DEV), 1.0)
+    with pytest.raises(tps.TPSError) as e:
+        tps.tps_check()
+    assert e.value.code == tps.BOUNDS

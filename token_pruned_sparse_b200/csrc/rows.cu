@@ -85,8 +85,16 @@ __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
 }
 
 // u = (floor(w / 2^9) + 1/2) * 2^-23: exact in fp32, strictly inside (0, 1).
+// Built from the bits: 1 + k * 2^-23 (exponent of 1.0, mantissa k = w >> 9),
+// minus (1 - 2^-24); both operands and the difference are exact in fp32.
 __device__ __forceinline__ float uniform01(uint32_t w) {
-  return (static_cast<float>(w >> 9) + 0.5f) * 1.1920928955078125e-07f;
+  return __uint_as_float(0x3F800000u | (w >> 9)) - 0.99999994039535522461f;
+}
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Box-Muller on one word pair: z0 = r cos(2 pi ub), z1 = r sin(2 pi ub),
@@ -94,7 +102,7 @@ __device__ __forceinline__ float uniform01(uint32_t w) {
 // the hardware sine/cosine are accurate, and the signs folded back.
 __device__ __forceinline__ void box_muller(uint32_t wa, uint32_t wb, float& z0, float& z1) {
   const float ua = uniform01(wa), ub = uniform01(wb);
-  const float r = sqrtf(-2.0f * logf(ua));
+  const float r = sqrt_approx(-2.0f * logf(ua));   // hardware sqrt, ~2^-23 relative
   const float th = 6.28318530717958647692f * (ub - 0.5f);
   float sn, cs;
   __sincosf(th, &sn, &cs);

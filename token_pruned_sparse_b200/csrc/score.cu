@@ -19,69 +19,101 @@
 namespace tps {
 namespace {
 
-template <int L>
+// kV > 0: vectors per row known at compile time (all loads of an iteration are
+// issued before any is used); kV == 0: runtime C.
+template <int L, int kV>
 __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__ x,
                                                     const uint16_t* __restrict__ xref,
                                                     const uint16_t* __restrict__ xprev,
-                                                    int64_t HW, int C, int64_t N,
+                                                    int64_t HW, int Crt, int64_t N,
                                                     float* __restrict__ score) {
   constexpr int kTokPerWarp = 32 / L;
   const int lane = threadIdx.x & 31;
   const int sub = lane & (L - 1);
-  const int V = C >> 3;  // 16-byte vectors per row
+  const int V = kV > 0 ? kV : (Crt >> 3);  // 16-byte vectors per row
+  const int C = kV > 0 ? kV * 8 : Crt;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += nwarps * kTokPerWarp) {
-    const int64_t t = w0 + lane / L;
-    const bool valid = t < N;
-    const uint16_t* ref = nullptr;
-    if (valid) {
-      if (xref) ref = xref + t * C;
-      else if (t >= HW) ref = x + (t - HW) * C;
-      else if (xprev) ref = xprev + t * C;
-    }
-    float num = 0.f, den = 0.f;
-    if (ref) {
-      const uint16_t* cur = x + t * C;
-#pragma unroll 4
-      for (int v = sub; v < V; v += L) {
-        const uint4 a = ld16(cur + v * 8);
-        const uint4 b = ld16(ref + v * 8);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+  // two token groups per iteration (w0 and w0 + half the grid stride) so more
+  // 16-byte loads are in flight per lane; the grid is one resident wave
+  const int64_t stride = nwarps * kTokPerWarp;
+  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += 2 * stride) {
+    const uint16_t* cur[2];
+    const uint16_t* ref[2];
+    int64_t tt[2];
+    bool valid[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
-          const float r0 = bf16lo(bw[i]), r1 = bf16hi(bw[i]);
-          num += fabsf(c0 - r0) + fabsf(c1 - r1);
-          den += fabsf(r0) + fabsf(r1);
-        }
+    for (int k = 0; k < 2; ++k) {
+      const int64_t t = w0 + k * stride + lane / L;
+      tt[k] = t;
+      valid[k] = t < N;
+      ref[k] = nullptr;
+      cur[k] = x + (valid[k] ? t : 0) * C;
+      if (valid[k]) {
+        if (xref) ref[k] = xref + t * C;
+        else if (t >= HW) ref[k] = x + (t - HW) * C;
+        else if (xprev) ref[k] = xprev + t * C;
       }
     }
+    float num[2] = {0.f, 0.f}, den[2] = {0.f, 0.f};
 #pragma unroll
-    for (int o = L / 2; o > 0; o >>= 1) {
-      num += __shfl_xor_sync(0xffffffffu, num, o);
-      den += __shfl_xor_sync(0xffffffffu, den, o);
+    for (int v = sub; v < (kV > 0 ? kV : V); v += L) {
+      uint4 a[2], b[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (ref[k]) {
+          a[k] = ld16(cur[k] + v * 8);
+          b[k] = ld16(ref[k] + v * 8);
+        }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (ref[k]) {
+          const uint32_t aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+          const uint32_t bw[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
+            const float r0 = bf16lo(bw[i]), r1 = bf16hi(bw[i]);
+            num[k] += fabsf(c0 - r0) + fabsf(c1 - r1);
+            den[k] += fabsf(r0) + fabsf(r1);
+          }
+        }
     }
-    if (valid && sub == 0) {
-      float s;
-      if (!ref) s = INFINITY;                       // frame 0 without a predecessor
-      else if (den > 0.f) s = num / den;
-      else s = num > 0.f ? INFINITY : 0.f;
-      score[t] = s;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+#pragma unroll
+      for (int o = L / 2; o > 0; o >>= 1) {
+        num[k] += __shfl_xor_sync(0xffffffffu, num[k], o);
+        den[k] += __shfl_xor_sync(0xffffffffu, den[k], o);
+      }
+      if (valid[k] && sub == 0) {
+        float s;
+        if (!ref[k]) s = INFINITY;                  // frame 0 without a predecessor
+        else if (den[k] > 0.f) s = num[k] / den[k];
+        else s = num[k] > 0.f ? INFINITY : 0.f;
+        score[tt[k]] = s;
+      }
     }
   }
 }
 
-template <int L>
+template <int L, int kV>
 void launch_score(const uint16_t* x, const uint16_t* xr, const uint16_t* xp, int64_t HW, int C,
                   int64_t N, float* score, cudaStream_t st) {
   constexpr int kThreads = 256;
   const int64_t tok_per_block = (kThreads / 32) * (32 / L);
-  int64_t blocks = (N + tok_per_block - 1) / tok_per_block;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  int64_t blocks = (N + 2 * tok_per_block - 1) / (2 * tok_per_block);
+  static int per_sm[64] = {0};                  // resident blocks per SM (one wave)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !per_sm[dev]) {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, score_kernel<L, kV>, kThreads, 0) != cudaSuccess || b < 1) b = 4;
+    per_sm[dev] = b;
+  }
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (dev >= 0 && dev < 64 ? per_sm[dev] : 4);
   if (blocks > cap) blocks = cap;
-  score_kernel<L><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
+  score_kernel<L, kV><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
 }
 
 }  // namespace
@@ -105,10 +137,13 @@ extern "C" int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_b
   const uint16_t* p = x_prev_frame;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int c = static_cast<int>(C);
-  if (V >= 8) launch_score<8>(a, r, p, HW, c, N, score, st);
-  else if (V >= 4) launch_score<4>(a, r, p, HW, c, N, score, st);
-  else if (V >= 2) launch_score<2>(a, r, p, HW, c, N, score, st);
-  else launch_score<1>(a, r, p, HW, c, N, score, st);
+  if (c == 128) launch_score<8, 16>(a, r, p, HW, c, N, score, st);
+  else if (c == 64) launch_score<8, 8>(a, r, p, HW, c, N, score, st);
+  else if (c == 256) launch_score<8, 32>(a, r, p, HW, c, N, score, st);
+  else if (V >= 8) launch_score<8, 0>(a, r, p, HW, c, N, score, st);
+  else if (V >= 4) launch_score<4, 0>(a, r, p, HW, c, N, score, st);
+  else if (V >= 2) launch_score<2, 0>(a, r, p, HW, c, N, score, st);
+  else launch_score<1, 0>(a, r, p, HW, c, N, score, st);
   if (int e = launch_status("lipar_score")) return e;
   return ok();
 }

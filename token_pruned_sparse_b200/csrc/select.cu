@@ -361,6 +361,226 @@ __global__ void __launch_bounds__(kThreads) group_write(const float* __restrict_
   }
 }
 
+// ---- single-launch cooperative path (threshold, top-k, schedule) ----------------------
+// For N up to 256 blocks of 2048 elements the whole selection runs as ONE
+// cooperative launch (all blocks co-resident, guaranteed by the launch): each
+// block keeps its 2048 keys in registers; the four radix passes and the final
+// compaction are separated by grid barriers. A barrier is a counter in the
+// workspace (zeroed before the launch) that thread 0 of every block increments
+// and then polls; each poll loop is bounded by clock64 and, if it expires, sets
+// the device status word (TPS_ERR_TIMEOUT) and the block leaves without
+// writing results.
+constexpr int kCoopItems = 8;
+constexpr int kCoopTile = kThreads * kCoopItems;   // elements per block
+constexpr int kCoopMaxBlocks = 256;
+constexpr long long kGridWaitCycles = 2000000000LL; // ~1 s
+constexpr int kCoopHdrWords = 64;                   // barrier counter + padding
+
+enum CoopMode { kCoopThresh = 0, kCoopTopk = 1, kCoopSched = 2 };
+
+struct CoopArgs {
+  const float* s;
+  float tau;
+  const int8_t* g;
+  unsigned int act;
+  int K;
+  unsigned int k;          // top-k target (>= 1)
+};
+
+inline int64_t coop_blocks(int64_t N) { return (N + kCoopTile - 1) / kCoopTile; }
+// Workspace: header (barrier counter), one 256-bin histogram per radix pass
+// (summed with atomics; zeroed together with the header before the launch),
+// then two counts per block.
+constexpr int kCoopZeroWords = kCoopHdrWords + 4 * 256;
+inline size_t coop_bytes(int64_t N, int mode) {
+  (void)mode;
+  return kCoopZeroWords * 4 + coop_blocks(N) * 2 * 4;
+}
+
+__device__ __forceinline__ bool grid_sync(unsigned int* bar, unsigned int target, unsigned int* status,
+                                          volatile int* s_fail) {
+  __syncthreads();
+  if (threadIdx.x == 0 && !*s_fail) {
+    __threadfence();
+    atomicAdd(bar, 1u);
+    const long long t0 = clock64();
+    while (*reinterpret_cast<volatile unsigned int*>(bar) < target) {
+      if (clock64() - t0 > kGridWaitCycles) {
+        *s_fail = 1;
+        raise_status(status, STATUS_TIMEOUT);
+        break;
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *s_fail == 0;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads) select_coop(CoopArgs a, int64_t N, unsigned int* ws,
+                                                        int32_t* __restrict__ idx, int32_t* __restrict__ count,
+                                                        unsigned int* status) {
+  __shared__ unsigned int sh[256];
+  __shared__ unsigned int s_pref, s_krem;
+  __shared__ volatile int s_fail;
+  __shared__ unsigned int s_sel[kWarps], s_tie[kWarps];
+  const unsigned int G = gridDim.x, b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  unsigned int* bar = ws;
+  unsigned int* hist = ws + kCoopHdrWords;                       // [4][256], top-k only
+  unsigned int* cnt = ws + kCoopZeroWords;                       // [G][2]
+  if (tid == 0) s_fail = 0;
+  const int64_t base = static_cast<int64_t>(b) * kCoopTile + w * (32 * kCoopItems);
+  uint32_t key[kCoopItems];
+  int cls[kCoopItems];
+#pragma unroll
+  for (int it = 0; it < kCoopItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    key[it] = 0u;
+    cls[it] = 0;
+    if (n < N) {
+      if (kMode == kCoopTopk) key[it] = score_key(a.s[n]);
+      else if (kMode == kCoopThresh) cls[it] = a.s[n] >= a.tau ? 1 : 0;
+      else {
+        const int v = a.g[n];
+        cls[it] = (v >= 0 && v < a.K && ((a.act >> v) & 1u)) ? 1 : 0;
+      }
+    }
+  }
+  unsigned int nbar = 0;
+  unsigned int krem = 0;
+  if (kMode == kCoopTopk) {
+    unsigned int prefix = 0;
+    krem = a.k;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      const unsigned int himask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+      sh[tid] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int it = 0; it < kCoopItems; ++it) {
+        const int64_t n = base + it * 32 + lane;
+        if (n < N && (key[it] & himask) == prefix) atomicAdd(&sh[(key[it] >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (sh[tid]) atomicAdd(&hist[pass * 256u + tid], sh[tid]);   // one global histogram per pass
+      if (!grid_sync(bar, ++nbar * G, status, &s_fail)) return;
+      const int bin = 255 - tid;                                  // descending buckets
+      const unsigned int c = __ldcg(&hist[pass * 256u + bin]);
+      unsigned int tot;
+      const unsigned int incl = block_incl_scan(c, &tot);
+      const unsigned int excl = incl - c;
+      if (excl < krem && incl >= krem) {
+        s_pref = prefix | (static_cast<unsigned int>(bin) << shift);
+        s_krem = krem - excl;
+      }
+      __syncthreads();
+      prefix = s_pref;
+      krem = s_krem;
+      __syncthreads();
+    }
+#pragma unroll
+    for (int it = 0; it < kCoopItems; ++it) {
+      const int64_t n = base + it * 32 + lane;
+      cls[it] = n >= N ? 0 : (key[it] > prefix ? 1 : (key[it] == prefix ? 2 : 0));
+    }
+  }
+  // ---- compaction ------------------------------------------------------------------
+  unsigned int msel[kCoopItems], mtie[kCoopItems];
+  unsigned int wsel = 0, wtie = 0;
+#pragma unroll
+  for (int it = 0; it < kCoopItems; ++it) {
+    msel[it] = __ballot_sync(0xffffffffu, cls[it] == 1);
+    mtie[it] = __ballot_sync(0xffffffffu, cls[it] == 2);
+    wsel += __popc(msel[it]);
+    wtie += __popc(mtie[it]);
+  }
+  if (lane == 0) {
+    s_sel[w] = wsel;
+    s_tie[w] = wtie;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    unsigned int bs = 0, bt = 0;
+    for (int i = 0; i < kWarps; ++i) {
+      bs += s_sel[i];
+      bt += s_tie[i];
+    }
+    cnt[2 * b] = bs;
+    cnt[2 * b + 1] = bt;
+  }
+  if (!grid_sync(bar, ++nbar * G, status, &s_fail)) return;
+  // offsets of this block: sums over the blocks before it; the last block also
+  // writes the device-side total
+  unsigned int ps = 0, pt = 0, as = 0, at = 0;
+  for (unsigned int g = tid; g < G; g += kThreads) {
+    const unsigned int cs = __ldcg(&cnt[2 * g]), ct = __ldcg(&cnt[2 * g + 1]);
+    if (g < b) {
+      ps += cs;
+      pt += ct;
+    }
+    as += cs;
+    at += ct;
+  }
+  ps = block_sum(ps);
+  pt = block_sum(pt);
+  as = block_sum(as);
+  at = block_sum(at);
+  if (b == G - 1 && tid == 0) *count = static_cast<int32_t>(as + (at < krem ? at : krem));
+  unsigned int sb = ps, tb = pt;
+  for (int i = 0; i < w; ++i) {
+    sb += s_sel[i];
+    tb += s_tie[i];
+  }
+  const unsigned int lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int it = 0; it < kCoopItems; ++it) {
+    const int64_t n = base + it * 32 + lane;
+    const unsigned int sr = sb + __popc(msel[it] & lt);
+    const unsigned int tr = tb + __popc(mtie[it] & lt);
+    if ((msel[it] >> lane) & 1u) idx[sr + (tr < krem ? tr : krem)] = static_cast<int32_t>(n);
+    else if (((mtie[it] >> lane) & 1u) && tr < krem) idx[sr + tr] = static_cast<int32_t>(n);
+    sb += __popc(msel[it]);
+    tb += __popc(mtie[it]);
+  }
+}
+
+// Max co-resident blocks of a cooperative kernel on the current device (cached).
+template <int kMode>
+int coop_capacity() {
+  static int cap[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cap[dev]) {
+    int per_sm = 0, coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_coop<kMode>, kThreads, 0) != cudaSuccess)
+      return 0;
+    cap[dev] = per_sm * sm_count();
+  }
+  return cap[dev];
+}
+
+// Runs the cooperative path when it applies; returns -1 when it does not.
+template <int kMode>
+int try_coop(const CoopArgs& ca, int64_t N, void* ws, size_t ws_bytes, int32_t* idx, int32_t* count,
+             cudaStream_t st) {
+  const int64_t G = coop_blocks(N);
+  if (G > kCoopMaxBlocks || G > coop_capacity<kMode>() || ws_bytes < coop_bytes(N, kMode)) return -1;
+  int err;
+  unsigned int* status = device_status(&err);
+  if (!status) return err;
+  if (int e = cuda_status(cudaMemsetAsync(ws, 0, kCoopZeroWords * 4, st), "selection: clear barrier")) return e;
+  CoopArgs a = ca;
+  int64_t n = N;
+  unsigned int* w = static_cast<unsigned int*>(ws);
+  void* args[] = {&a, &n, &w, &idx, &count, &status};
+  cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_coop<kMode>),
+                                              dim3(static_cast<unsigned int>(G)), dim3(kThreads), args, 0, st);
+  return cuda_status(e, "selection: cooperative launch");
+}
+
 // ---- host helpers ------------------------------------------------------------------
 struct WsView {
   SelHdr* hdr;
@@ -374,15 +594,25 @@ inline int ncols_for(int op, int K) {
   return 1;
 }
 
-size_t ws_bytes_for(int op, int64_t N, int K) {
+// Minimum workspace: what the multi-launch path needs.
+size_t ws_min_bytes(int op, int64_t N, int K) {
   const int64_t nb = n_blocks(N > 0 ? N : 1);
   return kHdrBytes + 2 * static_cast<size_t>(ncols_for(op, K)) * nb * sizeof(unsigned int);
+}
+
+// Recommended workspace: also enough for the single-launch cooperative path.
+size_t ws_bytes_for(int op, int64_t N, int K) {
+  const size_t classic = ws_min_bytes(op, N, K);
+  size_t coop = 0;
+  if (op != TPS_OP_GROUP && coop_blocks(N > 0 ? N : 1) <= kCoopMaxBlocks)
+    coop = coop_bytes(N > 0 ? N : 1, op == TPS_OP_SELECT ? kCoopTopk : kCoopSched);
+  return classic > coop ? classic : coop;
 }
 
 int check_ws(void* ws, size_t bytes, int op, int64_t N, int K, WsView* v, const char* who) {
   if (!ws) return fail(TPS_ERR_WORKSPACE, "%s: workspace is null", who);
   if (!aligned16(ws)) return fail(TPS_ERR_ALIGN, "%s: workspace must be 16-byte aligned", who);
-  const size_t need = ws_bytes_for(op, N, K);
+  const size_t need = ws_min_bytes(op, N, K);
   if (bytes < need)
     return fail(TPS_ERR_WORKSPACE, "%s: workspace %zu bytes < required %zu", who, bytes, need);
   const int64_t nb = n_blocks(N);
@@ -445,6 +675,12 @@ extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, 
   WsView v;
   if (int e = check_ws(ws, ws_bytes, TPS_OP_SELECT, N, 0, &v, "lipar_select")) return e;
   int e;
+  {
+    CoopArgs ca{score, tau, nullptr, 0u, 0, static_cast<unsigned int>(k)};
+    e = mode == TPS_SELECT_THRESHOLD ? try_coop<kCoopThresh>(ca, N, ws, ws_bytes, idx, count, st)
+                                     : try_coop<kCoopTopk>(ca, N, ws, ws_bytes, idx, count, st);
+    if (e >= 0) return e ? e : ok();
+  }
   if (mode == TPS_SELECT_THRESHOLD) {
     e = run_compact(ThreshCls{score, tau}, N, v, 1, idx, count, st, true);
   } else {
@@ -507,6 +743,11 @@ extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32
   }
   WsView v;
   if (int e = check_ws(ws, ws_bytes, TPS_OP_SCHEDULE, N, K, &v, "lipar_schedule")) return e;
+  {
+    CoopArgs ca{nullptr, 0.f, group, act, K, 0u};
+    const int e = try_coop<kCoopSched>(ca, N, ws, ws_bytes, idx, count, st);
+    if (e >= 0) return e ? e : ok();
+  }
   if (int e = run_compact(SchedCls{group, act, K}, N, v, 1, idx, count, st, true)) return e;
   return ok();
 }

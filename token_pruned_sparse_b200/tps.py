@@ -36,6 +36,7 @@ SIGNATURES = {
     "pruned_attn": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
+    "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
     "tps_workspace_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_last_error": (C.c_char_p, []),
     "tps_check": (_INT, [_P]),
@@ -211,6 +212,15 @@ def scatter_out(o_full, o_act, idx, count, cap=None, stream=None):
     cap = o_act.shape[0] if cap is None else cap
     _chk(lib().scatter_out(_ptr(o_full), _ptr(o_act), _ptr(idx), _ptr(count), cap, N, H, d, _stream(stream)))
     return o_full
+
+
+def hsa_euler_update(x, v_cache, v_fresh, idx, count, dsigma, cap=None, stream=None):
+    """x [N, C] float32 and v_cache [N, C] bf16 updated in place."""
+    N, Cc = x.shape
+    cap = v_fresh.shape[0] if cap is None else cap
+    _chk(lib().hsa_euler_update(_ptr(x), _ptr(v_cache), _ptr(v_fresh), _ptr(idx), _ptr(count), cap, N, Cc,
+                                float(dsigma), _stream(stream)))
+    return x
 
 
 def tps_check(stream=None):
