@@ -35,7 +35,7 @@ __all__ = [
     "f64", "round_bf16", "lipar_score", "select_threshold", "select_topk", "group_split",
     "schedule_groups", "schedule_active", "compact", "kv_sync", "philox4x32_10",
     "philox_words", "renoise_normals", "pruned_attn", "scatter_out", "gather_rows",
-    "attn_flops", "euler_update",
+    "attn_flops", "euler_update", "lse_merge", "lipar_score_motion",
 ]
 
 
@@ -308,6 +308,48 @@ def pruned_attn(q_act, k, v, idx, scale: float, blockmask=None, block: int = 128
             o[c0:c0 + len(r), hi] = np.where(ok[:, None], O / np.where(ok, l, 1.0)[:, None], 0.0)
             lse[c0:c0 + len(r), hi] = np.where(ok, mx + np.log(np.where(ok, l, 1.0)), -np.inf)
     return o, lse
+
+
+def lse_merge(o1, lse1, o2, lse2):
+    """[LIPAR] 2.C (Spanish summary, M-degree approximation): the attention of
+    removed tokens is recovered through a log-sum-exp based combination. Reading:
+    attention over a key set split into two disjoint parts is assembled exactly
+    from the two partial results. With w_i = exp(lse_i):
+        o = (w1 * o1 + w2 * o2) / (w1 + w2),   lse = log(w1 + w2).
+    A part with lse = -inf (no key) contributes nothing; two empty parts give
+    o = 0, lse = -inf. Returns float64 (o [A, H, d], lse [A, H])."""
+    O1, O2 = f64(o1), f64(o2)
+    L1, L2 = f64(lse1), f64(lse2)
+    m = np.maximum(L1, L2)
+    ok = np.isfinite(m)
+    mm = np.where(ok, m, 0.0)
+    a = np.where(ok, np.exp(L1 - mm), 0.0)
+    b = np.where(ok, np.exp(L2 - mm), 0.0)
+    den = np.where(ok, a + b, 1.0)
+    o = (a[..., None] * O1 + b[..., None] * O2) / den[..., None]
+    return np.where(ok[..., None], o, 0.0), np.where(ok, m + np.log(den), -np.inf)
+
+
+def lipar_score_motion(x, L: int) -> np.ndarray:
+    """[LIPAR] 2.B (both summaries): motion detection with short- and long-term
+    differences makes the pruning mask robust. Reading: a token is pruned only
+    when BOTH its short-term change (against frame f-1) and its long-term change
+    (against the key frame max(f-L, 0)) are small, i.e. the score is
+        s(f, p) = max(s_short(f, p), s_long(f, p)),
+    each a relative L1 change as in lipar_score; frame 0 is +inf. L >= 1
+    (L = 1 is the plain inter-frame score)."""
+    X = f64(x)
+    F, HW, C = X.shape
+    s = np.full((F, HW), np.inf)
+    for f in range(1, F):
+        parts = []
+        for r in (f - 1, max(f - L, 0)):
+            num = np.abs(X[f] - X[r]).sum(axis=1)
+            den = np.abs(X[r]).sum(axis=1)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                parts.append(np.where(den > 0, num / np.where(den > 0, den, 1.0), np.where(num > 0, np.inf, 0.0)))
+        s[f] = np.maximum(parts[0], parts[1])
+    return s.reshape(-1)
 
 
 def attn_flops(A: int, N: int, H: int, d: int, keys_per_query=None) -> float:

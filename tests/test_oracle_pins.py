@@ -356,3 +356,37 @@ def test_euler_closed_forms():
         xi, vc = O.euler_update(x, vc, v[act], act, sig[i + 1] - sig[i])
         x = torch.from_numpy(xi)
     np.testing.assert_array_equal(x.numpy(), x0.double().numpy() + (sig[T] - sig[0]) * v.double().numpy())
+
+
+# --------------------------------------------- attention-recovery LSE merge ---
+def test_lse_merge_equals_attention_over_all_keys():
+    """Attention over keys [0, N) equals the merge of attention over [0, M) and
+    [M, N) (the merge is checked against the attention definition, not itself)."""
+    N, M, A, H, d = 300, 111, 40, 2, 64
+    q = synth.gaussian_bf16((A, H, d), 61)
+    k = synth.gaussian_bf16((N, H, d), 62)
+    v = synth.gaussian_bf16((N, H, d), 63)
+    idx = np.arange(A)
+    o_all, l_all = O.pruned_attn(q, k, v, idx, 0.2)
+    o1, l1 = O.pruned_attn(q, k[:M], v[:M], idx, 0.2)
+    o2, l2 = O.pruned_attn(q, k[M:], v[M:], idx, 0.2)
+    o, l = O.lse_merge(o1, l1, o2, l2)
+    np.testing.assert_allclose(o, o_all, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l, l_all, rtol=1e-13)
+    # an empty part is the identity; two empty parts give 0 / -inf
+    e_o, e_l = np.zeros_like(o1), np.full_like(l1, -np.inf)
+    o3, l3 = O.lse_merge(o1, l1, e_o, e_l)
+    np.testing.assert_array_equal(o3, o1)
+    np.testing.assert_array_equal(l3, l1)
+    o4, l4 = O.lse_merge(e_o, e_l, e_o, e_l)
+    assert not o4.any() and np.all(np.isneginf(l4))
+
+
+# ------------------------------------------------------ motion-robust score ---
+def test_motion_score_worked_and_reductions():
+    g = _gold("motion_worked.json")
+    s = O.lipar_score_motion(np.array(g["x"], float), g["L"])
+    assert list(s) == [_num(v) for v in g["score"]]
+    x = synth.gaussian_bf16((6, 30, 16), 71)
+    np.testing.assert_array_equal(O.lipar_score_motion(x, 1), O.lipar_score(x))   # L = 1: plain score
+    assert np.all(O.lipar_score_motion(x, 3) >= O.lipar_score(x))                 # never below short-term
