@@ -410,6 +410,8 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     x_frames = rnd(cfg.video.F, cfg.video.HW, C)
     t = _time(lambda: tps.lipar_score(x_frames, out=score), flush)
     stages["score_interframe"] = (t, N * (2 * C + 4))
+    t = _time(lambda: tps.lipar_score_motion(x_frames, 4, out=score), flush)
+    stages["score_motion_L4"] = (t, N * (2 * C + 4))
     ws = tps.workspace(tps.OP_SELECT, N, 0, dev)
     idx_all = torch.empty(N, dtype=torch.int32, device=dev)
     cnt = torch.empty(1, dtype=torch.int32, device=dev)
@@ -441,6 +443,11 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     o_full, o_act = rnd(N, H, d), rnd(A, H, d)
     t = _time(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
     stages["scatter_out"] = (t, 2 * R * A)
+    # attention-recovery merge of two partial results for the A active rows
+    lse_a, lse_b, lse_o = (torch.randn(A, H, generator=g, device=dev) for _ in range(3))
+    o_b = rnd(A, H, d)
+    t = _time(lambda: tps.attn_lse_merge(o_act, lse_a, o_b, lse_b, cnt, o=o_act, lse=lse_o), flush)
+    stages["lse_merge"] = (t, 3 * R * A + 3 * 4 * H * A)
     # cached Euler update (HSA 2.3): fp32 state [N, C], bf16 velocity cache
     xs = torch.randn(N, C, generator=g, device=dev, dtype=torch.float32)
     vcache = rnd(N, C)

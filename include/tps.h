@@ -82,6 +82,15 @@ typedef void*    tps_stream; /* cudaStream_t                          */
 TPS_API int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame,
                 int64_t F, int64_t HW, int64_t C, float* score, tps_stream stream);
 
+/* ---- motion-robust inter-frame score ([LIPAR] 2.B: motion detection with
+ * short- and long-term differences) ---------------------------------------------
+ * s(f, p) = max(rel-L1 of x[f,p] vs x[f-1,p], rel-L1 of x[f,p] vs x[max(f-L,0),p]),
+ * frame 0 = +inf; a token is pruned only when both changes are small. L >= 1
+ * (L = 1 is lipar_score's inter-frame mode). x [F, HW, C] bf16, C in {64, 128};
+ * score float32 [F*HW]. */
+TPS_API int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int64_t C, int L, float* score,
+                               tps_stream stream);
+
 /* ---- steps 2-3: active set and compaction ([LIPAR] 2.B; [HSA] 2.1) ---------
  * mode TPS_SELECT_THRESHOLD: active iff score >= tau (a token below tau is
  *   redundant and pruned). NaN is never active.
@@ -193,6 +202,18 @@ TPS_API int pruned_attn_mma(const tps_bf16* q_act, const tps_bf16* k, const tps_
                     const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H,
                     int d, float scale, const uint8_t* blockmask, int block, tps_bf16* o_act,
                     float* lse, tps_stream stream);
+
+/* ---- attention-recovery merge ([LIPAR] 2.C, log-sum-exp recovery) -------------
+ * Exact merge of two attention results over DISJOINT key sets (e.g. two
+ * pruned_attn calls over two key ranges): with w_i = exp(lse_i),
+ *   o = (w1 o1 + w2 o2) / (w1 + w2),  lse = log(w1 + w2)   (fp32, bf16 output).
+ * A part with lse = -inf contributes nothing; both -inf give o = 0, lse = -inf.
+ * o1, o2, o bf16 [cap, H, d]; lse1, lse2, lse float32 [cap, H]; rows
+ * j >= min(*count, cap) untouched. o may alias o1 or o2; lse (may be NULL)
+ * must not alias lse1 / lse2. d in {64, 128}. */
+TPS_API int attn_lse_merge(const tps_bf16* o1, const float* lse1, const tps_bf16* o2, const float* lse2,
+                           const int32_t* count, int64_t cap, int H, int d, tps_bf16* o, float* lse,
+                           tps_stream stream);
 
 /* ---- step 6: restoration ([LIPAR] Dutch summary 2.D) -------------------------
  * o_full[idx[j]] = o_act[j] for j < min(*count, cap); every other row of

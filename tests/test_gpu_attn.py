@@ -247,3 +247,49 @@ def test_hsa_steps_with_renoise_sampled(impl):
                                        1 / math.sqrt(d), rows=rows)
         _check(o_act[:, torch.from_numpy(heads)].cpu(), lse[:, torch.from_numpy(heads)].cpu().numpy(),
                o_ref, lse_ref, rows=rows)
+
+
+# ----------------------------------------------- attention-recovery merge ---
+def test_lse_merge_parity_and_empty_parts():
+    A, H, d = 777, 3, 128
+    o1 = synth.gaussian_bf16((A, H, d), 81)
+    o2 = synth.gaussian_bf16((A, H, d), 82)
+    rng = np.random.default_rng(83)
+    l1 = torch.from_numpy((rng.standard_normal((A, H)) * 3).astype(np.float32))
+    l2 = torch.from_numpy((rng.standard_normal((A, H)) * 3).astype(np.float32))
+    l1[::7] = -np.inf
+    l2[::11] = -np.inf
+    cnt = torch.tensor([A], dtype=torch.int32, device=DEV)
+    lse = torch.empty((A, H), device=DEV)
+    o = tps.attn_lse_merge(o1.to(DEV), l1.to(DEV), o2.to(DEV), l2.to(DEV), cnt, lse=lse)
+    o_ref, l_ref = O.lse_merge(o1, l1, o2, l2)
+    g = o.cpu().double().numpy()
+    assert np.all(np.abs(g - o_ref) <= 2.0 ** -8 * np.abs(o_ref) + 1e-6)     # one bf16 rounding
+    lg = lse.cpu().numpy()
+    assert np.array_equal(np.isneginf(lg), np.isneginf(l_ref))
+    fin = np.isfinite(l_ref)
+    np.testing.assert_allclose(lg[fin], l_ref[fin], rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_split_key_attention_merges_to_full(impl):
+    """Attention over keys [0, M) and [M, N) by two calls, merged with
+    attn_lse_merge, equals attention over all N keys (oracle)."""
+    N, M, A, H, d = 3000, 1234, 500, 2, 128
+    q = synth.gaussian_bf16((A, H, d), 91)
+    k = synth.gaussian_bf16((N, H, d), 92)
+    v = synth.gaussian_bf16((N, H, d), 93)
+    idx = np.sort(np.random.default_rng(94).choice(N, A, replace=False))
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    di = torch.from_numpy(idx.astype(np.int32)).to(DEV)
+    dc = torch.tensor([A], dtype=torch.int32, device=DEV)
+    fn = getattr(tps, impl)
+    o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
+    l1, l2 = torch.empty((A, H), device=DEV), torch.empty((A, H), device=DEV)
+    fn(qd, kd[:M], vd[:M], di, dc, 0.25, o_act=o1, lse=l1)
+    fn(qd, kd[M:], vd[M:], di, dc, 0.25, o_act=o2, lse=l2)
+    lse = torch.empty((A, H), device=DEV)
+    o = tps.attn_lse_merge(o1, l1, o2, l2, dc, lse=lse)
+    tps.tps_check()
+    o_ref, l_ref = O.pruned_attn(q, k, v, idx, 0.25)
+    _check(o.cpu(), lse.cpu().numpy(), o_ref, l_ref)

@@ -148,3 +148,15 @@ def test_schedule_ignores_out_of_range_groups():
     g = torch.tensor([0, 1, 2, -1, 5, 1, 0, 127], dtype=torch.int8)
     idx, cnt = tps.lipar_schedule(g.to(DEV), 3, [4, 2, 1], 4, 0, 0)
     assert np.array_equal(_idx(idx, cnt), O.schedule_active(g.numpy(), 3, [4, 2, 1], 4, 0, 0))
+
+
+# -------------------------------------------------- motion-robust score -----
+@pytest.mark.parametrize("name", ["tiny", "mid", "block"])
+@pytest.mark.parametrize("L", [1, 3, 8])
+def test_score_motion(name, L):
+    cfg, xb, _ = frame_case(name)
+    s = tps.lipar_score_motion(xb.to(DEV), L).cpu().numpy()
+    ref = O.lipar_score_motion(xb, L)
+    assert np.array_equal(np.isinf(s), np.isinf(ref))
+    fin = np.isfinite(ref)
+    np.testing.assert_allclose(s[fin], ref[fin], rtol=_rtol(cfg.video.C), atol=0)

@@ -116,8 +116,83 @@ void launch_score(const uint16_t* x, const uint16_t* xr, const uint16_t* xp, int
   score_kernel<L, kV><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
 }
 
+// Motion-robust inter-frame score ([LIPAR] 2.B, short- and long-term
+// differences): s = max(rel-L1 vs frame f-1, rel-L1 vs key frame max(f-L, 0)),
+// frame 0 = +inf. Same lane layout as score_kernel; three rows per token (the
+// two references were read moments before by other warps and come from L2).
+template <int L, int kV>
+__global__ void __launch_bounds__(256) score_motion_kernel(const uint16_t* __restrict__ x, int64_t HW, int64_t N,
+                                                           int Lkey, float* __restrict__ score) {
+  constexpr int kTokPerWarp = 32 / L;
+  constexpr int C = kV * 8;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & (L - 1);
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += nwarps * kTokPerWarp) {
+    const int64_t t = w0 + lane / L;
+    const bool valid = t < N;
+    const int64_t f = valid ? t / HW : 0;
+    const bool first = f == 0;
+    float n1 = 0.f, d1 = 0.f, n2 = 0.f, d2 = 0.f;
+    if (valid && !first) {
+      const int64_t fl = f - Lkey > 0 ? f - Lkey : 0;
+      const uint16_t* cur = x + t * C;
+      const uint16_t* r1 = x + (t - HW) * C;
+      const uint16_t* r2 = x + (t - (f - fl) * HW) * C;
+#pragma unroll
+      for (int v = sub; v < kV; v += L) {
+        const uint4 a = ld16(cur + v * 8), b = ld16(r1 + v * 8), c = ld16(r2 + v * 8);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
+          const float p0 = bf16lo(bw[i]), p1 = bf16hi(bw[i]);
+          const float k0 = bf16lo(cw[i]), k1 = bf16hi(cw[i]);
+          n1 += fabsf(c0 - p0) + fabsf(c1 - p1);
+          d1 += fabsf(p0) + fabsf(p1);
+          n2 += fabsf(c0 - k0) + fabsf(c1 - k1);
+          d2 += fabsf(k0) + fabsf(k1);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) {
+      n1 += __shfl_xor_sync(0xffffffffu, n1, o);
+      d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+      n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+      d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+    }
+    if (valid && sub == 0) {
+      auto ratio = [](float n, float d) { return d > 0.f ? n / d : (n > 0.f ? INFINITY : 0.f); };
+      score[t] = first ? INFINITY : fmaxf(ratio(n1, d1), ratio(n2, d2));
+    }
+  }
+}
+
 }  // namespace
 }  // namespace tps
+
+extern "C" int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int64_t C, int L, float* score,
+                                  tps_stream stream) {
+  using namespace tps;
+  if (!x || !score) return fail(TPS_ERR_INVALID_ARG, "lipar_score_motion: x and score must be non-null");
+  if (F < 1 || HW < 1 || F > (INT64_C(1) << 31) / HW) return fail(TPS_ERR_SHAPE, "lipar_score_motion: bad F/HW");
+  if (C != 64 && C != 128) return fail(TPS_ERR_SHAPE, "lipar_score_motion: C=%lld must be 64 or 128", (long long)C);
+  if (L < 1) return fail(TPS_ERR_INVALID_ARG, "lipar_score_motion: L=%d must be >= 1", L);
+  if (!aligned16(x)) return fail(TPS_ERR_ALIGN, "lipar_score_motion: x must be 16-byte aligned");
+  const int64_t N = F * HW;
+  constexpr int kThreads = 256;
+  const int64_t tok_per_block = (kThreads / 32) * 4;
+  int64_t blocks = (N + tok_per_block - 1) / tok_per_block;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (C == 128) score_motion_kernel<8, 16><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, HW, N, L, score);
+  else score_motion_kernel<8, 8><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, HW, N, L, score);
+  if (int e = launch_status("lipar_score_motion")) return e;
+  return ok();
+}
 
 extern "C" int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame,
                            int64_t F, int64_t HW, int64_t C, float* score, tps_stream stream) {

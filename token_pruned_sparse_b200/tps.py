@@ -37,6 +37,8 @@ SIGNATURES = {
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
     "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
+    "lipar_score_motion": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P]),
+    "attn_lse_merge": (_INT, [_P, _P, _P, _P, _P, _I64, _INT, _INT, _P, _P, _P]),
     "tps_workspace_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_last_error": (C.c_char_p, []),
     "tps_check": (_INT, [_P]),
@@ -221,6 +223,24 @@ def hsa_euler_update(x, v_cache, v_fresh, idx, count, dsigma, cap=None, stream=N
     _chk(lib().hsa_euler_update(_ptr(x), _ptr(v_cache), _ptr(v_fresh), _ptr(idx), _ptr(count), cap, N, Cc,
                                 float(dsigma), _stream(stream)))
     return x
+
+
+def lipar_score_motion(x, L, out=None, stream=None):
+    F, HW, Cc = x.shape
+    if out is None:
+        out = torch.empty(F * HW, dtype=torch.float32, device=x.device)
+    _chk(lib().lipar_score_motion(_ptr(x), F, HW, Cc, int(L), _ptr(out), _stream(stream)))
+    return out
+
+
+def attn_lse_merge(o1, lse1, o2, lse2, count, o=None, lse=None, cap=None, stream=None):
+    A, H, d = o1.shape
+    cap = A if cap is None else cap
+    if o is None:
+        o = torch.empty_like(o1)
+    _chk(lib().attn_lse_merge(_ptr(o1), _ptr(lse1), _ptr(o2), _ptr(lse2), _ptr(count), cap, H, d, _ptr(o),
+                              _ptr(lse), _stream(stream)))
+    return o
 
 
 def tps_check(stream=None):
