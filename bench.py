@@ -264,8 +264,22 @@ def keep_sweep(dev, attn, reps=5):
                 ms.append(a.elapsed_time(b))
         t = float(np.median(ms))
         fl = 4.0 * d * H * A * N
+        # the same call through pruned_attn_ws (key-range splits when the grid is thin)
+        ws, nws = tps.attn_workspace(A, N, H, d, dev)
+        ms = []
+        for i in range(reps + 2):
+            flush_l2(flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            tps.pruned_attn_ws(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o, ws=ws)
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                ms.append(a.elapsed_time(b))
+        tw = float(np.median(ms))
         out.append({"keep": r, "active": A, "attn_ms": round(t, 4), "tflops": round(fl / t / 1e9, 1),
-                    "active_tokens_per_s": round(A / t * 1e3, 1)})
+                    "active_tokens_per_s": round(A / t * 1e3, 1), "attn_ws_ms": round(tw, 4),
+                    "tflops_ws": round(fl / tw / 1e9, 1), "ws_bytes": nws})
     return out
 
 

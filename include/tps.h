@@ -195,6 +195,20 @@ TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16
                 float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
                 tps_stream stream);
 
+/* Same contract as pruned_attn, with a caller workspace that lets a launch
+ * that would fill the GPU poorly (few query tiles x heads, e.g. a low keep
+ * ratio) run as S <= 4 key-range splits in one grid plus an S-way
+ * log-sum-exp merge (dense mode only). ws: device memory of
+ * tps_attn_workspace_size(cap, N, H, d) bytes (0 when no split is chosen),
+ * 16-byte aligned; with a smaller or NULL workspace the call runs unsplit.
+ * Results agree with pruned_attn within the attention tolerance (the merge
+ * rounds to bf16 once, from fp32 partials). */
+TPS_API int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
+                           const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
+                           float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
+                           void* ws, size_t ws_bytes, tps_stream stream);
+TPS_API size_t tps_attn_workspace_size(int64_t cap, int64_t N, int H, int d);
+
 /* Same contract as pruned_attn, computed with the legacy warp-level
  * mma.sync tensor-core path (kept as the baseline the tcgen05 kernel is
  * measured against). */

@@ -293,3 +293,47 @@ def test_split_key_attention_merges_to_full(impl):
     tps.tps_check()
     o_ref, l_ref = O.pruned_attn(q, k, v, idx, 0.25)
     _check(o.cpu(), lse.cpu().numpy(), o_ref, l_ref)
+
+
+# --------------------------------------------- split-key attention (ws) -----
+@pytest.mark.parametrize("N,A,H,d", [(3000, 300, 2, 128), (2600, 200, 3, 64), (5000, 1, 1, 128)])
+def test_attn_ws_split_matches_oracle(N, A, H, d):
+    """Few query tiles x heads: pruned_attn_ws splits the key range (its
+    workspace size is non-zero) and the merged result matches the oracle."""
+    assert tps.lib().tps_attn_workspace_size(A, N, H, d) > 0
+    q = synth.gaussian_bf16((A, H, d), N + 7)
+    k = synth.gaussian_bf16((N, H, d), N + 8)
+    v = synth.gaussian_bf16((N, H, d), N + 9)
+    idx = np.sort(np.random.default_rng(A).choice(N, A, replace=False))
+    for scale in (1 / math.sqrt(d), 0.35):
+        qd = q.to(DEV)
+        o = torch.full_like(qd, 7.0)
+        lse = torch.full((A, H), 7.0, device=DEV)
+        tps.pruned_attn_ws(qd, k.to(DEV), v.to(DEV), torch.from_numpy(idx.astype(np.int32)).to(DEV),
+                           torch.tensor([A], dtype=torch.int32, device=DEV), scale, o_act=o, lse=lse)
+        tps.tps_check()
+        o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
+        _check(o.cpu(), lse.cpu().numpy(), o_ref, lse_ref)
+
+
+def test_attn_ws_wan_keep10_sampled():
+    """The Wan-like layer at keep 10% (3276 x 32760 keys, 12 heads): split path
+    vs the oracle on sampled rows."""
+    Q, K, V = qkv("wan")
+    N, H, d = Q.shape
+    idx = oracle_idx("wan", 0)
+    A = len(idx)
+    assert tps.lib().tps_attn_workspace_size(A, N, H, d) > 0
+    o = torch.empty((A, H, d), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((A, H), device=DEV)
+    tps.pruned_attn_ws(Q[idx].to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV),
+                       torch.tensor([A], dtype=torch.int32, device=DEV), 1 / math.sqrt(d), o_act=o, lse=lse)
+    tps.tps_check()
+    rows = _sample(A, 192, 5)
+    o_ref, lse_ref = O.pruned_attn(Q[idx], K, V, idx, 1 / math.sqrt(d), rows=rows)
+    _check(o.cpu(), lse.cpu().numpy(), o_ref, lse_ref, rows=rows)
+
+
+def test_attn_ws_no_split_when_grid_is_full():
+    # 24 x 12 = 288 CTAs fill 148 SMs twice at 97%: no split, no workspace
+    assert tps.lib().tps_attn_workspace_size(6084, 20280, 12, 128) == 0

@@ -81,6 +81,9 @@ struct TcParams {
   AttnArgs a;
   float scale_log2;
   unsigned int* status;
+  int nsplit;          // key-range splits (blockIdx.z); 1 = whole key range
+  float* o_part;       // nsplit > 1: normalised partial outputs, fp32 [nsplit][cap][H][D]
+  float* lse_part;     // nsplit > 1: partial log-sum-exp, fp32 [nsplit][cap][H]
 };
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -126,7 +129,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint16_t* sList = reinterpret_cast<uint16_t*>(gbase + L::kList);
   const uint32_t bar0 = sbase + L::kBar;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const int nkt = static_cast<int>((p.N + kBN - 1) / kBN);   // key tiles = key blocks
+  const int nkt_all = static_cast<int>((p.N + kBN - 1) / kBN);   // key tiles = key blocks
+  // split z of nsplit (dense mode only) covers key tiles [kt0, kt0 + nkt)
+  const int kt0 = static_cast<int>((static_cast<int64_t>(nkt_all) * blockIdx.z) / prm.nsplit);
+  const int nkt = static_cast<int>((static_cast<int64_t>(nkt_all) * (blockIdx.z + 1)) / prm.nsplit) - kt0;
 
   // ---- setup: barriers, TMEM, key-tile list ---------------------------------------------
   if (tid == 0) {
@@ -185,7 +191,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = s_tmem;
   auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
-  auto tile_kb = [&](int j) -> int { return p.bm ? static_cast<int>(sList[j]) : j; };
+  auto tile_kb = [&](int j) -> int { return p.bm ? static_cast<int>(sList[j]) : kt0 + j; };
 
   if (warp == kTmaWarp) {
     // ================================ TMA producer =====================================
@@ -365,24 +371,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_after();
     if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
+      if (prm.nsplit > 1) {
+        // partial result of this key range: normalised fp32 row + its log-sum-exp
+        const int64_t prow = (static_cast<int64_t>(blockIdx.z) * p.cap + row) * p.H + h;
+        float4* frow = reinterpret_cast<float4*>(prm.o_part + prow * D);
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        float o[32];
-        if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
-        else
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
+          else
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
-        if (valid) {
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          if (valid) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
-                                         pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                         pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                         pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+            for (int q = 0; q < 8; ++q)
+              frow[c / 4 + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
+          }
         }
+        if (valid) prm.lse_part[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      } else {
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
+  #pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
+          else
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          if (valid) {
+  #pragma unroll
+            for (int q = 0; q < 4; ++q)
+              orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
+                                           pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                           pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                           pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+          }
+        }
+        if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
-      if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 
@@ -433,7 +459,7 @@ int make_map(EncodeTiled enc, CUtensorMap* m, const void* base, int64_t rows, in
 }
 
 template <int D>
-int launch(const AttnArgs& a, cudaStream_t st) {
+int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr) {
   if (a.cap == 0) return TPS_OK;
   EncodeTiled enc;
   if (int e = get_encoder(&enc)) return e;
@@ -453,14 +479,84 @@ int launch(const AttnArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_status(e, "pruned_attn: smem attribute");
     attr_done[dev] = true;
   }
-  TcParams prm{a, a.scale * kLog2e, status};
-  dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H));
+  TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part};
+  dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
+            static_cast<unsigned int>(nsplit));
   attn_tc_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   return launch_status("pruned_attn");
 }
 
+// Key-range splits for a launch that would fill the GPU poorly: one pass of
+// ceil(cap/256) x H CTAs that leaves most of its last wave empty (e.g. 156
+// CTAs on 148 SMs) runs as S <= 4 key-range splits in one grid, followed by an
+// S-way log-sum-exp merge. Dense mode only; >= 4 key tiles per split.
+int choose_split(int64_t cap, int H, int64_t N, bool masked) {
+  if (masked) return 1;
+  const int64_t units = ((cap + kQT * kBM - 1) / (kQT * kBM)) * H;
+  const int64_t sms = sm_count();
+  const int64_t nkt = (N + kBN - 1) / kBN;
+  auto eff = [&](int64_t s) {
+    const int64_t u = units * s;
+    return static_cast<double>(u) / static_cast<double>(((u + sms - 1) / sms) * sms);
+  };
+  if (units <= 0 || eff(1) >= 0.9) return 1;
+  int best = 1;
+  double be = eff(1);
+  for (int s = 2; s <= 4; ++s) {
+    if (nkt < 4 * s) break;
+    const double e = eff(s);
+    if (e > be + 0.02) {
+      best = s;
+      be = e;
+    }
+  }
+  return best;
+}
+
+size_t split_ws_bytes(int nsplit, int64_t cap, int H, int d) {
+  if (nsplit <= 1) return 0;
+  const size_t o = static_cast<size_t>(nsplit) * cap * H * d * sizeof(float);
+  return (o + 255) / 256 * 256 + static_cast<size_t>(nsplit) * cap * H * sizeof(float);
+}
+
 }  // namespace
+
+// S-way merge of the split partials (merge.cu).
+int merge_split_parts(const float* o_part, const float* lse_part, int nsplit, const int32_t* count, int64_t cap,
+                      int H, int d, uint16_t* o, float* lse, cudaStream_t st);
+
 }  // namespace tps
+
+extern "C" size_t tps_attn_workspace_size(int64_t cap, int64_t N, int H, int d) {
+  using namespace tps;
+  if (cap <= 0 || N <= 0 || H <= 0 || (d != 64 && d != 128)) return 0;
+  return split_ws_bytes(choose_split(cap, H, N, false), cap, H, d);
+}
+
+extern "C" int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
+                              const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,
+                              const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse, void* ws,
+                              size_t ws_bytes, tps_stream stream) {
+  using namespace tps;
+  AttnArgs a;
+  if (int e = attn_validate("pruned_attn_ws", q_act, k, v, idx, count, cap, N, H, d, scale, blockmask, block, o_act,
+                            lse, &a))
+    return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int S = choose_split(cap, H, N, blockmask != nullptr);
+  const size_t need = split_ws_bytes(S, cap, H, d);
+  if (S <= 1 || !ws || ws_bytes < need || !aligned16(ws)) {   // no split possible or needed
+    const int e = d == 64 ? launch<64>(a, st) : launch<128>(a, st);
+    return e ? e : ok();
+  }
+  float* o_part = static_cast<float*>(ws);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                             (static_cast<size_t>(S) * cap * H * d * sizeof(float) + 255) / 256 * 256);
+  int e = d == 64 ? launch<64>(a, st, S, o_part, lse_part) : launch<128>(a, st, S, o_part, lse_part);
+  if (e) return e;
+  e = merge_split_parts(o_part, lse_part, S, count, cap, H, d, o_act, lse, st);
+  return e ? e : ok();
+}
 
 extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
                            const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,

@@ -47,7 +47,65 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const uint4* __restrict_
   }
 }
 
+// S-way merge of the fp32 partials written by split-key attention:
+// o = sum_s w_s o_s / sum_s w_s, w_s = exp(lse_s - max_s lse_s).
+template <int kVpd>
+__global__ void __launch_bounds__(256) merge_parts_kernel(const float4* __restrict__ op,
+                                                          const float* __restrict__ lp, int S, int64_t cap, int H,
+                                                          const int32_t* count, uint4* __restrict__ o,
+                                                          float* __restrict__ l) {
+  const int64_t rows = active_count(count, cap);
+  const int64_t total = rows * H * kVpd;
+  const int64_t plane = cap * H;                       // (row, head) pairs per split
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t f = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; f < total; f += stride) {
+    const int64_t rh = f / kVpd;
+    float m = -INFINITY;
+    for (int s = 0; s < S; ++s) m = fmaxf(m, lp[s * plane + rh]);
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    float lse = -INFINITY;
+    if (m != -INFINITY) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float sum = 0.f;
+      for (int s = 0; s < S; ++s) {
+        const float w = expf(lp[s * plane + rh] - m);
+        const float4 a = op[(s * plane * kVpd + f) * 2], b = op[(s * plane * kVpd + f) * 2 + 1];
+        acc[0] = fmaf(w, a.x, acc[0]);
+        acc[1] = fmaf(w, a.y, acc[1]);
+        acc[2] = fmaf(w, a.z, acc[2]);
+        acc[3] = fmaf(w, a.w, acc[3]);
+        acc[4] = fmaf(w, b.x, acc[4]);
+        acc[5] = fmaf(w, b.y, acc[5]);
+        acc[6] = fmaf(w, b.z, acc[6]);
+        acc[7] = fmaf(w, b.w, acc[7]);
+        sum += w;
+      }
+      const float inv = 1.f / sum;
+      out = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                       pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+      lse = m + logf(sum);
+    }
+    o[f] = out;
+    if (l && f % kVpd == 0) l[rh] = lse;
+  }
+}
+
 }  // namespace
+
+int merge_split_parts(const float* o_part, const float* lse_part, int nsplit, const int32_t* count, int64_t cap,
+                      int H, int d, uint16_t* o, float* lse, cudaStream_t st) {
+  const int64_t vecs = cap * H * (d / 8);
+  int64_t grid = (vecs + 255) / 256;
+  const int64_t maxg = static_cast<int64_t>(sm_count()) * 16;
+  if (grid > maxg) grid = maxg;
+  if (grid < 1) return TPS_OK;
+  const auto* op = reinterpret_cast<const float4*>(o_part);
+  auto* oo = reinterpret_cast<uint4*>(o);
+  if (d == 128) merge_parts_kernel<16><<<static_cast<unsigned>(grid), 256, 0, st>>>(op, lse_part, nsplit, cap, H, count, oo, lse);
+  else merge_parts_kernel<8><<<static_cast<unsigned>(grid), 256, 0, st>>>(op, lse_part, nsplit, cap, H, count, oo, lse);
+  return launch_status("pruned_attn_ws: merge");
+}
+
 }  // namespace tps
 
 extern "C" int attn_lse_merge(const tps_bf16* o1, const float* lse1, const tps_bf16* o2, const float* lse2,

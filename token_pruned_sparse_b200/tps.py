@@ -34,6 +34,9 @@ SIGNATURES = {
     "tps_gather_rows": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "kv_sync": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P, _P, _P]),
     "pruned_attn": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
+    "pruned_attn_ws": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P,
+                              C.c_size_t, _P]),
+    "tps_attn_workspace_size": (C.c_size_t, [_I64, _I64, _INT, _INT]),
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
     "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
@@ -201,6 +204,25 @@ def _attn(fn, q_act, k, v, idx, count, scale, blockmask, block, o_act, lse, cap,
 def pruned_attn(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None,
                 cap=None, stream=None):
     return _attn(lib().pruned_attn, q_act, k, v, idx, count, scale, blockmask, block, o_act, lse, cap, stream)
+
+
+def attn_workspace(cap, N, H, d, device=None):
+    n = int(lib().tps_attn_workspace_size(cap, N, H, d))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda"), n
+
+
+def pruned_attn_ws(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None, cap=None,
+                   ws=None, stream=None):
+    N, H, d = k.shape
+    cap = q_act.shape[0] if cap is None else cap
+    if o_act is None:
+        o_act = torch.empty_like(q_act)
+    if ws is None:
+        ws, _ = attn_workspace(cap, N, H, d, q_act.device)
+    _chk(lib().pruned_attn_ws(_ptr(q_act), _ptr(k), _ptr(v), _ptr(idx), _ptr(count), cap, N, H, d, float(scale),
+                              _ptr(blockmask), int(block), _ptr(o_act), _ptr(lse), _ptr(ws), ws.numel(),
+                              _stream(stream)))
+    return o_act
 
 
 def pruned_attn_mma(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None,
