@@ -400,17 +400,20 @@ def executed_key_tiles(idx: np.ndarray, N: int, nb_mask=None, rows_per_cta=256):
     return tot, ctas
 
 
-def config_sweep(dev, peak_tflops, hbm_gbs):
+def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     """Kernel-level numbers on the larger configs (inputs resident in HBM, L2
     flushed before every timed call). Attention: algorithmic FLOPs (4*d per
     query-key-head pair over allowed keys) and executed FLOPs (padded 256-row
     query tiles x whole 128-key tiles that the kernel runs). Memory-bound
-    stages: algorithmic bytes / time against the measured HBM copy peak."""
+    stages: algorithmic bytes / time against the measured HBM copy peak.
+    stages_once: each HSA stage runs exactly once and attention is skipped
+    (the launch sequence a per-kernel DRAM-counter capture wants)."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
     g.manual_seed(4)
     flush = L2Flush(dev)
     out = {}
+    timer = (lambda fn, fl, reps=1, warm=0: _time(fn, fl, reps=1, warm=0)) if stages_once else _time
     # ---- HSA: 33 x 45x80 = 118800 tokens, 24 heads, d = 128 -----------------------------
     cfg = synth.CONFIGS["hsa"]
     N, H, d, C = cfg.video.N, cfg.H, cfg.d, cfg.video.C
@@ -419,28 +422,28 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     v_prev, v_cur = rnd(cfg.video.F, cfg.video.HW, C), rnd(cfg.video.F, cfg.video.HW, C)
     score = torch.empty(N, dtype=torch.float32, device=dev)
     stages = {}
-    t = _time(lambda: tps.lipar_score(v_cur, v_prev, out=score), flush)
+    t = timer(lambda: tps.lipar_score(v_cur, v_prev, out=score), flush)
     stages["score_interstep"] = (t, N * (4 * C + 4))
     x_frames = rnd(cfg.video.F, cfg.video.HW, C)
-    t = _time(lambda: tps.lipar_score(x_frames, out=score), flush)
+    t = timer(lambda: tps.lipar_score(x_frames, out=score), flush)
     stages["score_interframe"] = (t, N * (2 * C + 4))
-    t = _time(lambda: tps.lipar_score_motion(x_frames, 4, out=score), flush)
+    t = timer(lambda: tps.lipar_score_motion(x_frames, 4, out=score), flush)
     stages["score_motion_L4"] = (t, N * (2 * C + 4))
     ws = tps.workspace(tps.OP_SELECT, N, 0, dev)
     idx_all = torch.empty(N, dtype=torch.int32, device=dev)
     cnt = torch.empty(1, dtype=torch.int32, device=dev)
     k3 = N // 3
-    t = _time(lambda: tps.lipar_select(score, tps.SELECT_TOPK, k=k3, idx=idx_all, count=cnt, ws=ws), flush)
+    t = timer(lambda: tps.lipar_select(score, tps.SELECT_TOPK, k=k3, idx=idx_all, count=cnt, ws=ws), flush)
     stages["select_topk"] = (t, N * 4 + k3 * 4)
-    t = _time(lambda: tps.lipar_select(score, tps.SELECT_THRESHOLD, tau=1.0, idx=idx_all, count=cnt, ws=ws), flush)
+    t = timer(lambda: tps.lipar_select(score, tps.SELECT_THRESHOLD, tau=1.0, idx=idx_all, count=cnt, ws=ws), flush)
     stages["select_threshold"] = (t, N * 4 + int(cnt.item()) * 4)
     K = cfg.extra["K"]
     wsg = tps.workspace(tps.OP_GROUP, N, K, dev)
     grp = torch.empty(N, dtype=torch.int8, device=dev)
-    t = _time(lambda: tps.lipar_group(score, K, group=grp, ws=wsg), flush)
+    t = timer(lambda: tps.lipar_group(score, K, group=grp, ws=wsg), flush)
     stages["group"] = (t, N * 4 + N)
     wss = tps.workspace(tps.OP_SCHEDULE, N, K, dev)
-    t = _time(lambda: tps.lipar_schedule(grp, K, cfg.extra["budgets"], cfg.extra["T"], 1, 0, idx=idx_all, count=cnt,
+    t = timer(lambda: tps.lipar_schedule(grp, K, cfg.extra["budgets"], cfg.extra["T"], 1, 0, idx=idx_all, count=cnt,
                                          ws=wss), flush)
     A = int(cnt.item())
     stages["schedule"] = (t, N + A * 4)
@@ -448,28 +451,30 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     kc, vc = rnd(N, H, d), rnd(N, H, d)
     kf, vf = rnd(A, H, d), rnd(A, H, d)
     ke, ve = torch.empty_like(kc), torch.empty_like(vc)
-    t = _time(lambda: tps.tps_gather_rows(kf, kc, idx, cnt), flush)
+    t = timer(lambda: tps.tps_gather_rows(kf, kc, idx, cnt), flush)
     stages["gather"] = (t, 2 * R * A)
-    t = _time(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt), flush)
+    t = timer(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt), flush)
     stages["kv_sync"] = (t, 4 * R * A + 4 * A)
-    t = _time(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve), flush)
+    t = timer(lambda: tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve), flush)
     stages["kv_sync_renoise"] = (t, 6 * R * A + 4 * R * (N - A) + 4 * A)
     o_full, o_act = rnd(N, H, d), rnd(A, H, d)
-    t = _time(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
+    t = timer(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
     stages["scatter_out"] = (t, 2 * R * A)
     # attention-recovery merge of two partial results for the A active rows
     lse_a, lse_b, lse_o = (torch.randn(A, H, generator=g, device=dev) for _ in range(3))
     o_b = rnd(A, H, d)
-    t = _time(lambda: tps.attn_lse_merge(o_act, lse_a, o_b, lse_b, cnt, o=o_act, lse=lse_o), flush)
+    t = timer(lambda: tps.attn_lse_merge(o_act, lse_a, o_b, lse_b, cnt, o=o_act, lse=lse_o), flush)
     stages["lse_merge"] = (t, 3 * R * A + 3 * 4 * H * A)
     # cached Euler update (HSA 2.3): fp32 state [N, C], bf16 velocity cache
     xs = torch.randn(N, C, generator=g, device=dev, dtype=torch.float32)
     vcache = rnd(N, C)
     vfresh = rnd(A, C)
-    t = _time(lambda: tps.hsa_euler_update(xs, vcache, vfresh, idx, cnt, -0.025), flush)
+    t = timer(lambda: tps.hsa_euler_update(xs, vcache, vfresh, idx, cnt, -0.025), flush)
     stages["euler_update"] = (t, A * (2 * C + 2 * C + 8 * C) + (N - A) * (2 * C + 8 * C) + 4 * A)
     out["stages_hsa"] = {k: {"ms": round(v[0], 4), "bytes": int(v[1]), "GBps": round(v[1] / v[0] / 1e6, 1),
                              "frac_hbm": round(v[1] / v[0] / 1e6 / hbm_gbs, 3)} for k, v in stages.items()}
+    if stages_once:
+        return out
     # ---- HSA attention per step size --------------------------------------------------
     att = {}
     scale = 1 / math.sqrt(d)
@@ -478,7 +483,7 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
         ii = torch.arange(0, N, N // Aq if Aq < N else 1, device=dev, dtype=torch.int32)[:Aq].contiguous()
         cc = torch.tensor([Aq], dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
-        t = _time(lambda: tps.pruned_attn(q, ke, ve, ii, cc, scale, o_act=o), flush, reps=3, warm=1)
+        t = timer(lambda: tps.pruned_attn(q, ke, ve, ii, cc, scale, o_act=o), flush, reps=3, warm=1)
         alg = 4.0 * d * H * Aq * N
         tiles, ctas = executed_key_tiles(np.arange(Aq), N)
         exe = 4.0 * d * H * 256 * 128 * tiles
@@ -496,7 +501,7 @@ def config_sweep(dev, peak_tflops, hbm_gbs):
     bmd = bm.to(dev)
     q = rnd(kb_, H, d)
     o = torch.empty_like(q)
-    t = _time(lambda: tps.pruned_attn(q, kc, vc, bidx, bcnt, scale, blockmask=bmd, o_act=o), flush, reps=3, warm=1)
+    t = timer(lambda: tps.pruned_attn(q, kc, vc, bidx, bcnt, scale, blockmask=bmd, o_act=o), flush, reps=3, warm=1)
     bidx_h = bidx.cpu().numpy()
     bm_h = bm.numpy()
     alg = 4.0 * d * H * 128 * float(bm_h[bidx_h // 128].sum())
@@ -522,6 +527,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
+    ap.add_argument("--stages-once", action="store_true",
+                    help="run each HSA-size stage kernel once, print its table and exit (for counter captures)")
     a = ap.parse_args()
     if a.warmup < 3:
         a.warmup = 3
@@ -541,6 +548,13 @@ def main():
 
     from token_pruned_sparse_b200 import tps
     tps.lib()
+    if a.stages_once:
+        pk, _ = peaks()
+        res = config_sweep(dev, float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), stages_once=True)
+        torch.cuda.synchronize()
+        tps.tps_check()
+        print(json.dumps(res["stages_hsa"]), flush=True)
+        return 0
     st = MidStep(rank_seed_offset(rank), dev, a.attn)
     flush = L2Flush(dev)
     for _ in range(a.warmup):

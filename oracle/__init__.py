@@ -10,6 +10,9 @@ arithmetic) feed both.
 Parity status per function (see each docstring for the pins):
   lipar_score, select_threshold, select_topk, group_split, schedule_active,
   kv_sync, pruned_attn, scatter_out  -- pinned by tests/test_oracle_pins.py
+  euler_update, lse_merge, lipar_score_motion,
+  timeripple_delta/_reuse/_token_score/_theta -- pinned likewise (hand-worked
+                                         fixtures, closed forms, invariants)
   philox4x32_10 raw stream            -- parity unpinned (no published
                                          known-answer vector available offline);
                                          its normals are pinned statistically.

@@ -23,6 +23,9 @@ Sources (gist.science summaries):
            1, 2, 3", SC'11 -- Philox4x32-10.
   [BM]     Box & Muller, "A Note on the Generation of Random Normal
            Deviates", Ann. Math. Stat. 29 (1958).
+  [TR]     "Timeripple: Accelerating vDiTs by Understanding the Spatio-Temporal
+           Correlations in Latent Space" (Metodologia 2: per-axis similarity
+           checks; Metodologia 3: threshold schedule)
 """
 from __future__ import annotations
 
@@ -36,6 +39,7 @@ __all__ = [
     "schedule_groups", "schedule_active", "compact", "kv_sync", "philox4x32_10",
     "philox_words", "renoise_normals", "pruned_attn", "scatter_out", "gather_rows",
     "attn_flops", "euler_update", "lse_merge", "lipar_score_motion",
+    "timeripple_delta", "timeripple_reuse", "timeripple_token_score", "timeripple_theta",
 ]
 
 
@@ -393,3 +397,71 @@ def gather_rows(src, idx):
     """Rows idx of src (the active tokens handed to the QKV projection,
     [HSA] 2.2 (1))."""
     return src[torch.as_tensor(np.asarray(idx, np.int64))].clone()
+
+
+# ---------------------------------------------------------------------------
+# Timeripple: per-axis similarity check of Q / K tokens
+# ---------------------------------------------------------------------------
+def timeripple_delta(x, F: int, Hs: int, Ws: int, windows) -> np.ndarray:
+    """[TR] Metodologia 2 (similarity checks): for every Q (or K) token three
+    independent checks run along the temporal, x and y axes, each measuring a
+    standard error over a window of the token's channels.
+
+    Readings: x is [N, H, d] with token n = (f * Hs + y) * Ws + x_col. The
+    neighbour along an axis is the previous token on it: t -> n - Hs*Ws (f >= 1),
+    x -> n - 1 (x_col >= 1), y -> n - Ws (y >= 1). windows[a] = (start, length)
+    picks the head-dim channels (start + j) mod d, j < length (a cyclic window,
+    0 <= length <= d). The standard error is the root-mean-square difference
+    over the window,
+        Delta_a(n, h) = sqrt( sum_{c in W_a} (x[n,h,c] - x[nb_a(n),h,c])^2 / length_a ),
+    and +inf when the token has no neighbour on that axis or length_a = 0.
+    Returns float64 [3, N, H] in axis order (t, x, y)."""
+    X = f64(x)
+    N, H, d = X.shape
+    assert N == F * Hs * Ws
+    G = X.reshape(F, Hs, Ws, H, d)
+    out = np.full((3, F, Hs, Ws, H), np.inf)
+    for a, (start, length) in enumerate(windows):
+        if length == 0:
+            continue
+        ch = (int(start) + np.arange(int(length))) % d
+        if a == 0:
+            cur, nb, dst = G[1:], G[:-1], out[0, 1:]
+        elif a == 1:
+            cur, nb, dst = G[:, :, 1:], G[:, :, :-1], out[1, :, :, 1:]
+        else:
+            cur, nb, dst = G[:, 1:], G[:, :-1], out[2, :, 1:]
+        diff = cur[..., ch] - nb[..., ch]
+        dst[...] = np.sqrt((diff * diff).sum(axis=-1) / float(length))
+    return out.reshape(3, N, H)
+
+
+def timeripple_reuse(delta, theta) -> np.ndarray:
+    """[TR] Metodologia 2 (reuse decision): a token is reusable when its
+    Delta is below the threshold on ANY of the three axes (logical OR).
+    Returns uint8 [N, H] with bit a set iff Delta_a < theta_a, so a
+    (token, head) is reusable iff its byte is non-zero."""
+    D = np.asarray(delta, np.float64)
+    bits = np.zeros(D.shape[1:], np.uint8)
+    for a in range(3):
+        bits |= (D[a] < float(theta[a])).astype(np.uint8) << a
+    return bits
+
+
+def timeripple_token_score(reuse) -> np.ndarray:
+    """Reading that joins the per-(token, head) decision to the token-level
+    active set: score[n] = number of heads of token n that are NOT reusable
+    (an integer, float64). Thresholding it at 1 (lipar_select, tau = 1)
+    keeps every token that needs any head recomputed."""
+    return (np.asarray(reuse) == 0).sum(axis=1).astype(np.float64)
+
+
+def timeripple_theta(step: int, theta_lo: float, theta_hi: float, i0: int = 11, i1: int = 21) -> float:
+    """[TR] Metodologia 3: thresholds rise linearly over the critical window of
+    steps i0..i1 (11..21, steps counted as on the page) and stay fixed
+    outside it: theta_lo up to i0, theta_hi from i1 on."""
+    if step <= i0:
+        return float(theta_lo)
+    if step >= i1:
+        return float(theta_hi)
+    return float(theta_lo) + (float(theta_hi) - float(theta_lo)) * (step - i0) / float(i1 - i0)

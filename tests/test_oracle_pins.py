@@ -390,3 +390,82 @@ def test_motion_score_worked_and_reductions():
     x = synth.gaussian_bf16((6, 30, 16), 71)
     np.testing.assert_array_equal(O.lipar_score_motion(x, 1), O.lipar_score(x))   # L = 1: plain score
     assert np.all(O.lipar_score_motion(x, 3) >= O.lipar_score(x))                 # never below short-term
+
+
+# ------------------------------------------------ Timeripple similarity ---
+def _tr_case(g):
+    gr = g["grid"]
+    x = torch.tensor(g["x"], dtype=torch.bfloat16).reshape(-1, gr["H"], gr["d"])
+    return x, gr["F"], gr["Hs"], gr["Ws"]
+
+
+def test_timeripple_worked_example():
+    g = _gold("timeripple_worked.json")
+    x, F, Hs, Ws = _tr_case(g)
+    D = O.timeripple_delta(x, F, Hs, Ws, g["windows"])
+    for a, key in enumerate(("delta_t", "delta_x", "delta_y")):
+        np.testing.assert_allclose(D[a][:, 0], [_num(v) for v in g[key]], rtol=1e-15, atol=0)
+    reuse = O.timeripple_reuse(D, g["theta"])
+    assert reuse[:, 0].tolist() == g["reuse"]
+    assert O.timeripple_token_score(reuse).tolist() == g["token_score"]
+
+
+def test_timeripple_axes_transpose_and_invariants():
+    rng = np.random.default_rng(11)
+    F, Hs, Ws, H, d = 3, 4, 5, 2, 8
+    g = rng.standard_normal((F, Hs, Ws, H, d))
+    x = torch.from_numpy(g.reshape(-1, H, d)).to(torch.bfloat16)
+    wins = [(0, 8), (3, 4), (6, 5)]
+    D = O.timeripple_delta(x, F, Hs, Ws, wins)
+    # transposing the grid swaps the x and y axes (and their windows)
+    xt = x.reshape(F, Hs, Ws, H, d).permute(0, 2, 1, 3, 4).reshape(-1, H, d)
+    Dt = O.timeripple_delta(xt, F, Ws, Hs, [wins[0], wins[2], wins[1]])
+    T = lambda a: a.reshape(F, Hs, Ws, H).transpose(0, 2, 1, 3).reshape(-1, H)
+    assert np.array_equal(Dt[0], T(D[0]))
+    assert np.array_equal(Dt[1], T(D[2])) and np.array_equal(Dt[2], T(D[1]))
+    # a common offset cancels, a common scale multiplies (powers of two: exact in bf16)
+    np.testing.assert_allclose(O.timeripple_delta(x.double() + 4.0, F, Hs, Ws, wins), D, rtol=1e-15)
+    np.testing.assert_allclose(O.timeripple_delta(x * 2, F, Hs, Ws, wins), 2 * D, rtol=1e-15)
+    # no neighbour -> +inf on exactly the first frame / column / row
+    Dg = D.reshape(3, F, Hs, Ws, H)
+    assert np.isinf(Dg[0, 0]).all() and np.isfinite(Dg[0, 1:]).all()
+    assert np.isinf(Dg[1, :, :, 0]).all() and np.isfinite(Dg[1, :, :, 1:]).all()
+    assert np.isinf(Dg[2, :, 0]).all() and np.isfinite(Dg[2, :, 1:]).all()
+    # a window of the full head equals the RMS computed by torch over whole rows
+    full = O.timeripple_delta(x, F, Hs, Ws, [(5, d)] * 3)
+    xx = x.double().reshape(F, Hs, Ws, H, d)
+    rms = torch.sqrt(torch.mean((xx[1:] - xx[:-1]) ** 2, dim=-1)).numpy().reshape(-1, H)
+    np.testing.assert_allclose(full[0][Hs * Ws:], rms, rtol=1e-14)
+    # a zero-length window disables its axis
+    assert np.isinf(O.timeripple_delta(x, F, Hs, Ws, [(0, 0), (0, 0), (0, 0)])).all()
+
+
+def test_timeripple_static_video_and_theta_ramp():
+    F, Hs, Ws, H, d = 4, 3, 3, 2, 8
+    one = synth.gaussian_bf16((1, Hs * Ws, H, d), 5)
+    x = one.expand(F, -1, -1, -1).reshape(-1, H, d).contiguous()
+    D = O.timeripple_delta(x, F, Hs, Ws, [(0, 8), (0, 8), (0, 8)])
+    r = O.timeripple_reuse(D, (1e-3, 0.0, 0.0)).reshape(F, Hs * Ws, H)
+    assert (r[0] == 0).all() and (r[1:] == 1).all()          # t-bit on every frame after the first
+    assert O.timeripple_token_score(r.reshape(-1, H)).tolist() == [H] * (Hs * Ws) + [0] * ((F - 1) * Hs * Ws)
+    # theta <= 0 never passes (Delta >= 0 and the test is strict)
+    assert not O.timeripple_reuse(D, (0.0, 0.0, 0.0)).any()
+    th = [O.timeripple_theta(i, 0.0, 0.05) for i in range(1, 41)]
+    assert th[:11] == [0.0] * 11 and th[20:] == [0.05] * 20
+    assert th[15] == pytest.approx(0.025, abs=1e-18)              # step 16, halfway
+    assert all(b >= a for a, b in zip(th, th[1:]))
+    assert O.timeripple_theta(12, 1.0, 3.0) == pytest.approx(1.2, abs=1e-15)
+
+
+def test_timeripple_pins_catch_planted_mistakes():
+    g = _gold("timeripple_worked.json")
+    x, F, Hs, Ws = _tr_case(g)
+    X = x.double().reshape(F, Hs, Ws, 4)
+    # a sum instead of a mean over the window, or the NEXT token as neighbour
+    assert math.sqrt(float(((X[1, 1, 1] - X[0, 1, 1]) ** 2).sum())) != _num(g["delta_t"][7])
+    assert float(torch.sqrt(((X[0, 0, 1, 2:] - X[0, 1, 1, 2:]) ** 2).mean())) != _num(g["delta_x"][1])
+    # a window that does not wrap (channels 3 only, or 3 and 4 clipped) changes Delta_y of token 3
+    assert float(torch.sqrt(((X[0, 1, 1, 3:] - X[0, 0, 1, 3:]) ** 2).mean())) != _num(g["delta_y"][3])
+    # '<=' instead of '<' would mark token 1 reusable on x (Delta_x = theta_x = 1)
+    D = O.timeripple_delta(x, F, Hs, Ws, g["windows"])
+    assert (D[1][1, 0] <= g["theta"][1]) and O.timeripple_reuse(D, g["theta"])[1, 0] == 0

@@ -37,6 +37,7 @@ import torch
 __all__ = [
     "VideoSpec", "CONFIGS", "latent_video", "velocity_pair", "projection_weights",
     "project", "to_bf16", "random_scores", "block_mask_band_random", "gaussian_bf16",
+    "timeripple_windows", "TR_THETA",
 ]
 
 
@@ -90,6 +91,27 @@ CONFIGS = {
     "block": Config("block", VideoSpec(33, 45, 80, 128, 6, 8, True, 5), 24, 128, "block", "frame",
                     keep=(0.4,), extra={"block": 128, "kept_per_row": 139}),
 }
+
+
+def timeripple_windows(d: int):
+    """Channel windows (start, length) of the t, x and y similarity checks for a
+    head of d channels, as cyclic ranges over the head dimension.
+
+    Configuration, not arithmetic: the head's rotary channels are taken as three
+    contiguous groups [t | x | y] of sizes (d - 4*(d//6), 2*(d//6), 2*(d//6)),
+    each even so rotary pairs stay whole. A check along an axis uses the channels
+    that axis does NOT rotate (they stay similar between neighbours on it): t ->
+    the x and y groups; x -> the y and t groups (the window wraps); y -> the t
+    and x groups."""
+    g = 2 * (d // 6)
+    dt = d - 2 * g
+    return ((dt, 2 * g), (dt + g, dt + g), (0, dt + g))
+
+
+# Threshold schedule of the per-axis checks (t, x, y): theta rises from 0 at
+# step 11 to these values at step 21. Background tokens of the synthetic video
+# move by jitter only (RMS about 0.01 after projection), moving tokens by ~1.4.
+TR_THETA = (0.05, 0.05, 0.05)
 
 
 def keep_count(N: int, ratio: float) -> int:
