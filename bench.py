@@ -471,6 +471,13 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     vfresh = rnd(A, C)
     t = timer(lambda: tps.hsa_euler_update(xs, vcache, vfresh, idx, cnt, -0.025), flush)
     stages["euler_update"] = (t, A * (2 * C + 2 * C + 8 * C) + (N - A) * (2 * C + 8 * C) + 4 * A)
+    # Timeripple per-axis check of all N query rows: reuse byte per (token, head) + token score
+    tr_reuse = torch.empty((N, H), dtype=torch.uint8, device=dev)
+    tr_score = torch.empty(N, dtype=torch.float32, device=dev)
+    wins = synth.timeripple_windows(d)
+    t = timer(lambda: tps.timeripple_score(kc, cfg.video.F, cfg.video.Hs, cfg.video.Ws, wins, synth.TR_THETA,
+                                           reuse=tr_reuse, score=tr_score), flush)
+    stages["timeripple_score"] = (t, N * R + 2 * N * H + 4 * N)
     out["stages_hsa"] = {k: {"ms": round(v[0], 4), "bytes": int(v[1]), "GBps": round(v[1] / v[0] / 1e6, 1),
                              "frac_hbm": round(v[1] / v[0] / 1e6 / hbm_gbs, 3)} for k, v in stages.items()}
     if stages_once:
@@ -515,6 +522,29 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     return out
 
 
+def kernel_case(name, dev):
+    """One small, self-contained launch sequence of a single kernel for a
+    detailed counter capture (a few hundred MB on the device, inputs larger than
+    L2): a warm-up launch, then the launch to capture."""
+    from token_pruned_sparse_b200 import tps
+    g = torch.Generator(device=dev)
+    g.manual_seed(4)
+    if name == "timeripple":
+        cfg = synth.CONFIGS["hsa"]
+        v = cfg.video
+        x = torch.randn((v.N, cfg.H, cfg.d), generator=g, device=dev).to(torch.bfloat16)   # 730 MB
+        reuse = torch.empty((v.N, cfg.H), dtype=torch.uint8, device=dev)
+        score = torch.empty(v.N, dtype=torch.float32, device=dev)
+        for _ in range(2):
+            tps.timeripple_score(x, v.F, v.Hs, v.Ws, synth.timeripple_windows(cfg.d), synth.TR_THETA,
+                                 reuse=reuse, score=score)
+    else:
+        raise SystemExit(f"unknown kernel case {name}")
+    torch.cuda.synchronize()
+    tps.tps_check()
+    return {"kernel_case": name, "ok": True}
+
+
 # ------------------------------------------------------------------ main ------
 def main():
     ap = argparse.ArgumentParser()
@@ -527,6 +557,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
+    ap.add_argument("--kernel-case", choices=["timeripple"], default=None,
+                    help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
                     help="run each HSA-size stage kernel once, print its table and exit (for counter captures)")
     a = ap.parse_args()
@@ -548,6 +580,9 @@ def main():
 
     from token_pruned_sparse_b200 import tps
     tps.lib()
+    if a.kernel_case:
+        print(json.dumps(kernel_case(a.kernel_case, dev)), flush=True)
+        return 0
     if a.stages_once:
         pk, _ = peaks()
         res = config_sweep(dev, float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), stages_once=True)

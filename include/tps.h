@@ -91,6 +91,42 @@ TPS_API int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16
 TPS_API int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int64_t C, int L, float* score,
                                tps_stream stream);
 
+/* ---- per-axis similarity check of Q or K tokens ([TR] Metodologia 2) ---------
+ * Three independent checks per (token, head), along t, x and y. The neighbour on
+ * an axis is the previous token on it: t -> (f-1, y, x), x -> (f, y, x-1),
+ * y -> (f, y-1, x). Each check measures the root-mean-square difference over
+ * a cyclic window of head channels,
+ *   Delta_a = sqrt( sum_{c in W_a} (x[n,h,c] - x[nb_a(n),h,c])^2 / len_a ),
+ *   W_a = { (start_a + j) mod d : 0 <= j < len_a },
+ * and Delta_a = +inf when the token has no neighbour on the axis or len_a = 0.
+ * fp32 arithmetic on bf16 inputs. A (token, head) is reusable iff Delta_a <
+ * theta_a on ANY axis (logical OR).
+ *   x        [F, Hs, Ws, H, d] bf16 (token-major [N, H, d], N = F*Hs*Ws,
+ *            n = (f*Hs + y)*Ws + x), 16-byte aligned; d in {64, 128}.
+ *   windows  HOST int32[6] = {start_t, len_t, start_x, len_x, start_y, len_y},
+ *            0 <= start < d, 0 <= len <= d.
+ *   theta    HOST float[3] = {theta_t, theta_x, theta_y}; not NaN. The check
+ *            is strict, so theta <= 0 never passes.
+ *   reuse    [N, H] uint8 output: bit a (0 = t, 1 = x, 2 = y) set iff
+ *            Delta_a < theta_a.
+ *   delta    [3, N, H] float32 output (Delta_t, Delta_x, Delta_y), or NULL.
+ *   score    [N] float32 output, or NULL: the number of heads of token n
+ *            whose reuse byte is 0 (an integer). lipar_select with threshold
+ *            tau = 1 then keeps every token that needs any head recomputed.
+ * The reading of the standard error as an RMS difference, the choice of
+ * neighbours and the token score are stated readings: the summary leaves them
+ * open. */
+TPS_API int timeripple_score(const tps_bf16* x, int64_t F, int64_t Hs, int64_t Ws, int H, int d,
+                             const int32_t* windows, const float* theta, uint8_t* reuse, float* delta,
+                             float* score, tps_stream stream);
+
+/* Threshold schedule ([TR] Metodologia 3): the thresholds rise linearly over a
+ * window of steps and stay fixed outside it. Returns theta_lo for step <= i0,
+ * theta_hi for step >= i1, and the linear interpolation in between (steps
+ * counted from 1; the summary's window is i0 = 11, i1 = 21). Host-only, pure;
+ * i1 <= i0 makes it a step at i0. */
+TPS_API float timeripple_theta(int step, float theta_lo, float theta_hi, int i0, int i1);
+
 /* ---- steps 2-3: active set and compaction ([LIPAR] 2.B; [HSA] 2.1) ---------
  * mode TPS_SELECT_THRESHOLD: active iff score >= tau (a token below tau is
  *   redundant and pruned). NaN is never active.

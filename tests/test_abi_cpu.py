@@ -97,3 +97,33 @@ def test_binding_raises_with_message():
     with pytest.raises(tps.TPSError) as e:
         tps._chk(tps.lib().lipar_score(NULL, NULL, NULL, 2, 4, 64, F, NULL))
     assert e.value.code == tps.INVALID_ARG and "non-null" in str(e.value)
+
+
+def test_timeripple_validation_and_theta_ramp():
+    import oracle as O
+    l = tps.lib()
+    win = (C.c_int32 * 6)(44, 84, 86, 86, 0, 86)
+    th = (C.c_float * 3)(0.05, 0.05, 0.05)
+    W, T = C.cast(win, C.c_void_p), C.cast(th, C.c_void_p)
+    assert l.timeripple_score(NULL, 2, 4, 4, 2, 128, W, T, F, NULL, NULL, NULL) == tps.INVALID_ARG
+    assert l.timeripple_score(F, 2, 4, 4, 2, 128, W, T, NULL, NULL, NULL, NULL) == tps.INVALID_ARG
+    code, msg = _err(l.timeripple_score(F, 2, 4, 4, 2, 96, W, T, F, NULL, NULL, NULL))
+    assert code == tps.INVALID_ARG and "d=96" in msg
+    assert l.timeripple_score(F, 0, 4, 4, 2, 128, W, T, F, NULL, NULL, NULL) == tps.SHAPE
+    assert l.timeripple_score(F, 2, 4, 4, 0, 128, W, T, F, NULL, NULL, NULL) == tps.SHAPE
+    bad = (C.c_int32 * 6)(44, 84, 128, 1, 0, 86)           # start = d
+    code, msg = _err(l.timeripple_score(F, 2, 4, 4, 2, 128, C.cast(bad, C.c_void_p), T, F, NULL, NULL, NULL))
+    assert code == tps.INVALID_ARG and "window 1" in msg
+    longw = (C.c_int32 * 6)(0, 65, 0, 64, 0, 64)           # longer than d = 64
+    assert l.timeripple_score(F, 2, 4, 4, 2, 64, C.cast(longw, C.c_void_p), T, F, NULL, NULL, NULL) == \
+        tps.INVALID_ARG
+    nan = (C.c_float * 3)(0.05, float("nan"), 0.05)
+    assert l.timeripple_score(F, 2, 4, 4, 2, 128, W, C.cast(nan, C.c_void_p), F, NULL, NULL, NULL) == \
+        tps.INVALID_ARG
+    assert l.timeripple_score(MIS, 2, 4, 4, 2, 128, W, T, F, NULL, NULL, NULL) == tps.ALIGN
+    # the host-only threshold ramp against the oracle's (fp32 vs fp64)
+    for lo, hi in ((0.0, 0.05), (0.2, 0.1), (1.0, 3.0)):
+        for step in range(0, 45):
+            assert tps.timeripple_theta(step, lo, hi) == pytest.approx(O.timeripple_theta(step, lo, hi),
+                                                                       rel=1e-6, abs=1e-8)
+    assert tps.timeripple_theta(5, 1.0, 2.0, 7, 7) == 1.0 and tps.timeripple_theta(8, 1.0, 2.0, 7, 7) == 2.0

@@ -42,6 +42,8 @@ SIGNATURES = {
     "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
     "lipar_score_motion": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _P]),
     "attn_lse_merge": (_INT, [_P, _P, _P, _P, _P, _I64, _INT, _INT, _P, _P, _P]),
+    "timeripple_score": (_INT, [_P, _I64, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _P]),
+    "timeripple_theta": (C.c_float, [_INT, C.c_float, C.c_float, _INT, _INT]),
     "tps_workspace_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_last_error": (C.c_char_p, []),
     "tps_check": (_INT, [_P]),
@@ -263,6 +265,30 @@ def attn_lse_merge(o1, lse1, o2, lse2, count, o=None, lse=None, cap=None, stream
     _chk(lib().attn_lse_merge(_ptr(o1), _ptr(lse1), _ptr(o2), _ptr(lse2), _ptr(count), cap, H, d, _ptr(o),
                               _ptr(lse), _stream(stream)))
     return o
+
+
+def timeripple_score(x, F, Hs, Ws, windows, theta, reuse=None, delta=False, score=False, stream=None):
+    """x [F*Hs*Ws, H, d] bf16. windows: ((start, len),) * 3 for t, x, y; theta:
+    3 floats. Returns (reuse uint8 [N, H], delta float32 [3, N, H] or None,
+    score float32 [N] or None); pass tensors as delta/score to reuse buffers."""
+    N, H, d = x.shape
+    if reuse is None:
+        reuse = torch.empty((N, H), dtype=torch.uint8, device=x.device)
+    if delta is True:
+        delta = torch.empty((3, N, H), dtype=torch.float32, device=x.device)
+    if score is True:
+        score = torch.empty(N, dtype=torch.float32, device=x.device)
+    delta = delta if isinstance(delta, torch.Tensor) else None
+    score = score if isinstance(score, torch.Tensor) else None
+    win = (C.c_int32 * 6)(*[int(v) for w in windows for v in w])
+    th = (C.c_float * 3)(*[float(v) for v in theta])
+    _chk(lib().timeripple_score(_ptr(x), F, Hs, Ws, H, d, C.cast(win, _P), C.cast(th, _P), _ptr(reuse),
+                                _ptr(delta), _ptr(score), _stream(stream)))
+    return reuse, delta, score
+
+
+def timeripple_theta(step, theta_lo, theta_hi, i0=11, i1=21) -> float:
+    return float(lib().timeripple_theta(int(step), float(theta_lo), float(theta_hi), int(i0), int(i1)))
 
 
 def tps_check(stream=None):
