@@ -305,6 +305,14 @@ TPS_API int tps_check(tps_stream stream);
 TPS_API int tps_philox_fill(uint32_t* out, uint64_t q0, int64_t nq, uint64_t seed, uint32_t step,
                     uint32_t tensor, tps_stream stream);
 
+/* Self-test of the failure-detection path (no counterpart on the pages). One
+ * CTA waits on a shared-memory barrier that nothing ever completes, through the
+ * same bounded wait every library kernel uses, but with a limit of
+ * limit_cycles SM clock cycles (clamped to [1000, 2e9]). The wait gives up,
+ * the CTA records TPS_ERR_TIMEOUT in the status word and exits normally, so the
+ * context stays usable; tps_check() then returns TPS_ERR_TIMEOUT once. */
+TPS_API int tps_wait_probe(int64_t limit_cycles, tps_stream stream);
+
 /* Library version string. */
 TPS_API const char* tps_version(void);
 

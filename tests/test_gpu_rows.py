@@ -146,3 +146,21 @@ def test_euler_update_flags_bad_index():
     with pytest.raises(tps.TPSError) as e:
         tps.tps_check()
     assert e.value.code == tps.BOUNDS
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """The failure-detection path without a fault: a barrier nothing completes,
+    waited on with a ~1 ms limit, must end in TPS_ERR_TIMEOUT from tps_check,
+    once, and leave the context usable."""
+    tps.tps_check()
+    tps.tps_wait_probe(2_000_000)
+    with pytest.raises(tps.TPSError) as e:
+        tps.tps_check()
+    assert e.value.code == tps.TIMEOUT
+    tps.tps_check()                                                         # cleared
+    full = synth.gaussian_bf16((64, 2, 64), 3).to(DEV)
+    act = synth.gaussian_bf16((4, 2, 64), 4).to(DEV)
+    di, dc = _dev_idx(np.array([1, 7, 30, 63], np.int32))
+    tps.scatter_out(full, act, di, dc, cap=4)
+    tps.tps_check()
+    assert torch.equal(full.cpu()[[1, 7, 30, 63]], act.cpu())

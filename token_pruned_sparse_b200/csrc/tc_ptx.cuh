@@ -44,20 +44,25 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 
 // Waits for the phase with the given parity to complete. Gives up -- setting
 // the CTA's abort flag and the device status word -- when another role has
-// aborted or the wait exceeds kWaitLimitCycles. Returns false on give-up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* status) {
+// aborted or the wait exceeds `limit` cycles. Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* status, long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       raise_status(status, STATUS_TIMEOUT);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* status) {
+  return mbar_wait_for(bar, parity, abort_flag, status, kWaitLimitCycles);
 }
 
 // Teardown wait: bounded, ignores the abort flag (used to drain work this

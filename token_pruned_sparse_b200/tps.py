@@ -48,6 +48,7 @@ SIGNATURES = {
     "tps_last_error": (C.c_char_p, []),
     "tps_check": (_INT, [_P]),
     "tps_philox_fill": (_INT, [_P, C.c_uint64, _I64, C.c_uint64, C.c_uint32, C.c_uint32, _P]),
+    "tps_wait_probe": (_INT, [_I64, _P]),
     "tps_version": (C.c_char_p, []),
 }
 
@@ -300,6 +301,10 @@ def tps_philox_fill(q0, nq, seed, step, tensor, out=None, stream=None):
         out = torch.empty(nq * 4, dtype=torch.int32, device="cuda")
     _chk(lib().tps_philox_fill(_ptr(out), q0, nq, seed, step, tensor, _stream(stream)))
     return out
+
+
+def tps_wait_probe(limit_cycles, stream=None):
+    _chk(lib().tps_wait_probe(int(limit_cycles), _stream(stream)))
 
 
 def version() -> str:
