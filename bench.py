@@ -478,6 +478,15 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     t = timer(lambda: tps.timeripple_score(kc, cfg.video.F, cfg.video.Hs, cfg.video.Ws, wins, synth.TR_THETA,
                                            reuse=tr_reuse, score=tr_score), flush)
     stages["timeripple_score"] = (t, N * R + 2 * N * H + 4 * N)
+    # size ceiling: a plain device copy moving the score kernels' byte counts (read + write), same
+    # flush and timing; at tens of MB launch, ramp-up and tail cap any kernel well below the peak
+    for mb in (31, 61):
+        n = mb * 1000000 // 4                         # bf16 elements per direction
+        src = torch.empty(n, dtype=torch.bfloat16, device=dev).normal_()
+        dst = torch.empty_like(src)
+        t = timer(lambda: dst.copy_(src), flush)
+        stages[f"copy_ceiling_{mb}MB"] = (t, 4 * n)
+        del src, dst
     out["stages_hsa"] = {k: {"ms": round(v[0], 4), "bytes": int(v[1]), "GBps": round(v[1] / v[0] / 1e6, 1),
                              "frac_hbm": round(v[1] / v[0] / 1e6 / hbm_gbs, 3)} for k, v in stages.items()}
     if stages_once:
