@@ -8,11 +8,12 @@
 //
 // Fused, HBM-bound single pass: the velocity cache is refreshed for the active
 // rows and every row of the fp32 state advances, v read once per token. A warp
-// owns a run of 8 consecutive tokens: one binary search in the ascending index
+// owns a run of 8 consecutive tokens: one warp-cooperative search in the ascending index
 // list finds the run's active entries, a warp-wide OR builds the run's active
 // mask, and the warp then sweeps the run's (token, 16-byte vector) items with
 // several loads in flight per lane.
 #include "tps_internal.cuh"
+#include "warp_search.cuh"
 
 namespace tps {
 namespace {
@@ -38,12 +39,7 @@ __global__ void __launch_bounds__(kThreads) euler_kernel(float* __restrict__ x, 
   const int items = kRun * vpr;                 // (token, vector) pairs of one run
   for (int64_t run = warp; run < nruns; run += nwarps) {
     const int64_t r0 = run * kRun;
-    int64_t lo = 0, hi = cnt;                   // lower_bound(idx, r0), every lane
-    while (lo < hi) {
-      const int64_t mid = (lo + hi) >> 1;
-      if (idx[mid] < r0) lo = mid + 1;
-      else hi = mid;
-    }
+    const int64_t lo = warp_lower_bound(idx, cnt, r0, lane);   // first list entry >= r0
     // lanes 0..7 look at the next 8 list entries; those below r0 + 8 are active rows of this run
     const int64_t mine = (lane < kRun && lo + lane < cnt) ? idx[lo + lane] : INT64_MAX;
     const bool in_run = mine >= r0 && mine < r0 + kRun;

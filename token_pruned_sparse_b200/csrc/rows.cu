@@ -18,6 +18,7 @@
 // (Box & Muller, Ann. Math. Stat. 1958), generated where the row is written so
 // the normals never touch memory.
 #include "tps_internal.cuh"
+#include "warp_search.cuh"
 
 namespace tps {
 namespace {
@@ -136,7 +137,7 @@ __device__ __forceinline__ uint4 renoise_vec(uint4 c, float a, float b, const fl
 }
 
 // ---- kv_sync with re-noise: one pass over all N rows --------------------------------
-// A warp owns a run of kRun consecutive rows; one binary search finds the first
+// A warp owns a run of kRun consecutive rows; one warp-cooperative search finds the first
 // active index >= the run start, then the (ascending) list is walked in step.
 constexpr int kRun = 8;
 
@@ -153,14 +154,7 @@ __global__ void __launch_bounds__(kThreads) kv_sync_renoise(
   const uint64_t epr = static_cast<uint64_t>(vpr) * 8;  // elements per row
   for (int64_t run = warp; run < nruns; run += nwarps) {
     const int64_t r0 = run * kRun;
-    // lower_bound(idx[0..cnt), r0), computed redundantly by every lane
-    int64_t lo = 0, hi = cnt;
-    while (lo < hi) {
-      const int64_t mid = (lo + hi) >> 1;
-      if (idx[mid] < r0) lo = mid + 1;
-      else hi = mid;
-    }
-    int64_t p = lo;
+    int64_t p = warp_lower_bound(idx, cnt, r0, lane);   // first list entry >= r0
     for (int64_t n = r0; n < r0 + kRun && n < N; ++n) {
       const bool active = p < cnt && idx[p] == n;
       const int64_t row = n * vpr;

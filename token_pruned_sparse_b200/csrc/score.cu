@@ -20,8 +20,11 @@ namespace tps {
 namespace {
 
 // kV > 0: vectors per row known at compile time (all loads of an iteration are
-// issued before any is used); kV == 0: runtime C.
-template <int L, int kV>
+// issued before any is used); kV == 0: runtime C. kG token groups per lane and
+// iteration, spaced a grid stride apart, so more 16-byte loads are in flight per
+// lane; the grid is one resident wave. (kG = 4 measured slower than 2 at the
+// HSA size: fewer, longer-running warps.)
+template <int L, int kV, int kG>
 __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__ x,
                                                     const uint16_t* __restrict__ xref,
                                                     const uint16_t* __restrict__ xprev,
@@ -34,16 +37,14 @@ __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__
   const int C = kV > 0 ? kV * 8 : Crt;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  // two token groups per iteration (w0 and w0 + half the grid stride) so more
-  // 16-byte loads are in flight per lane; the grid is one resident wave
   const int64_t stride = nwarps * kTokPerWarp;
-  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += 2 * stride) {
-    const uint16_t* cur[2];
-    const uint16_t* ref[2];
-    int64_t tt[2];
-    bool valid[2];
+  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += kG * stride) {
+    const uint16_t* cur[kG];
+    const uint16_t* ref[kG];
+    int64_t tt[kG];
+    bool valid[kG];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kG; ++k) {
       const int64_t t = w0 + k * stride + lane / L;
       tt[k] = t;
       valid[k] = t < N;
@@ -55,18 +56,20 @@ __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__
         else if (xprev) ref[k] = xprev + t * C;
       }
     }
-    float num[2] = {0.f, 0.f}, den[2] = {0.f, 0.f};
+    float num[kG], den[kG];
+#pragma unroll
+    for (int k = 0; k < kG; ++k) num[k] = 0.f, den[k] = 0.f;
 #pragma unroll
     for (int v = sub; v < (kV > 0 ? kV : V); v += L) {
-      uint4 a[2], b[2];
+      uint4 a[kG], b[kG];
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
+      for (int k = 0; k < kG; ++k)
         if (ref[k]) {
           a[k] = ld16(cur[k] + v * 8);
           b[k] = ld16(ref[k] + v * 8);
         }
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
+      for (int k = 0; k < kG; ++k)
         if (ref[k]) {
           const uint32_t aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
           const uint32_t bw[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
@@ -80,7 +83,7 @@ __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__
         }
     }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < kG; ++k) {
 #pragma unroll
       for (int o = L / 2; o > 0; o >>= 1) {
         num[k] += __shfl_xor_sync(0xffffffffu, num[k], o);
@@ -97,23 +100,24 @@ __global__ void __launch_bounds__(256) score_kernel(const uint16_t* __restrict__
   }
 }
 
-template <int L, int kV>
+template <int L, int kV, int kG>
 void launch_score(const uint16_t* x, const uint16_t* xr, const uint16_t* xp, int64_t HW, int C,
                   int64_t N, float* score, cudaStream_t st) {
   constexpr int kThreads = 256;
   const int64_t tok_per_block = (kThreads / 32) * (32 / L);
-  int64_t blocks = (N + 2 * tok_per_block - 1) / (2 * tok_per_block);
+  int64_t blocks = (N + kG * tok_per_block - 1) / (kG * tok_per_block);
   static int per_sm[64] = {0};                  // resident blocks per SM (one wave)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !per_sm[dev]) {
     int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, score_kernel<L, kV>, kThreads, 0) != cudaSuccess || b < 1) b = 4;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, score_kernel<L, kV, kG>, kThreads, 0) != cudaSuccess || b < 1)
+      b = 4;
     per_sm[dev] = b;
   }
   const int64_t cap = static_cast<int64_t>(sm_count()) * (dev >= 0 && dev < 64 ? per_sm[dev] : 4);
   if (blocks > cap) blocks = cap;
-  score_kernel<L, kV><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
+  score_kernel<L, kV, kG><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
 }
 
 // Motion-robust inter-frame score ([LIPAR] 2.B, short- and long-term
@@ -212,13 +216,13 @@ extern "C" int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_b
   const uint16_t* p = x_prev_frame;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int c = static_cast<int>(C);
-  if (c == 128) launch_score<8, 16>(a, r, p, HW, c, N, score, st);
-  else if (c == 64) launch_score<8, 8>(a, r, p, HW, c, N, score, st);
-  else if (c == 256) launch_score<8, 32>(a, r, p, HW, c, N, score, st);
-  else if (V >= 8) launch_score<8, 0>(a, r, p, HW, c, N, score, st);
-  else if (V >= 4) launch_score<4, 0>(a, r, p, HW, c, N, score, st);
-  else if (V >= 2) launch_score<2, 0>(a, r, p, HW, c, N, score, st);
-  else launch_score<1, 0>(a, r, p, HW, c, N, score, st);
+  if (c == 128) launch_score<8, 16, 2>(a, r, p, HW, c, N, score, st);
+  else if (c == 64) launch_score<8, 8, 2>(a, r, p, HW, c, N, score, st);
+  else if (c == 256) launch_score<8, 32, 2>(a, r, p, HW, c, N, score, st);
+  else if (V >= 8) launch_score<8, 0, 2>(a, r, p, HW, c, N, score, st);
+  else if (V >= 4) launch_score<4, 0, 2>(a, r, p, HW, c, N, score, st);
+  else if (V >= 2) launch_score<2, 0, 2>(a, r, p, HW, c, N, score, st);
+  else launch_score<1, 0, 2>(a, r, p, HW, c, N, score, st);
   if (int e = launch_status("lipar_score")) return e;
   return ok();
 }
