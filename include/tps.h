@@ -292,6 +292,10 @@ TPS_API int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_fres
 /* Workspace bytes for lipar_select / lipar_group / lipar_schedule (0 on bad op). */
 TPS_API size_t tps_workspace_size(int op, int64_t N, int K);
 
+/* The smallest workspace those calls accept (0 on bad op): enough for the
+ * multi-launch path only. Results are identical with either size. */
+TPS_API size_t tps_workspace_min_size(int op, int64_t N, int K);
+
 /* Message of the last failing call on this host thread ("" if none). */
 TPS_API const char* tps_last_error(void);
 

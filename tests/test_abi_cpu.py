@@ -127,3 +127,14 @@ def test_timeripple_validation_and_theta_ramp():
             assert tps.timeripple_theta(step, lo, hi) == pytest.approx(O.timeripple_theta(step, lo, hi),
                                                                        rel=1e-6, abs=1e-8)
     assert tps.timeripple_theta(5, 1.0, 2.0, 7, 7) == 1.0 and tps.timeripple_theta(8, 1.0, 2.0, 7, 7) == 2.0
+
+
+def test_workspace_min_size_is_a_lower_bound():
+    for op, K in ((tps.OP_SELECT, 0), (tps.OP_GROUP, 3), (tps.OP_SCHEDULE, 3)):
+        for N in (1, 1000, 118800, 600000, 1 << 22):
+            lo, rec = tps.workspace_min_size(op, N, K), tps.workspace_size(op, N, K)
+            assert 0 < lo <= rec
+    assert tps.workspace_min_size(9, 10, 0) == 0
+    F = C.c_void_p(0x1000)
+    need = tps.workspace_min_size(tps.OP_SELECT, 100000)
+    assert tps.lib().lipar_select(F, 100000, tps.SELECT_TOPK, 0.0, 5, F, F, F, need - 1, NULL) == tps.WORKSPACE

@@ -61,6 +61,33 @@ def test_attn_random_dense(impl, N, A, H, d, sharp):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("growth", ["rising", "falling", "spike"])
+def test_attn_running_max_moves(impl, growth):
+    """Score scales that change along the keys: rising makes later key tiles
+    dominate (tile sums far above 2^40 against the first tile's maximum, so the
+    kernel must take the slow path, find the new maximum and rescale O);
+    falling keeps the first tile's maximum; spike puts one huge tile mid-way."""
+    N, A, H, d = 1500, 200, 2, 128
+    q = synth.gaussian_bf16((A, H, d), 11)
+    k = synth.gaussian_bf16((N, H, d), 12).double()
+    pos = torch.arange(N, dtype=torch.float64)[:, None, None] / N
+    if growth == "rising":
+        g = 1.0 + 24.0 * pos
+    elif growth == "falling":
+        g = 25.0 - 24.0 * pos
+    else:
+        g = torch.ones_like(pos)
+        g[640:768] = 30.0
+    k = (k * g).to(torch.bfloat16)
+    v = synth.gaussian_bf16((N, H, d), 13)
+    idx = np.sort(np.random.default_rng(5).choice(N, A, replace=False))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _run(impl, q, k, v, idx, scale)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
+    _check(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
 def test_attn_constant_keys_mean_of_v(impl):
     N, H, d = 1500, 2, 128
     k = synth.gaussian_bf16((1, H, d), 1).expand(N, H, d).contiguous()

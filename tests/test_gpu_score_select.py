@@ -160,3 +160,20 @@ def test_score_motion(name, L):
     assert np.array_equal(np.isinf(s), np.isinf(ref))
     fin = np.isfinite(ref)
     np.testing.assert_allclose(s[fin], ref[fin], rtol=_rtol(cfg.video.C), atol=0)
+
+
+@pytest.mark.parametrize("N", [1000, 118800, 600000])
+def test_select_multi_launch_path_matches_oracle(N):
+    """The multi-launch path (taken with the minimum workspace, and for N beyond
+    one cooperative launch) gives the oracle's lists too."""
+    s = synth.random_scores(N, 77 + N, ties=True, specials=True)
+    sd = s.to(DEV)
+    sn = s.numpy()
+    for ws in (tps.workspace(tps.OP_SELECT, N, 0, DEV, minimal=True), tps.workspace(tps.OP_SELECT, N, 0, DEV)):
+        for k in (0, 1, N // 7, N // 2, N):
+            idx, cnt = tps.lipar_select(sd, tps.SELECT_TOPK, k=k, ws=ws)
+            assert np.array_equal(_idx(idx, cnt), O.select_topk(sn, k)), (N, k, ws.numel())
+        for tau in (0.25, 1.0):
+            idx, cnt = tps.lipar_select(sd, tps.SELECT_THRESHOLD, tau=tau, ws=ws)
+            assert np.array_equal(_idx(idx, cnt), O.select_threshold(sn, tau)), (N, tau, ws.numel())
+    tps.tps_check()

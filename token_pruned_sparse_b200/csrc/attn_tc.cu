@@ -14,11 +14,16 @@
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r of
 //              its tile (= TMEM lane r). Loads S from TMEM, online softmax in
 //              the log2 domain, writes P (bf16) back over the first half of
-//              its S columns, and rescales O in TMEM only when the running
-//              maximum grew by more than 2^8 (exact: the final normalisation
-//              uses the same reference maximum as every P).
+//              its S columns. After the first tile it skips the row maximum:
+//              P is formed against the running reference maximum, which is
+//              exact for any reference (the final normalisation uses the same
+//              one), and only when a tile's row sum exceeds 2^40 does the warp
+//              reload S, take the maximum and rescale O in TMEM.
 //   warp 8     TMA producer: Q (both tiles) once, then K and V tiles of 128
-//              keys into a two-stage ring, 128-byte swizzled.
+//              keys into two-stage rings, 128-byte swizzled. A K stage is
+//              freed when the last S MMA reading it completes and a V stage
+//              when the last P V MMA does, so the next K tile streams in about
+//              one tile period earlier than a shared K/V stage would allow.
 //   warp 9     MMA issuer and TMEM owner. Per key tile j and tile t:
 //              O_t += P_t(j) V_j (A operand read from TMEM), then
 //              S_t(j+1) = Q_t K_{j+1}^T; completion via tcgen05.commit.
@@ -49,7 +54,7 @@ constexpr int kTmaWarp = kSoftmaxThreads / 32;
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kTmemCols = 512;
 constexpr int kSubBytes = 128 * 128;   // one [128 rows x 64 bf16] swizzled sub-tile
-constexpr float kRescaleLog2 = 8.f;    // rescale O only when the max grows by > 2^8
+constexpr float kSumLimit = 1099511627776.f;   // 2^40: largest tile row sum kept without a new max
 
 template <int D>
 struct Layout {
@@ -68,8 +73,9 @@ struct Bars {  // mbarrier indices inside the barrier block (8 bytes each)
   static constexpr int q_full = 0;                     // + tile
   static constexpr int k_full = q_full + kQT;          // + stage
   static constexpr int v_full = k_full + kStages;      // + stage
-  static constexpr int kv_empty = v_full + kStages;    // + stage
-  static constexpr int s_full = kv_empty + kStages;    // + tile
+  static constexpr int k_empty = v_full + kStages;     // + stage: freed by the last S MMA reading it
+  static constexpr int v_empty = k_empty + kStages;    // + stage: freed by the last PV MMA reading it
+  static constexpr int s_full = v_empty + kStages;     // + tile
   static constexpr int p_full = s_full + kQT;          // + tile
   static constexpr int pv_done = p_full + kQT;         // + tile
   static constexpr int drain = pv_done + kQT;          // last commit of the MMA thread
@@ -146,7 +152,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(Bars::k_full + s), 1);
       mbar_init(bar(Bars::v_full + s), 1);
-      mbar_init(bar(Bars::kv_empty + s), 1);
+      mbar_init(bar(Bars::k_empty + s), 1);
+      mbar_init(bar(Bars::v_empty + s), 1);
     }
     mbar_init(bar(Bars::drain), 1);
     fence_mbar_init();
@@ -196,32 +203,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == kTmaWarp) {
     // ================================ TMA producer =====================================
     if (lane == 0) {
-      int issued = 0;
+      int issued_k = 0, issued_v = 0;
       for (int t = 0; t < kQT; ++t) {
         mbar_expect_tx(bar(Bars::q_full + t), L::kSub * kSubBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d(sbase + L::kQ + (t * L::kSub + s) * kSubBytes, &tmQ, 64 * s, h,
                       static_cast<int>(row0 + t * kBM), bar(Bars::q_full + t));
       }
+      // K and V stages are freed separately: a K stage as soon as the last S MMA
+      // reading it completes (about one period before its PV stage), so the next
+      // K tile streams in while the current P.V products still run.
       for (int j = 0; j < ntiles; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(bar(Bars::kv_empty + st), ((j / kStages) - 1) & 1, &s_abort, prm.status))
-          break;
+        const uint32_t ph = ((j / kStages) - 1) & 1;
         const int key0 = tile_kb(j) * kBN;
+        if (j >= kStages && !mbar_wait(bar(Bars::k_empty + st), ph, &s_abort, prm.status)) break;
         mbar_expect_tx(bar(Bars::k_full + st), L::kSub * kSubBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d(sbase + L::kK + (st * L::kSub + s) * kSubBytes, &tmK, 64 * s, h, key0, bar(Bars::k_full + st));
+        issued_k = j + 1;
+        if (j >= kStages && !mbar_wait(bar(Bars::v_empty + st), ph, &s_abort, prm.status)) break;
         mbar_expect_tx(bar(Bars::v_full + st), L::kSub * kSubBytes);
         for (int s = 0; s < L::kSub; ++s)
           tma_load_3d(sbase + L::kV + (st * L::kSub + s) * kSubBytes, &tmV, 64 * s, h, key0, bar(Bars::v_full + st));
-        issued = j + 1;
+        issued_v = j + 1;
       }
       // drain: every load issued above must land before the CTA may exit
       for (int t = 0; t < kQT; ++t) drain_wait(bar(Bars::q_full + t), 0);
-      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j) {
+      for (int j = issued_k > kStages ? issued_k - kStages : 0; j < issued_k; ++j)
         drain_wait(bar(Bars::k_full + j % kStages), (j / kStages) & 1);
+      for (int j = issued_v > kStages ? issued_v - kStages : 0; j < issued_v; ++j)
         drain_wait(bar(Bars::v_full + j % kStages), (j / kStages) & 1);
-      }
     }
   } else if (warp == kMmaWarp) {
     // ================================ MMA issuer =======================================
@@ -238,6 +250,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_f16_ss(tS(t), da, db, kIdescS, kk > 0);
         }
         mma_commit(bar(Bars::s_full + t));
+        if (t == kQT - 1) mma_commit(bar(Bars::k_empty + st));   // last reader of this K stage
       };
       bool ok = ntiles > 0;
       if (ok) ok = mbar_wait(bar(Bars::k_full), 0, &s_abort, prm.status);
@@ -262,7 +275,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mma_f16_ts(tO(t), tS(t) + 8 * kk, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(Bars::pv_done + t));
-          if (t == kQT - 1) mma_commit(bar(Bars::kv_empty + st));
+          if (t == kQT - 1) mma_commit(bar(Bars::v_empty + st));   // last reader of this V stage
           if (j + 1 < ntiles) {
             // S_t(j+1) overwrites the columns P_t(j) was read from: tcgen05.mma
             // operations of one thread execute in issue order.
@@ -299,68 +312,88 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      uint32_t sr[kBN];
-      tmem_ld128(tS(t) + lane_off, sr);
-
       const int kb = tile_kb(j);
       const int64_t key0 = static_cast<int64_t>(kb) * kBN;
       const bool row_ok = !p.bm || p.bm[static_cast<int64_t>(qb) * p.nb + kb] != 0;
       const int nvalid = row_ok ? static_cast<int>(p.N - key0 < kBN ? p.N - key0 : kBN) : 0;
-      if (nvalid < kBN) {
+      uint32_t sr[kBN];
+      auto load_s = [&]() {
+        tmem_ld128(tS(t) + lane_off, sr);
+        if (nvalid < kBN) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
-#pragma unroll
-      for (int c = 4; c < kBN; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
-      }
-      const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
-      if (j == 0) {
-        m_run = m_new;
-      } else if (__any_sync(0xffffffffu, m_new - m_run > kRescaleLog2)) {
-        // the warp moves its reference maxima; O (complete up to tile j-1) is rescaled
-        const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
-          ok = false;
-          break;
+          for (int c = 0; c < kBN; ++c)
+            if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
         }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {           // 32 columns at a time: S stays in registers
-          float o[32];
-          tmem_ld32(tO(t) + lane_off + c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO(t) + lane_off + c, o);
-        }
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      const float base = m_run == -INFINITY ? 0.f : m_run;
-      const uint64_t nbase = f2_pack(-base, -base);
-      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+      };
       uint32_t pk[kBN / 2];
+      // P = exp2(S * scale_log2 - base) as bf16 pairs into pk; returns the row sum of this tile
+      auto exp_pass = [&](float base) -> float {
+        const uint64_t nbase = f2_pack(-base, -base);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-      for (int c = 0; c < kBN; c += 4) {
-        float a0, a1, a2, a3;
-        f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
-        f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
-        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
-        acc0 = fadd2(acc0, f2_pack(p0, p1));
-        acc1 = fadd2(acc1, f2_pack(p2, p3));
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-        pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
+        for (int c = 0; c < kBN; c += 4) {
+          float a0, a1, a2, a3;
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+          acc0 = fadd2(acc0, f2_pack(p0, p1));
+          acc1 = fadd2(acc1, f2_pack(p2, p3));
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
+        }
+        float s0, s1, s2, s3;
+        f2_unpack(acc0, s0, s1);
+        f2_unpack(acc1, s2, s3);
+        return (s0 + s1) + (s2 + s3);
+      };
+      load_s();
+      // Fast path: keep the running reference max and skip the row max. Softmax is
+      // exact for any reference; the tile's sum bounds every P, so P stays finite
+      // and well inside bf16/fp32 range while the sum is at most kSumLimit.
+      bool slow = j == 0;
+      float lt = 0.f;
+      if (!slow) {
+        const float base = m_run == -INFINITY ? 0.f : m_run;
+        lt = exp_pass(base);
+        slow = __any_sync(0xffffffffu, !(lt <= kSumLimit));
+        if (slow) load_s();                         // S is intact: P has not been stored yet
+        else m_run = base;                          // a row with only masked keys so far now uses 0
       }
-      float s0, s1, s2, s3;
-      f2_unpack(acc0, s0, s1);
-      f2_unpack(acc1, s2, s3);
-      l_run += (s0 + s1) + (s2 + s3);
+      if (slow) {
+        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+        float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+        for (int c = 4; c < kBN; c += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+        }
+        const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+        if (j == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m_run)) {
+          // the warp moves its reference maxima; O (complete up to tile j-1) is rescaled
+          const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {         // 32 columns at a time: S stays in registers
+            float o[32];
+            tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO(t) + lane_off + c, o);
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        lt = exp_pass(m_run == -INFINITY ? 0.f : m_run);
+      }
+      l_run += lt;
       tmem_st64(tS(t) + lane_off, pk);            // P_t(j) over the first 64 columns of S_t
       tc_fence_before();
       mbar_arrive(bar(Bars::p_full + t));

@@ -656,6 +656,12 @@ extern "C" size_t tps_workspace_size(int op, int64_t N, int K) {
   return tps::ws_bytes_for(op, N, K);
 }
 
+extern "C" size_t tps_workspace_min_size(int op, int64_t N, int K) {
+  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
+  if (N < 0) return 0;
+  return tps::ws_min_bytes(op, N, K);
+}
+
 extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
                             int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                             tps_stream stream) {

@@ -45,6 +45,7 @@ SIGNATURES = {
     "timeripple_score": (_INT, [_P, _I64, _I64, _I64, _INT, _INT, _P, _P, _P, _P, _P, _P]),
     "timeripple_theta": (C.c_float, [_INT, C.c_float, C.c_float, _INT, _INT]),
     "tps_workspace_size": (C.c_size_t, [_INT, _I64, _INT]),
+    "tps_workspace_min_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_last_error": (C.c_char_p, []),
     "tps_check": (_INT, [_P]),
     "tps_philox_fill": (_INT, [_P, C.c_uint64, _I64, C.c_uint64, C.c_uint32, C.c_uint32, _P]),
@@ -102,8 +103,13 @@ def workspace_size(op: int, N: int, K: int = 0) -> int:
     return int(lib().tps_workspace_size(op, N, K))
 
 
-def workspace(op: int, N: int, K: int = 0, device=None) -> torch.Tensor:
-    return torch.empty(max(workspace_size(op, N, K), 16), dtype=torch.uint8, device=device or "cuda")
+def workspace_min_size(op: int, N: int, K: int = 0) -> int:
+    return int(lib().tps_workspace_min_size(op, N, K))
+
+
+def workspace(op: int, N: int, K: int = 0, device=None, minimal: bool = False) -> torch.Tensor:
+    n = workspace_min_size(op, N, K) if minimal else workspace_size(op, N, K)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
 
 
 # ---- the path -----------------------------------------------------------------------
