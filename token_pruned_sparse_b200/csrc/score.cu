@@ -129,70 +129,47 @@ __global__ void __launch_bounds__(256) score_motion_kernel(const uint16_t* __res
                                                            int Lkey, float* __restrict__ score) {
   constexpr int kTokPerWarp = 32 / L;
   constexpr int C = kV * 8;
-  constexpr int kG = 2;                            // token groups per lane and iteration
   const int lane = threadIdx.x & 31;
   const int sub = lane & (L - 1);
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t stride = nwarps * kTokPerWarp;
-  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += kG * stride) {
-    int64_t tt[kG];
-    bool valid[kG], first[kG];
-    const uint16_t* cur[kG];
-    const uint16_t* r1[kG];
-    const uint16_t* r2[kG];
-#pragma unroll
-    for (int g = 0; g < kG; ++g) {
-      const int64_t t = w0 + g * stride + lane / L;
-      tt[g] = t;
-      valid[g] = t < N;
-      const int64_t f = valid[g] ? t / HW : 0;
-      first[g] = f == 0;
+  for (int64_t w0 = warp * kTokPerWarp; w0 < N; w0 += nwarps * kTokPerWarp) {
+    const int64_t t = w0 + lane / L;
+    const bool valid = t < N;
+    const int64_t f = valid ? t / HW : 0;
+    const bool first = f == 0;
+    float n1 = 0.f, d1 = 0.f, n2 = 0.f, d2 = 0.f;
+    if (valid && !first) {
       const int64_t fl = f - Lkey > 0 ? f - Lkey : 0;
-      const bool work = valid[g] && !first[g];
-      cur[g] = work ? x + t * C : nullptr;
-      r1[g] = work ? x + (t - HW) * C : nullptr;
-      r2[g] = work ? x + (t - (f - fl) * HW) * C : nullptr;
-    }
-    float n1[kG], d1[kG], n2[kG], d2[kG];
+      const uint16_t* cur = x + t * C;
+      const uint16_t* r1 = x + (t - HW) * C;
+      const uint16_t* r2 = x + (t - (f - fl) * HW) * C;
 #pragma unroll
-    for (int g = 0; g < kG; ++g) n1[g] = d1[g] = n2[g] = d2[g] = 0.f;
+      for (int v = sub; v < kV; v += L) {
+        const uint4 a = ld16(cur + v * 8), b = ld16(r1 + v * 8), c = ld16(r2 + v * 8);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int v = sub; v < kV; v += L) {
-      uint4 a[kG], b[kG], c[kG];
-#pragma unroll
-      for (int g = 0; g < kG; ++g)
-        if (cur[g]) a[g] = ld16(cur[g] + v * 8), b[g] = ld16(r1[g] + v * 8), c[g] = ld16(r2[g] + v * 8);
-#pragma unroll
-      for (int g = 0; g < kG; ++g)
-        if (cur[g]) {
-          const uint32_t aw[4] = {a[g].x, a[g].y, a[g].z, a[g].w}, bw[4] = {b[g].x, b[g].y, b[g].z, b[g].w},
-                         cw[4] = {c[g].x, c[g].y, c[g].z, c[g].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
-            const float p0 = bf16lo(bw[i]), p1 = bf16hi(bw[i]);
-            const float k0 = bf16lo(cw[i]), k1 = bf16hi(cw[i]);
-            n1[g] += fabsf(c0 - p0) + fabsf(c1 - p1);
-            d1[g] += fabsf(p0) + fabsf(p1);
-            n2[g] += fabsf(c0 - k0) + fabsf(c1 - k1);
-            d2[g] += fabsf(k0) + fabsf(k1);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
+          const float p0 = bf16lo(bw[i]), p1 = bf16hi(bw[i]);
+          const float k0 = bf16lo(cw[i]), k1 = bf16hi(cw[i]);
+          n1 += fabsf(c0 - p0) + fabsf(c1 - p1);
+          d1 += fabsf(p0) + fabsf(p1);
+          n2 += fabsf(c0 - k0) + fabsf(c1 - k1);
+          d2 += fabsf(k0) + fabsf(k1);
         }
+      }
     }
 #pragma unroll
-    for (int g = 0; g < kG; ++g) {
-#pragma unroll
-      for (int o = L / 2; o > 0; o >>= 1) {
-        n1[g] += __shfl_xor_sync(0xffffffffu, n1[g], o);
-        d1[g] += __shfl_xor_sync(0xffffffffu, d1[g], o);
-        n2[g] += __shfl_xor_sync(0xffffffffu, n2[g], o);
-        d2[g] += __shfl_xor_sync(0xffffffffu, d2[g], o);
-      }
-      if (valid[g] && sub == 0) {
-        auto ratio = [](float n, float d) { return d > 0.f ? n / d : (n > 0.f ? INFINITY : 0.f); };
-        score[tt[g]] = first[g] ? INFINITY : fmaxf(ratio(n1[g], d1[g]), ratio(n2[g], d2[g]));
-      }
+    for (int o = L / 2; o > 0; o >>= 1) {
+      n1 += __shfl_xor_sync(0xffffffffu, n1, o);
+      d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+      n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+      d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+    }
+    if (valid && sub == 0) {
+      auto ratio = [](float n, float d) { return d > 0.f ? n / d : (n > 0.f ? INFINITY : 0.f); };
+      score[t] = first ? INFINITY : fmaxf(ratio(n1, d1), ratio(n2, d2));
     }
   }
 }
@@ -211,7 +188,7 @@ extern "C" int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int6
   const int64_t N = F * HW;
   constexpr int kThreads = 256;
   const int64_t tok_per_block = (kThreads / 32) * 4;
-  int64_t blocks = (N + 2 * tok_per_block - 1) / (2 * tok_per_block);
+  int64_t blocks = (N + tok_per_block - 1) / tok_per_block;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
