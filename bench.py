@@ -164,20 +164,52 @@ class MidStep:
         self.flops = 4.0 * self.d * self.H * self.k * self.N
         self.launches = sum(LAUNCHES.values())
 
-    def step(self, ev_attn=None):
+    def _pre(self, inp=None):
         t = self.tps
-        t.lipar_score(self.x, out=self.score)
+        x, q, kf, vf = (self.x, self.q, self.kf, self.vf) if inp is None else inp
+        t.lipar_score(x, out=self.score)
         t.lipar_select(self.score, t.SELECT_TOPK, k=self.k, idx=self.idx, count=self.cnt, ws=self.ws)
-        t.tps_gather_rows(self.q_act, self.q, self.idx, self.cnt)
-        t.tps_gather_rows(self.k_new, self.kf, self.idx, self.cnt)
-        t.tps_gather_rows(self.v_new, self.vf, self.idx, self.cnt)
+        t.tps_gather_rows(self.q_act, q, self.idx, self.cnt)
+        t.tps_gather_rows(self.k_new, kf, self.idx, self.cnt)
+        t.tps_gather_rows(self.v_new, vf, self.idx, self.cnt)
         t.kv_sync(self.kc, self.vc, self.k_new, self.v_new, self.idx, self.cnt)
+
+    def _post(self):
+        self.tps.scatter_out(self.o_full, self.o_act, self.idx, self.cnt)
+
+    def capture_graphs(self) -> bool:
+        """Capture the stages before and after attention as two CUDA graphs
+        (score, select, gathers, kv_sync; scatter_out), replayed each step; the
+        attention launch stays outside so its own events time it. Returns False
+        (eager launches) if capture is not possible."""
+        try:
+            self.g_pre, self.g_post = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_pre):
+                self._pre()
+            with torch.cuda.graph(self.g_post):
+                self._post()
+            torch.cuda.synchronize()
+            self.graphs = True
+        except Exception as e:        # noqa: BLE001 - report and run eagerly
+            print(f"bench: CUDA graph capture unavailable ({e}); eager launches", file=sys.stderr)
+            self.g_pre = self.g_post = None
+            self.graphs = False
+        return self.graphs
+
+    def step(self, ev_attn=None):
+        if getattr(self, "graphs", False):
+            self.g_pre.replay()
+        else:
+            self._pre()
         if ev_attn:
             ev_attn[0].record()
         self.attn_fn(self.q_act, self.kc, self.vc, self.idx, self.cnt, self.scale, o_act=self.o_act)
         if ev_attn:
             ev_attn[1].record()
-        t.scatter_out(self.o_full, self.o_act, self.idx, self.cnt)
+        if getattr(self, "graphs", False):
+            self.g_post.replay()
+        else:
+            self._post()
 
 
 def rank_seed_offset(rank: int) -> int:
@@ -566,6 +598,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
     ap.add_argument("--kernel-case", choices=["timeripple"], default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
@@ -601,6 +634,10 @@ def main():
         return 0
     st = MidStep(rank_seed_offset(rank), dev, a.attn)
     flush = L2Flush(dev)
+    st.step()                     # first eager step: one-time setup (status word, occupancy queries)
+    torch.cuda.synchronize()
+    if not a.no_graph:
+        st.capture_graphs()
     for _ in range(a.warmup):
         st.step()
     torch.cuda.synchronize()
@@ -661,7 +698,8 @@ def main():
                    "N": st.N, "active": st.k, "heads": st.H, "head_dim": st.d,
                    "l2": "flushed between timed steps (512 MiB write, then 512 MiB read: L2 left clean)",
                    "parallelism": f"replicas x{world}",
-                   "attn_kernel": roofline["kernel"]},
+                   "attn_kernel": roofline["kernel"],
+                   "cuda_graphs": bool(getattr(st, "graphs", False))},
         "active_tokens_per_s": round(tok_s, 1),
         "gpu_launches": st.launches * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
@@ -674,33 +712,68 @@ def main():
 def e2e_leg(st, dev, steps, world):
     """Same metric through the C ABI with host buffers: each step copies the
     step's inputs (latents + Q/K/V projections) from pinned host memory and
-    reads the full output back; copies are inside the timed region."""
+    reads the full output back; copies are inside the timed region.
+
+    The copies overlap the computation on separate streams, as a serving loop
+    would run them: step i+1's inputs stream in (into the second of two device
+    input sets) while step i computes, and step i's output is copied to a
+    device staging buffer and read back while step i+1 runs."""
     host_in = {k: v.pin_memory() for k, v in st.host.items()}
-    host_out = torch.empty((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory()
+    host_out = [torch.empty((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    sets = [(st.x, st.q, st.kf, st.vf),
+            tuple(torch.empty_like(t) for t in (st.x, st.q, st.kf, st.vf))]
+    stage = [torch.empty_like(st.o_full) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()            # noqa: E731
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    out_ready, out_free = [ev(), ev()], [ev(), ev()]
+    for e in in_free + out_free:
+        e.record(comp)
 
-    def one():
-        st.x.copy_(host_in["x"], non_blocking=True)
-        st.q.copy_(host_in["q"], non_blocking=True)
-        st.kf.copy_(host_in["k"], non_blocking=True)
-        st.vf.copy_(host_in["v"], non_blocking=True)
-        st.step()
-        host_out.copy_(st.o_full, non_blocking=True)
+    def copy_in(i):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(in_free[b])
+            for dst, key in zip(sets[b], ("x", "q", "k", "v")):
+                dst.copy_(host_in[key], non_blocking=True)
+            in_ready[b].record(s_in)
 
-    for _ in range(2):
-        one()
+    def run(n):
+        copy_in(0)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:
+                copy_in(i + 1)
+            comp.wait_event(in_ready[b])
+            st._pre(sets[b])
+            in_free[b].record(comp)
+            st.attn_fn(st.q_act, st.kc, st.vc, st.idx, st.cnt, st.scale, o_act=st.o_act)
+            st._post()
+            comp.wait_event(out_free[b])
+            stage[b].copy_(st.o_full, non_blocking=True)
+            out_ready[b].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[b])
+                host_out[b].copy_(stage[b], non_blocking=True)
+                out_free[b].record(s_out)
+        comp.wait_stream(s_out)
+
+    run(2)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
+    a.record(comp)
+    s_in.wait_event(a)
+    run(steps)
+    b.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
     return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": round(ms / steps, 4)}
+            "ms_per_step": round(ms / steps, 4),
+            "overlap": "H2D of step i+1 and D2H of step i-1 run beside step i on two copy streams"}
 
 
 def reference_arm(a, rank, world):
