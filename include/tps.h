@@ -183,7 +183,9 @@ TPS_API int lipar_schedule(const int8_t* group, int64_t N, int K, const int32_t*
 /* ---- gather of active rows ([HSA] 2.2 (1): only active tokens enter the
  * QKV projection) --------------------------------------------------------------
  * dst[j] = src[idx[j]] for j < min(*count, cap); rows of row_bytes bytes
- * (row_bytes % 16 == 0); src has N rows, dst cap rows. */
+ * (row_bytes % 16 == 0); src has N rows, dst cap rows. src may also be pinned
+ * host memory mapped into the device's address space (see
+ * tps_pointer_is_device_accessible): only the active rows then cross PCIe. */
 TPS_API int tps_gather_rows(void* dst, const void* src, const int32_t* idx, const int32_t* count,
                     int64_t cap, int64_t N, int64_t row_bytes, tps_stream stream);
 
@@ -267,7 +269,8 @@ TPS_API int attn_lse_merge(const tps_bf16* o1, const float* lse1, const tps_bf16
 
 /* ---- step 6: restoration ([LIPAR] Dutch summary 2.D) -------------------------
  * o_full[idx[j]] = o_act[j] for j < min(*count, cap); every other row of
- * o_full [N, H, d] keeps its cached output bit for bit. */
+ * o_full [N, H, d] keeps its cached output bit for bit. o_full may also be
+ * pinned, device-mapped host memory: only the active rows then cross PCIe. */
 TPS_API int scatter_out(tps_bf16* o_full, const tps_bf16* o_act, const int32_t* idx,
                 const int32_t* count, int64_t cap, int64_t N, int H, int d, tps_stream stream);
 
@@ -295,6 +298,12 @@ TPS_API size_t tps_workspace_size(int op, int64_t N, int K);
 /* The smallest workspace those calls accept (0 on bad op): enough for the
  * multi-launch path only. Results are identical with either size. */
 TPS_API size_t tps_workspace_min_size(int op, int64_t N, int K);
+
+/* 1 if kernels of the current device may dereference p: device or managed
+ * memory, or pinned host memory mapped into the device's address space at the
+ * same address (the unified-addressing case); 0 otherwise (pageable host
+ * memory, unknown pointers). Host-only query; it never faults. */
+TPS_API int tps_pointer_is_device_accessible(const void* p);
 
 /* Message of the last failing call on this host thread ("" if none). */
 TPS_API const char* tps_last_error(void);

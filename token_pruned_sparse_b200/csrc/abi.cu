@@ -79,6 +79,24 @@ extern "C" {
 
 const char* tps_last_error(void) { return tps::g_msg; }
 
+int tps_pointer_is_device_accessible(const void* p) {
+  if (!p) return 0;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();   // clear the (non-sticky) error an unknown pointer leaves behind
+    return 0;
+  }
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+      return 1;
+    case cudaMemoryTypeHost:
+      return a.devicePointer == p ? 1 : 0;
+    default:
+      return 0;
+  }
+}
+
 const char* tps_version(void) { return "libtps 0.1.0 (sm_100a)"; }
 
 int tps_check(tps_stream stream) {

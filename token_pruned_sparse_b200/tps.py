@@ -47,6 +47,7 @@ SIGNATURES = {
     "tps_workspace_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_workspace_min_size": (C.c_size_t, [_INT, _I64, _INT]),
     "tps_last_error": (C.c_char_p, []),
+    "tps_pointer_is_device_accessible": (_INT, [_P]),
     "tps_check": (_INT, [_P]),
     "tps_philox_fill": (_INT, [_P, C.c_uint64, _I64, C.c_uint64, C.c_uint32, C.c_uint32, _P]),
     "tps_wait_probe": (_INT, [_I64, _P]),
@@ -296,6 +297,12 @@ def timeripple_score(x, F, Hs, Ws, windows, theta, reuse=None, delta=False, scor
 
 def timeripple_theta(step, theta_lo, theta_hi, i0=11, i1=21) -> float:
     return float(lib().timeripple_theta(int(step), float(theta_lo), float(theta_hi), int(i0), int(i1)))
+
+
+def pointer_is_device_accessible(t) -> bool:
+    """True if library kernels may read/write tensor t in place (device memory,
+    or pinned host memory mapped into the device address space)."""
+    return bool(lib().tps_pointer_is_device_accessible(_P(t.data_ptr())))
 
 
 def tps_check(stream=None):
