@@ -164,3 +164,25 @@ def test_bounded_wait_gives_up_and_context_survives():
     tps.scatter_out(full, act, di, dc, cap=4)
     tps.tps_check()
     assert torch.equal(full.cpu()[[1, 7, 30, 63]], act.cpu())
+
+
+def test_gather_and_scatter_through_pinned_host_memory():
+    """Zero-copy use: gathers read rows straight from pinned host memory and
+    scatter_out writes rows straight into it; results are the oracle's, bit
+    for bit, and pageable memory is reported as not device-accessible."""
+    N, H, d, A = 3000, 4, 128, 777
+    full = synth.gaussian_bf16((N, H, d), 21).pin_memory()
+    assert tps.pointer_is_device_accessible(full)
+    assert not tps.pointer_is_device_accessible(torch.zeros(16))       # pageable
+    idx = np.sort(np.random.default_rng(22).choice(N, A, replace=False)).astype(np.int32)
+    di, dc = _dev_idx(idx)
+    g = torch.empty((A, H, d), dtype=torch.bfloat16, device=DEV)
+    tps.tps_gather_rows(g, full, di, dc, cap=A)
+    tps.tps_check()
+    assert torch.equal(g.cpu(), O.gather_rows(full, idx))
+    out = synth.gaussian_bf16((N, H, d), 23).pin_memory()
+    before = out.clone()
+    act = synth.gaussian_bf16((A, H, d), 24)
+    tps.scatter_out(out, act.to(DEV), di, dc, cap=A)
+    tps.tps_check()
+    assert torch.equal(out, O.scatter_out(before, act, idx))
