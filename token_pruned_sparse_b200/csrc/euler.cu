@@ -8,10 +8,11 @@
 //
 // Fused, HBM-bound single pass: the velocity cache is refreshed for the active
 // rows and every row of the fp32 state advances, v read once per token. A warp
-// owns a run of 8 consecutive tokens: one warp-cooperative search in the ascending index
-// list finds the run's active entries, a warp-wide OR builds the run's active
-// mask, and the warp then sweeps the run's (token, 16-byte vector) items with
-// several loads in flight per lane.
+// owns a group of 4 runs of 8 consecutive tokens: one warp-cooperative search in
+// the ascending index list finds the group's first active entry, and each run
+// continues from where the previous one stopped. Per run a warp-wide OR builds
+// the run's active mask, and the warp then sweeps the run's (token, 16-byte
+// vector) items with several loads in flight per lane.
 #include "tps_internal.cuh"
 #include "warp_search.cuh"
 
@@ -37,45 +38,50 @@ __global__ void __launch_bounds__(kThreads) euler_kernel(float* __restrict__ x, 
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
   const int64_t nruns = (N + kRun - 1) / kRun;
   const int items = kRun * vpr;                 // (token, vector) pairs of one run
-  for (int64_t run = warp; run < nruns; run += nwarps) {
-    const int64_t r0 = run * kRun;
-    const int64_t lo = warp_lower_bound(idx, cnt, r0, lane);   // first list entry >= r0
-    // lanes 0..7 look at the next 8 list entries; those below r0 + 8 are active rows of this run
-    const int64_t mine = (lane < kRun && lo + lane < cnt) ? idx[lo + lane] : INT64_MAX;
-    const bool in_run = mine >= r0 && mine < r0 + kRun;
-    const unsigned int rowbits =
-        __reduce_or_sync(0xffffffffu, in_run ? (1u << static_cast<unsigned int>(mine - r0)) : 0u);
-    const unsigned int nin = __popc(__ballot_sync(0xffffffffu, in_run));
-    if (lane == 0) {
-      // duplicates in the list, or entries outside [0, N), are not consumed
-      if (nin != static_cast<unsigned int>(__popc(rowbits))) raise_status(status, STATUS_BOUNDS);
-      if (run == nruns - 1 && cnt > 0 && (idx[cnt - 1] >= N || idx[0] < 0)) raise_status(status, STATUS_BOUNDS);
-    }
-#pragma unroll
-    for (int i = lane; i < (kVpr > 0 ? kRun * kVpr : items); i += 32) {
-      const int r = i / vpr, v = i - r * vpr;
-      const int64_t n = r0 + r;
-      if (n >= N) continue;
-      uint4 vel;
-      if ((rowbits >> r) & 1u) {
-        const int64_t pos = lo + __popc(rowbits & ((1u << r) - 1u));
-        vel = vfresh[pos * vpr + v];
-        vcache[n * vpr + v] = vel;
-      } else {
-        vel = vcache[n * vpr + v];
+  constexpr int kGroup = 4;                     // runs per search: later runs continue from the last
+  const int64_t ngroups = (nruns + kGroup - 1) / kGroup;
+  for (int64_t grp = warp; grp < ngroups; grp += nwarps) {
+    int64_t lo = warp_lower_bound(idx, cnt, grp * kGroup * kRun, lane);   // first list entry >= the group start
+    for (int64_t run = grp * kGroup; run < nruns && run < (grp + 1) * kGroup; ++run) {
+      const int64_t r0 = run * kRun;
+      // lanes 0..7 look at the next 8 list entries; those below r0 + 8 are active rows of this run
+      const int64_t mine = (lane < kRun && lo + lane < cnt) ? idx[lo + lane] : INT64_MAX;
+      const bool in_run = mine >= r0 && mine < r0 + kRun;
+      const unsigned int rowbits =
+          __reduce_or_sync(0xffffffffu, in_run ? (1u << static_cast<unsigned int>(mine - r0)) : 0u);
+      const unsigned int nin = __popc(__ballot_sync(0xffffffffu, in_run));
+      if (lane == 0) {
+        // duplicates in the list, or entries outside [0, N), are not consumed
+        if (nin != static_cast<unsigned int>(__popc(rowbits))) raise_status(status, STATUS_BOUNDS);
+        if (run == nruns - 1 && cnt > 0 && (idx[cnt - 1] >= N || idx[0] < 0)) raise_status(status, STATUS_BOUNDS);
       }
-      float4* xp = reinterpret_cast<float4*>(x + (n * vpr + v) * 8);
-      float4 x0 = xp[0], x1 = xp[1];
-      x0.x = fmaf(dsigma, bf16lo(vel.x), x0.x);
-      x0.y = fmaf(dsigma, bf16hi(vel.x), x0.y);
-      x0.z = fmaf(dsigma, bf16lo(vel.y), x0.z);
-      x0.w = fmaf(dsigma, bf16hi(vel.y), x0.w);
-      x1.x = fmaf(dsigma, bf16lo(vel.z), x1.x);
-      x1.y = fmaf(dsigma, bf16hi(vel.z), x1.y);
-      x1.z = fmaf(dsigma, bf16lo(vel.w), x1.z);
-      x1.w = fmaf(dsigma, bf16hi(vel.w), x1.w);
-      xp[0] = x0;
-      xp[1] = x1;
+#pragma unroll
+      for (int i = lane; i < (kVpr > 0 ? kRun * kVpr : items); i += 32) {
+        const int r = i / vpr, v = i - r * vpr;
+        const int64_t n = r0 + r;
+        if (n >= N) continue;
+        uint4 vel;
+        if ((rowbits >> r) & 1u) {
+          const int64_t pos = lo + __popc(rowbits & ((1u << r) - 1u));
+          vel = vfresh[pos * vpr + v];
+          vcache[n * vpr + v] = vel;
+        } else {
+          vel = vcache[n * vpr + v];
+        }
+        float4* xp = reinterpret_cast<float4*>(x + (n * vpr + v) * 8);
+        float4 x0 = xp[0], x1 = xp[1];
+        x0.x = fmaf(dsigma, bf16lo(vel.x), x0.x);
+        x0.y = fmaf(dsigma, bf16hi(vel.x), x0.y);
+        x0.z = fmaf(dsigma, bf16lo(vel.y), x0.z);
+        x0.w = fmaf(dsigma, bf16hi(vel.y), x0.w);
+        x1.x = fmaf(dsigma, bf16lo(vel.z), x1.x);
+        x1.y = fmaf(dsigma, bf16hi(vel.z), x1.y);
+        x1.z = fmaf(dsigma, bf16lo(vel.w), x1.z);
+        x1.w = fmaf(dsigma, bf16hi(vel.w), x1.w);
+        xp[0] = x0;
+        xp[1] = x1;
+      }
+      lo += nin;                                   // the next run's entries start after this run's
     }
   }
 }
@@ -98,7 +104,7 @@ extern "C" int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_f
   int err;
   unsigned int* st = device_status(&err);
   if (!st) return err;
-  const int64_t runs = (N + kRun - 1) / kRun;
+  const int64_t runs = ((N + kRun - 1) / kRun + 4 - 1) / 4;   // groups of runs
   int64_t grid = (runs + kWarps - 1) / kWarps;
   const int64_t maxg = static_cast<int64_t>(sm_count()) * 8;
   if (grid > maxg) grid = maxg;
