@@ -326,6 +326,12 @@ TPS_API int tps_philox_fill(uint32_t* out, uint64_t q0, int64_t nq, uint64_t see
  * context stays usable; tps_check() then returns TPS_ERR_TIMEOUT once. */
 TPS_API int tps_wait_probe(int64_t limit_cycles, tps_stream stream);
 
+/* Test hook (host-side fault injection): the next n launches report
+ * TPS_ERR_CUDA ("injected launch failure") instead of success. The kernels
+ * still run; the hook exercises the error path of every entry point and of
+ * its callers without faulting a GPU. n <= 0 clears it. */
+TPS_API void tps_debug_inject_launch_failures(int n);
+
 /* Library version string. */
 TPS_API const char* tps_version(void);
 

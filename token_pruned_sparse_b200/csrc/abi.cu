@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "tps_internal.cuh"
@@ -29,7 +30,18 @@ int cuda_status(cudaError_t e, const char* what) {
   return fail(TPS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-int launch_status(const char* what) { return cuda_status(cudaGetLastError(), what); }
+// Host-side fault injection for tests: the next n launch checks report a launch
+// failure (after consuming the real launch status) instead of success.
+static std::atomic<int> g_inject_launch_failures{0};
+
+int launch_status(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  int n = g_inject_launch_failures.load();
+  while (n > 0 && !g_inject_launch_failures.compare_exchange_weak(n, n - 1)) {
+  }
+  if (n > 0) return fail(TPS_ERR_CUDA, "%s: injected launch failure (test hook)", what);
+  return cuda_status(e, what);
+}
 
 // One status word per device: bit 0 = an out-of-range index was skipped,
 // bit 1 = a bounded wait gave up.
@@ -78,6 +90,8 @@ int sm_count() {
 extern "C" {
 
 const char* tps_last_error(void) { return tps::g_msg; }
+
+void tps_debug_inject_launch_failures(int n) { tps::g_inject_launch_failures.store(n > 0 ? n : 0); }
 
 int tps_pointer_is_device_accessible(const void* p) {
   if (!p) return 0;

@@ -10,6 +10,7 @@
 // head (16 per warp) and streams 64-key K/V tiles through shared memory with
 // cp.async double buffering. In masked mode the CTA first builds the list of
 // key blocks that any of its query blocks keeps and loads only those tiles.
+#include "trace.cuh"
 #include "attn_common.cuh"
 
 namespace tps {
@@ -318,6 +319,7 @@ extern "C" int pruned_attn_mma(const tps_bf16* q_act, const tps_bf16* k, const t
                                const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H,
                                int d, float scale, const uint8_t* blockmask, int block, tps_bf16* o_act,
                                float* lse, tps_stream stream) {
+  TPS_TRACE("pruned_attn_mma");
   using namespace tps;
   AttnArgs a;
   if (int e = attn_validate("pruned_attn_mma", q_act, k, v, idx, count, cap, N, H, d, scale, blockmask,

@@ -35,6 +35,7 @@
 // frees TMEM and returns.
 #include <mutex>
 
+#include "trace.cuh"
 #include "attn_common.cuh"
 #include "tc_ptx.cuh"
 
@@ -570,6 +571,7 @@ extern "C" int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tp
                               const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,
                               const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse, void* ws,
                               size_t ws_bytes, tps_stream stream) {
+  TPS_TRACE("pruned_attn_ws");
   using namespace tps;
   AttnArgs a;
   if (int e = attn_validate("pruned_attn_ws", q_act, k, v, idx, count, cap, N, H, d, scale, blockmask, block, o_act,
@@ -594,6 +596,7 @@ extern "C" int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tp
 extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
                            const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,
                            const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse, tps_stream stream) {
+  TPS_TRACE("pruned_attn");
   using namespace tps;
   AttnArgs a;
   if (int e = attn_validate("pruned_attn", q_act, k, v, idx, count, cap, N, H, d, scale, blockmask, block, o_act,

@@ -13,6 +13,7 @@
 // continues from where the previous one stopped. Per run a warp-wide OR builds
 // the run's active mask, and the warp then sweeps the run's (token, 16-byte
 // vector) items with several loads in flight per lane.
+#include "trace.cuh"
 #include "tps_internal.cuh"
 #include "warp_search.cuh"
 
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(kThreads) euler_kernel(float* __restrict__ x, 
 extern "C" int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_fresh, const int32_t* idx,
                                 const int32_t* count, int64_t cap, int64_t N, int64_t C, float dsigma,
                                 tps_stream stream) {
+  TPS_TRACE("hsa_euler_update");
   using namespace tps;
   if (!x || !v_cache || !idx || !count || (cap > 0 && !v_fresh))
     return fail(TPS_ERR_INVALID_ARG, "hsa_euler_update: null pointer");

@@ -9,6 +9,7 @@
 // ranges). HBM-bound elementwise pass: one thread per 16-byte vector of o.
 #include <cmath>
 
+#include "trace.cuh"
 #include "tps_internal.cuh"
 
 namespace tps {
@@ -111,6 +112,7 @@ int merge_split_parts(const float* o_part, const float* lse_part, int nsplit, co
 extern "C" int attn_lse_merge(const tps_bf16* o1, const float* lse1, const tps_bf16* o2, const float* lse2,
                               const int32_t* count, int64_t cap, int H, int d, tps_bf16* o, float* lse,
                               tps_stream stream) {
+  TPS_TRACE("attn_lse_merge");
   using namespace tps;
   if (!o1 || !lse1 || !o2 || !lse2 || !count || !o) return fail(TPS_ERR_INVALID_ARG, "attn_lse_merge: null pointer");
   if (d != 64 && d != 128) return fail(TPS_ERR_INVALID_ARG, "attn_lse_merge: d=%d must be 64 or 128", d);

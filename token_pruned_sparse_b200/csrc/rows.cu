@@ -17,6 +17,7 @@
 // Random Numbers: As Easy as 1, 2, 3", SC'11) and the Box-Muller transform
 // (Box & Muller, Ann. Math. Stat. 1958), generated where the row is written so
 // the normals never touch memory.
+#include "trace.cuh"
 #include "tps_internal.cuh"
 #include "warp_search.cuh"
 
@@ -225,6 +226,7 @@ using namespace tps;
 
 extern "C" int tps_gather_rows(void* dst, const void* src, const int32_t* idx, const int32_t* count,
                                int64_t cap, int64_t N, int64_t row_bytes, tps_stream stream) {
+  TPS_TRACE("tps_gather_rows");
   if (!dst || !src || !idx || !count) return fail(TPS_ERR_INVALID_ARG, "tps_gather_rows: null pointer");
   if (cap < 0 || N < 1 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "tps_gather_rows: bad cap/N");
   if (row_bytes < 16 || row_bytes % 16 || row_bytes > (INT64_C(1) << 20))
@@ -245,6 +247,7 @@ extern "C" int tps_gather_rows(void* dst, const void* src, const int32_t* idx, c
 extern "C" int scatter_out(tps_bf16* o_full, const tps_bf16* o_act, const int32_t* idx,
                            const int32_t* count, int64_t cap, int64_t N, int H, int d,
                            tps_stream stream) {
+  TPS_TRACE("scatter_out");
   if (!o_full || !o_act || !idx || !count) return fail(TPS_ERR_INVALID_ARG, "scatter_out: null pointer");
   if (int e = check_rows("scatter_out", cap, N, H, d)) return e;
   if (!aligned16(o_full) || !aligned16(o_act)) return fail(TPS_ERR_ALIGN, "scatter_out: rows must be 16-byte aligned");
@@ -264,6 +267,7 @@ extern "C" int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_f
                        const tps_bf16* v_fresh, const int32_t* idx, const int32_t* count, int64_t cap,
                        int64_t N, int H, int d, const tps_renoise* rn, tps_bf16* k_eff,
                        tps_bf16* v_eff, tps_stream stream) {
+  TPS_TRACE("kv_sync");
   if (!k_cache || !v_cache || !k_fresh || !v_fresh || !idx || !count)
     return fail(TPS_ERR_INVALID_ARG, "kv_sync: null pointer");
   if (int e = check_rows("kv_sync", cap, N, H, d)) return e;
@@ -296,6 +300,7 @@ extern "C" int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_f
 
 extern "C" int tps_philox_fill(uint32_t* out, uint64_t q0, int64_t nq, uint64_t seed, uint32_t step,
                                uint32_t tensor, tps_stream stream) {
+  TPS_TRACE("tps_philox_fill");
   if (!out) return fail(TPS_ERR_INVALID_ARG, "tps_philox_fill: out is null");
   if (nq < 0) return fail(TPS_ERR_SHAPE, "tps_philox_fill: nq < 0");
   if (!aligned16(out)) return fail(TPS_ERR_ALIGN, "tps_philox_fill: out must be 16-byte aligned");

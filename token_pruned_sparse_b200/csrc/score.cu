@@ -14,6 +14,7 @@
 // read is served by the 126 MB L2 and DRAM sees each latent once.
 #include <cmath>
 
+#include "trace.cuh"
 #include "tps_internal.cuh"
 
 namespace tps {
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(256) score_motion_kernel(const uint16_t* __res
 
 extern "C" int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int64_t C, int L, float* score,
                                   tps_stream stream) {
+  TPS_TRACE("lipar_score_motion");
   using namespace tps;
   if (!x || !score) return fail(TPS_ERR_INVALID_ARG, "lipar_score_motion: x and score must be non-null");
   if (F < 1 || HW < 1 || F > (INT64_C(1) << 31) / HW) return fail(TPS_ERR_SHAPE, "lipar_score_motion: bad F/HW");
@@ -200,6 +202,7 @@ extern "C" int lipar_score_motion(const tps_bf16* x, int64_t F, int64_t HW, int6
 
 extern "C" int lipar_score(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame,
                            int64_t F, int64_t HW, int64_t C, float* score, tps_stream stream) {
+  TPS_TRACE("lipar_score");
   using namespace tps;
   if (!x || !score) return fail(TPS_ERR_INVALID_ARG, "lipar_score: x and score must be non-null");
   if (F < 1 || HW < 1) return fail(TPS_ERR_SHAPE, "lipar_score: F=%lld HW=%lld must be >= 1",

@@ -22,6 +22,7 @@
 //     order, so the result is unique.
 #include <mutex>
 
+#include "trace.cuh"
 #include "tps_internal.cuh"
 
 namespace tps {
@@ -665,6 +666,7 @@ extern "C" size_t tps_workspace_min_size(int op, int64_t N, int K) {
 extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, int64_t k,
                             int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                             tps_stream stream) {
+  TPS_TRACE("lipar_select");
   using namespace tps;
   if (mode != TPS_SELECT_THRESHOLD && mode != TPS_SELECT_TOPK)
     return fail(TPS_ERR_INVALID_ARG, "lipar_select: mode %d is not 0 (threshold) or 1 (top-k)", mode);
@@ -700,6 +702,7 @@ extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, 
 
 extern "C" int lipar_group(const float* score, int64_t N, int K, int8_t* group, void* ws,
                            size_t ws_bytes, tps_stream stream) {
+  TPS_TRACE("lipar_group");
   using namespace tps;
   if (!score || !group) return fail(TPS_ERR_INVALID_ARG, "lipar_group: score and group must be non-null");
   if (N < 1 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "lipar_group: N=%lld out of [1, 2^31)", (long long)N);
@@ -727,6 +730,7 @@ extern "C" int lipar_group(const float* score, int64_t N, int K, int8_t* group, 
 extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32_t* budgets, int T,
                               int step, int m, int32_t* idx, int32_t* count, void* ws,
                               size_t ws_bytes, tps_stream stream) {
+  TPS_TRACE("lipar_schedule");
   using namespace tps;
   if (!count || !budgets) return fail(TPS_ERR_INVALID_ARG, "lipar_schedule: count and budgets must be non-null");
   if (N < 0 || N >= (INT64_C(1) << 31)) return fail(TPS_ERR_SHAPE, "lipar_schedule: N=%lld out of [0, 2^31)", (long long)N);
@@ -798,6 +802,7 @@ int static_scratch(void** out) {
 
 extern "C" int lipar_select_static(const float* score, int64_t N, int mode, float tau, int64_t k,
                                    int32_t* idx, int32_t* count, tps_stream stream) {
+  TPS_TRACE("lipar_select_static");
   using namespace tps;
   if (N > kStaticMaxN)
     return fail(TPS_ERR_SHAPE, "lipar_select_static: N=%lld exceeds the static scratch limit of %lld tokens "

@@ -19,6 +19,7 @@
 // Threads: d = 128 runs two channel halves of 64 in separate warp groups (so
 // every branch on the channel windows is warp-uniform); the halves' partial sums
 // meet in shared memory. d = 64 runs one half.
+#include "trace.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.cuh"
 
@@ -347,6 +348,7 @@ int launch(const tps_bf16* x, int64_t F, int64_t Hs, int64_t Ws, int H, TrParams
 extern "C" int timeripple_score(const tps_bf16* x, int64_t F, int64_t Hs, int64_t Ws, int H, int d,
                                 const int32_t* windows, const float* theta, uint8_t* reuse, float* delta,
                                 float* score, tps_stream stream) {
+  TPS_TRACE("timeripple_score");
   using namespace tps;
   if (!x || !windows || !theta || !reuse) return fail(TPS_ERR_INVALID_ARG, "timeripple_score: null pointer");
   if (d != 64 && d != 128) return fail(TPS_ERR_INVALID_ARG, "timeripple_score: d=%d must be 64 or 128", d);

@@ -51,6 +51,7 @@ SIGNATURES = {
     "tps_check": (_INT, [_P]),
     "tps_philox_fill": (_INT, [_P, C.c_uint64, _I64, C.c_uint64, C.c_uint32, C.c_uint32, _P]),
     "tps_wait_probe": (_INT, [_I64, _P]),
+    "tps_debug_inject_launch_failures": (None, [_INT]),
     "tps_version": (C.c_char_p, []),
 }
 
@@ -318,6 +319,10 @@ def tps_philox_fill(q0, nq, seed, step, tensor, out=None, stream=None):
 
 def tps_wait_probe(limit_cycles, stream=None):
     _chk(lib().tps_wait_probe(int(limit_cycles), _stream(stream)))
+
+
+def debug_inject_launch_failures(n: int):
+    lib().tps_debug_inject_launch_failures(int(n))
 
 
 def version() -> str:
