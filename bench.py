@@ -402,6 +402,109 @@ def oracle_baseline():
 
 
 # ------------------------------------------------------- per-config sweep ------
+def oracle_config_baselines(rows: int = 128):
+    """The fp64 oracle on every config, each a bounded sample, reported beside the
+    GPU numbers (a baseline, not a target). Per config and step size: the O(N)
+    stages (score, select or HSA groups/schedule, gather, kv_sync -- re-noise on
+    one head at the HSA size -- and scatter) run over all tokens; attention runs
+    for `rows` sampled active rows of one head, and the layer step is
+    extrapolated as O(N) stages + per-(row, head) attention cost x |A| x H."""
+    import oracle as O
+    out = {}
+    rng = np.random.default_rng(11)
+
+    def tm(fn):
+        t0 = time.perf_counter()
+        r = fn()
+        return time.perf_counter() - t0, r
+
+    def attn_cost(q, k, v, idx, scale, bm=None):
+        """(per-head fixed cost, per-(row, head) cost) from samples of rows/2 and 2*rows rows"""
+        ts = []
+        for n in (rows // 2, 2 * rows):
+            r = rng.choice(len(idx), min(n, len(idx)), replace=False)
+            t, _ = tm(lambda: O.pruned_attn(q, k, v, idx, scale, blockmask=bm, rows=r, heads=[0]))
+            ts.append((len(r), t))
+        (n1, t1), (n2, t2) = ts
+        b = max((t2 - t1) / max(n2 - n1, 1), 1e-9)
+        return max(t1 - b * n1, 0.0), b
+
+    def report(name, t_lin, cost, A, H, N, d, flops, sampled):
+        step = t_lin + H * (cost[0] + cost[1] * A)
+        out[name] = {"seconds_per_step": round(step, 4), "tflops_alg": round(flops / step / 1e12, 6),
+                     "active_tokens_per_s": round(A / step, 1), "measured_linear_seconds": round(sampled, 3),
+                     "active": int(A), "tokens": int(N)}
+
+    def qkv(tok, cfg):
+        W = synth.projection_weights(cfg.video.C, cfg.H, cfg.d, cfg.video.seed)
+        return [synth.project(tok, w, cfg.H, cfg.d) for w in W]
+
+    # tiny: the complete step, all rows and heads
+    cfg = synth.CONFIGS["tiny"]
+    x, _ = synth.latent_video(cfg.video)
+    xb = synth.to_bf16(x)
+    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
+    t_all, _ = tm(lambda: O.pruned_attn(q, kf, vf, O.select_threshold(O.lipar_score(xb), cfg.tau),
+                                        1 / math.sqrt(cfg.d)))
+    A = len(O.select_threshold(O.lipar_score(xb), cfg.tau))
+    report("tiny", t_all, (0.0, 0.0), A, cfg.H, cfg.video.N, cfg.d, O.attn_flops(A, cfg.video.N, cfg.H, cfg.d),
+           t_all)
+
+    # Wan, inter-step score, keep 10/30/50/100%
+    cfg = synth.CONFIGS["wan"]
+    vp, delta = synth.velocity_pair(cfg.video)
+    vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    q, kf, vf = qkv(vcb, cfg)
+    t_score, s = tm(lambda: O.lipar_score(vcb[None], vpb[None]))
+    for ratio in cfg.keep:
+        k = synth.keep_count(N, ratio)
+        t_sel, idx = tm(lambda: O.select_topk(s, k))
+        t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.kv_sync(kf, vf, kf[idx], vf[idx], idx),
+                                O.scatter_out(q, q[idx], idx)))
+        per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d))
+        report(f"wan_keep{int(ratio * 100)}", t_score + t_sel + t_rows, per, k, H, N, d,
+               O.attn_flops(k, N, H, d), t_score + t_sel + t_rows)
+
+    # HSA: groups + schedule, re-noise, attention at |A| = N/3 (odd steps)
+    cfg = synth.CONFIGS["hsa"]
+    vp, delta = synth.velocity_pair(cfg.video)
+    vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    K, T, budgets = cfg.extra["K"], cfg.extra["T"], cfg.extra["budgets"]
+    q, kf, vf = qkv(vcb, cfg)
+    t_score, s = tm(lambda: O.lipar_score(vcb[None], vpb[None]))
+    t_grp, g = tm(lambda: O.group_split(s, K))
+    t_sch, idx = tm(lambda: O.schedule_active(g, K, budgets, T, 1, 0))
+    t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.scatter_out(q, q[idx], idx)))
+    t_rn, _ = tm(lambda: O.kv_sync(kf, vf, kf[idx], vf[idx], idx, renoise=(0.025, 0.975, 4, 1), heads=[0]))
+    per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d))
+    A = len(idx)
+    t_lin = t_score + t_grp + t_sch + t_rows + t_rn * H
+    report("hsa_step_A_N/3", t_lin, per, A, H, N, d, O.attn_flops(A, N, H, d),
+           t_score + t_grp + t_sch + t_rows + t_rn)
+
+    # block-sparse: inter-frame top-k 40%, 139 of 929 key blocks per query block
+    cfg = synth.CONFIGS["block"]
+    x, _ = synth.latent_video(cfg.video)
+    xb = synth.to_bf16(x)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
+    t_score, s = tm(lambda: O.lipar_score(xb))
+    kk = synth.keep_count(N, cfg.keep[0])
+    t_sel, idx = tm(lambda: O.select_topk(s, kk))
+    bm = synth.block_mask_band_random(cfg.video, 128, cfg.extra["kept_per_row"], cfg.video.seed)
+    per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d), bm=bm)
+    keys = bm.numpy()[np.asarray(idx) // 128].sum(axis=1) * 128.0
+    report("block_sparse", t_score + t_sel, per, kk, H, N, d, O.attn_flops(kk, N, H, d, keys),
+           t_score + t_sel)
+    for v in out.values():
+        v["sample"] = (f"O(N) stages over all tokens (HSA re-noise on one head, x H); attention timed for "
+                       f"{rows // 2} and {2 * rows} sampled active rows of one head, split into a per-head and "
+                       f"a per-row cost, and extrapolated to all rows and heads")
+    return out
+
+
 def _time(fn, flush, reps=5, warm=2):
     ms = []
     for i in range(warm + reps):
@@ -678,9 +781,10 @@ def main():
                 "flops_per_launch": st.flops, "avg_launch_ms": round(attn_avg, 4)}
 
     configs = None if (a.no_configs or world > 1) else config_sweep(dev, peak, float(pk["hbm_gbs"]))
-    cpu = None
+    cpu = cpu_configs = None
     if rank == 0 and world == 1 and not a.no_cpu:
         cpu = oracle_baseline()
+        cpu_configs = oracle_config_baselines()
 
     if world > 1:
         dist.barrier()
@@ -703,7 +807,7 @@ def main():
         "active_tokens_per_s": round(tok_s, 1),
         "gpu_launches": st.launches * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
-        "keep_sweep_wan": sweep, "configs": configs,
+        "keep_sweep_wan": sweep, "configs": configs, "cpu_baseline_configs": cpu_configs,
     }
     print(json.dumps(line), flush=True)
     return 0
