@@ -27,19 +27,23 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;
+// Row moves run as 128-thread blocks, up to 16 per SM: at the HSA size this moves
+// rows at 6.42 TB/s against 6.09-6.25 TB/s with 256-thread blocks and 8 per SM.
+constexpr int kMoveThreads = 128;
+constexpr int kMoveWarps = kMoveThreads / 32;
 
 // ---- row move: dst[dst_row] = src[src_row] for one or two tensors -----------------
 // kScatter: dst row = idx[j], src row = j.  !kScatter: dst row = j, src row = idx[j].
 template <bool kScatter>
-__global__ void __launch_bounds__(kThreads) rows_move(uint4* __restrict__ d0, const uint4* __restrict__ s0,
+__global__ void __launch_bounds__(kMoveThreads) rows_move(uint4* __restrict__ d0, const uint4* __restrict__ s0,
                                                       uint4* __restrict__ d1, const uint4* __restrict__ s1,
                                                       const int32_t* __restrict__ idx,
                                                       const int32_t* __restrict__ count, int64_t cap,
                                                       int64_t N, int vpr, unsigned int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t rows = active_count(count, cap);
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kMoveThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kMoveWarps;
   for (int64_t j = warp; j < rows; j += nwarps) {
     const int64_t n = idx[j];
     if (n < 0 || n >= N) {
@@ -202,6 +206,14 @@ __global__ void philox_fill(uint4* out, uint64_t q0, int64_t nq, uint32_t k0, ui
   }
 }
 
+unsigned int move_grid(int64_t rows) {
+  int64_t g = (rows + kMoveWarps - 1) / kMoveWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<unsigned int>(g);
+}
+
 unsigned int row_grid(int64_t rows) {
   int64_t g = (rows + kWarps - 1) / kWarps;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -237,7 +249,7 @@ extern "C" int tps_gather_rows(void* dst, const void* src, const int32_t* idx, c
   if (!st) return err;
   if (cap == 0) return ok();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rows_move<false><<<row_grid(cap), kThreads, 0, s>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src),
+  rows_move<false><<<move_grid(cap), kMoveThreads, 0, s>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src),
                                                       nullptr, nullptr, idx, count, cap, N,
                                                       static_cast<int>(row_bytes / 16), st);
   if (int e = launch_status("tps_gather_rows")) return e;
@@ -256,7 +268,7 @@ extern "C" int scatter_out(tps_bf16* o_full, const tps_bf16* o_act, const int32_
   if (!st) return err;
   if (cap == 0) return ok();
   const int vpr = H * d / 8;
-  rows_move<true><<<row_grid(cap), kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+  rows_move<true><<<move_grid(cap), kMoveThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<uint4*>(o_full), reinterpret_cast<const uint4*>(o_act), nullptr, nullptr, idx,
       count, cap, N, vpr, st);
   if (int e = launch_status("scatter_out")) return e;
@@ -282,7 +294,7 @@ extern "C" int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!rn) {
     if (cap == 0) return ok();
-    rows_move<true><<<row_grid(cap), kThreads, 0, s>>>(
+    rows_move<true><<<move_grid(cap), kMoveThreads, 0, s>>>(
         reinterpret_cast<uint4*>(k_cache), reinterpret_cast<const uint4*>(k_fresh),
         reinterpret_cast<uint4*>(v_cache), reinterpret_cast<const uint4*>(v_fresh), idx, count, cap, N,
         vpr, st);
