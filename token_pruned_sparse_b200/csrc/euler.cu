@@ -20,7 +20,7 @@
 namespace tps {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRun = 8;
 
@@ -108,7 +108,7 @@ extern "C" int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_f
   if (!st) return err;
   const int64_t runs = ((N + kRun - 1) / kRun + 4 - 1) / 4;   // groups of runs
   int64_t grid = (runs + kWarps - 1) / kWarps;
-  const int64_t maxg = static_cast<int64_t>(sm_count()) * 8;
+  const int64_t maxg = static_cast<int64_t>(sm_count()) * 16;
   if (grid > maxg) grid = maxg;
   const dim3 g(static_cast<unsigned int>(grid));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -27,8 +27,9 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;
-// Row moves run as 128-thread blocks, up to 16 per SM: at the HSA size this moves
-// rows at 6.42 TB/s against 6.09-6.25 TB/s with 256-thread blocks and 8 per SM.
+// Row moves and the re-noise pass run as 128-thread blocks, up to 16 per SM: at
+// the HSA size rows move at 6.42 TB/s against 6.09-6.25 TB/s with 256-thread
+// blocks and 8 per SM, and re-noise gains 2%.
 constexpr int kMoveThreads = 128;
 constexpr int kMoveWarps = kMoveThreads / 32;
 
@@ -146,15 +147,15 @@ __device__ __forceinline__ uint4 renoise_vec(uint4 c, float a, float b, const fl
 // active index >= the run start, then the (ascending) list is walked in step.
 constexpr int kRun = 8;
 
-__global__ void __launch_bounds__(kThreads) kv_sync_renoise(
+__global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
     uint4* __restrict__ kc, uint4* __restrict__ vc, const uint4* __restrict__ kf,
     const uint4* __restrict__ vf, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
     int64_t cap, int64_t N, int vpr, float a, float b, uint32_t k0, uint32_t k1, uint32_t step,
     uint4* __restrict__ ke, uint4* __restrict__ ve, unsigned int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t cnt = active_count(count, cap);
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kMoveThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kMoveWarps;
   const int64_t nruns = (N + kRun - 1) / kRun;
   const uint64_t epr = static_cast<uint64_t>(vpr) * 8;  // elements per row
   for (int64_t run = warp; run < nruns; run += nwarps) {
@@ -300,7 +301,7 @@ extern "C" int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_f
         vpr, st);
   } else {
     const int64_t runs = (N + kRun - 1) / kRun;
-    kv_sync_renoise<<<row_grid(runs), kThreads, 0, s>>>(
+    kv_sync_renoise<<<move_grid(runs), kMoveThreads, 0, s>>>(
         reinterpret_cast<uint4*>(k_cache), reinterpret_cast<uint4*>(v_cache),
         reinterpret_cast<const uint4*>(k_fresh), reinterpret_cast<const uint4*>(v_fresh), idx, count, cap,
         N, vpr, rn->a, rn->b, static_cast<uint32_t>(rn->seed), static_cast<uint32_t>(rn->seed >> 32),
