@@ -24,8 +24,6 @@
 namespace tps {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;
 // Row moves and the re-noise pass run as 128-thread blocks, up to 16 per SM: at
 // the HSA size rows move at 6.42 TB/s against 6.09-6.25 TB/s with 256-thread
@@ -210,14 +208,6 @@ __global__ void philox_fill(uint4* out, uint64_t q0, int64_t nq, uint32_t k0, ui
 unsigned int move_grid(int64_t rows) {
   int64_t g = (rows + kMoveWarps - 1) / kMoveWarps;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
-  if (g > cap) g = cap;
-  if (g < 1) g = 1;
-  return static_cast<unsigned int>(g);
-}
-
-unsigned int row_grid(int64_t rows) {
-  int64_t g = (rows + kWarps - 1) / kWarps;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<unsigned int>(g);
