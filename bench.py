@@ -55,7 +55,7 @@ def peaks():
 
 def attn_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("attn_tc.cu", "attn_common.cuh", "tc_ptx.cuh", "tps_internal.cuh"):
+    for name in ("attn_tc.cu", "attn_common.cuh", "tc_ptx.cuh", "tps_internal.cuh", "tma_host.cuh", "trace.cuh"):
         p = os.path.join(ROOT, "token_pruned_sparse_b200", "csrc", name)
         if os.path.exists(p):
             with open(p, "rb") as f:

@@ -33,11 +33,10 @@
 // Every mbarrier wait is bounded: on expiry the CTA sets an abort flag and the
 // device status word (TPS_ERR_TIMEOUT via tps_check), drains what it issued,
 // frees TMEM and returns.
-#include <mutex>
-
 #include "trace.cuh"
 #include "attn_common.cuh"
 #include "tc_ptx.cuh"
+#include "tma_host.cuh"
 
 namespace tps {
 namespace {
@@ -458,29 +457,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 }
 
 // ---- host ------------------------------------------------------------------------------------
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-int get_encoder(EncodeTiled* fn) {
-  static EncodeTiled cached = nullptr;
-  static std::once_flag once;
-  static int err = TPS_OK;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f)
-      err = fail(TPS_ERR_CUDA, "pruned_attn: cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(e));
-    else
-      cached = reinterpret_cast<EncodeTiled>(f);
-  });
-  *fn = cached;
-  return cached ? TPS_OK : (err ? err : fail(TPS_ERR_CUDA, "pruned_attn: no tensor-map encoder"));
-}
-
 // [rows, H, d] bf16, token-major -> 3-D map (d, H, rows), box (64, 1, 128), 128-byte swizzle.
-int make_map(EncodeTiled enc, CUtensorMap* m, const void* base, int64_t rows, int H, int d) {
+int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, int H, int d) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
   cuuint32_t box[3] = {64, 1, 128};
@@ -495,8 +473,8 @@ int make_map(EncodeTiled enc, CUtensorMap* m, const void* base, int64_t rows, in
 template <int D>
 int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr) {
   if (a.cap == 0) return TPS_OK;
-  EncodeTiled enc;
-  if (int e = get_encoder(&enc)) return e;
+  EncodeTiledFn enc;
+  if (int e = tensor_map_encoder(&enc, "pruned_attn")) return e;
   int err;
   unsigned int* status = device_status(&err);
   if (!status) return err;
