@@ -13,9 +13,9 @@ Parity status per function (see each docstring for the pins):
   euler_update, lse_merge, lipar_score_motion,
   timeripple_delta/_reuse/_token_score/_theta -- pinned likewise (hand-worked
                                          fixtures, closed forms, invariants)
-  philox4x32_10 raw stream            -- parity unpinned (no published
-                                         known-answer vector available offline);
-                                         its normals are pinned statistically.
+  philox4x32_10 raw stream            -- pinned by the published
+                                         known-answer vectors (Salmon et al.,
+                                         SC'11), and its normals statistically.
 """
 from .tps_oracle import *  # noqa: F401,F403
 from .tps_oracle import __all__  # noqa: F401

@@ -176,8 +176,8 @@ def philox4x32_10(c0, c1, c2, c3, k0: int, k1: int):
 
     One round: (hi0, lo0) = M0 * c0, (hi1, lo1) = M1 * c2 (64-bit products);
     new counter = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0). The key is bumped
-    by the Weyl constants between rounds. Parity unpinned: no published
-    known-answer vector is available offline."""
+    by the Weyl constants between rounds. Pinned by the published
+    known-answer vectors (tests/golden/philox_kat.json)."""
     c = [np.asarray(v, np.uint64) & _MASK32 for v in (c0, c1, c2, c3)]
     k = [np.uint64(k0) & _MASK32, np.uint64(k1) & _MASK32]
     m0, m1 = np.uint64(_PHILOX_M[0]), np.uint64(_PHILOX_M[1])

@@ -186,3 +186,18 @@ def test_gather_and_scatter_through_pinned_host_memory():
     tps.scatter_out(out, act.to(DEV), di, dc, cap=A)
     tps.tps_check()
     assert torch.equal(out, O.scatter_out(before, act, idx))
+
+
+def test_philox_known_answer_vectors_on_gpu():
+    """The kernels' Philox4x32-10 against the published known-answer vectors:
+    counter = (q mod 2^32, q div 2^32, step, tensor), key = (seed mod 2^32, seed div 2^32)."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "philox_kat.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        c = [int(v, 16) for v in case["counter"]]
+        k = [int(v, 16) for v in case["key"]]
+        words = tps.tps_philox_fill(c[0] | (c[1] << 32), 1, k[0] | (k[1] << 32), c[2], c[3])
+        got = words.cpu().numpy().view(np.uint32).tolist()
+        assert got == [int(v, 16) for v in case["out"]]

@@ -188,8 +188,8 @@ def test_renoise_statistics():
 
 
 def test_philox_words_uniform_and_distinct():
-    """Raw stream: parity unpinned (no known-answer vectors offline); only
-    uniformity of the bytes and distinctness across counters are checked."""
+    """Raw stream properties beyond the known-answer vectors: uniform bytes
+    and distinct streams across counters, steps, tensors and seeds."""
     from scipy import stats
     w = O.philox_words(42, 0, 0, np.arange(1 << 14))
     assert len(np.unique(w.reshape(-1))) > 0.999 * w.size
@@ -469,3 +469,14 @@ def test_timeripple_pins_catch_planted_mistakes():
     # '<=' instead of '<' would mark token 1 reusable on x (Delta_x = theta_x = 1)
     D = O.timeripple_delta(x, F, Hs, Ws, g["windows"])
     assert (D[1][1, 0] <= g["theta"][1]) and O.timeripple_reuse(D, g["theta"])[1, 0] == 0
+
+
+def test_philox_known_answer_vectors():
+    """The oracle's Philox4x32-10 against the published known-answer vectors."""
+    g = _gold("philox_kat.json")
+    for case in g["cases"]:
+        c = [np.array([int(v, 16)], dtype=np.uint64) for v in case["counter"]]
+        k = [int(v, 16) for v in case["key"]]
+        out = O.philox4x32_10(*c, k[0], k[1])
+        got = [int(np.asarray(o).reshape(-1)[0]) for o in out]
+        assert got == [int(v, 16) for v in case["out"]]
