@@ -18,7 +18,11 @@
 //
 // Threads: d = 128 runs two channel halves of 64 in separate warp groups (so
 // every branch on the channel windows is warp-uniform); the halves' partial sums
-// meet in shared memory. d = 64 runs one half.
+// meet in shared memory. d = 64 runs one half. When the windows are the
+// rotary-group windows (the default split of d into t, x, y groups), each
+// chunk's channel masks are compile-time constants: chunks outside a window
+// emit no code and full chunks take the unmasked path. Other windows read their
+// masks at run time.
 #include "trace.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.cuh"
@@ -52,6 +56,7 @@ struct TrParams {
   int start[3], len[3];
   float inv_len[3];
   float theta[3];
+  int fixed_windows;        // 1: the windows are the rotary-group windows of d (compile-time masks)
   int64_t N;
   uint8_t* reuse;
   float* delta;
@@ -123,6 +128,79 @@ __device__ __forceinline__ uint64_t window_mask(int s, int len, int d, int half)
   uint64_t m = bit_range(s - b, (s + len < d ? s + len : d) - b);
   if (s + len > d) m |= bit_range(-b, s + len - d - b);
   return m;
+}
+
+// The configured windows (rotary groups [t | x | y] of sizes d - 4*(d/6), 2*(d/6),
+// 2*(d/6); each check uses the groups its axis does not rotate), as (start, len)
+// per axis. When a call passes exactly these, the chunk masks below are
+// compile-time constants and the per-chunk branches on them disappear.
+__host__ __device__ constexpr int fixed_window(int d, int a, int which) {
+  return a == 0 ? (which == 0 ? d - 4 * (d / 6) : 4 * (d / 6))
+       : a == 1 ? (which == 0 ? d - 2 * (d / 6) : d - 2 * (d / 6))
+                : (which == 0 ? 0 : d - 2 * (d / 6));
+}
+
+// 8-bit mask of chunk j (channels c0 .. c0+7) in the cyclic window [s, s+len) mod d.
+__host__ __device__ constexpr uint32_t chunk_bits(int s, int len, int d, int c0) {
+  uint32_t m = 0;
+  for (int e = 0; e < 8; ++e) m |= (((c0 + e - s) % d + d) % d < len ? 1u : 0u) << e;
+  return m;
+}
+
+template <int D, int HALF, int J, int A>
+__device__ __forceinline__ constexpr uint32_t fixed_bits() {
+  return chunk_bits(fixed_window(D, A, 0), fixed_window(D, A, 1), D, 64 * HALF + 8 * J);
+}
+
+// The checks of one frame for this thread's token and 64 channels: chunk j+1's
+// three rows are loaded while chunk j is checked. kFixed: compile-time windows.
+template <int D, int HALF, bool kFixed>
+__device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, uint32_t (&prev)[32], float2 (&at)[2],
+                                            float2 (&ax)[2], float2 (&ay)[2], const uint32_t (&wlo)[3],
+                                            const uint32_t (&whi)[3]) {
+  uint4 ncw = lds128(swz(box, rc, 0)), nlw = lds128(swz(box, rc - 1, 0)), nuw = lds128(swz(box, rc - kBoxCols, 0));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint4 cw = ncw, lw = nlw, uw = nuw;
+    if (j < 7) {
+      ncw = lds128(swz(box, rc, j + 1));
+      nlw = lds128(swz(box, rc - 1, j + 1));
+      nuw = lds128(swz(box, rc - kBoxCols, j + 1));
+    }
+    float2 c[4], nb[4];
+    unpack(cw, c);
+    uint32_t mt, mx, my;
+    if constexpr (kFixed) {
+      // j is a compile-time constant after unrolling
+      constexpr uint32_t f0[8] = {fixed_bits<D, HALF, 0, 0>(), fixed_bits<D, HALF, 1, 0>(), fixed_bits<D, HALF, 2, 0>(),
+                                  fixed_bits<D, HALF, 3, 0>(), fixed_bits<D, HALF, 4, 0>(), fixed_bits<D, HALF, 5, 0>(),
+                                  fixed_bits<D, HALF, 6, 0>(), fixed_bits<D, HALF, 7, 0>()};
+      constexpr uint32_t f1[8] = {fixed_bits<D, HALF, 0, 1>(), fixed_bits<D, HALF, 1, 1>(), fixed_bits<D, HALF, 2, 1>(),
+                                  fixed_bits<D, HALF, 3, 1>(), fixed_bits<D, HALF, 4, 1>(), fixed_bits<D, HALF, 5, 1>(),
+                                  fixed_bits<D, HALF, 6, 1>(), fixed_bits<D, HALF, 7, 1>()};
+      constexpr uint32_t f2[8] = {fixed_bits<D, HALF, 0, 2>(), fixed_bits<D, HALF, 1, 2>(), fixed_bits<D, HALF, 2, 2>(),
+                                  fixed_bits<D, HALF, 3, 2>(), fixed_bits<D, HALF, 4, 2>(), fixed_bits<D, HALF, 5, 2>(),
+                                  fixed_bits<D, HALF, 6, 2>(), fixed_bits<D, HALF, 7, 2>()};
+      mt = f0[j], mx = f1[j], my = f2[j];
+    } else {
+      mt = j < 4 ? (wlo[0] >> (8 * j)) & 0xffu : (whi[0] >> (8 * (j - 4))) & 0xffu;
+      mx = j < 4 ? (wlo[1] >> (8 * j)) & 0xffu : (whi[1] >> (8 * (j - 4))) & 0xffu;
+      my = j < 4 ? (wlo[2] >> (8 * j)) & 0xffu : (whi[2] >> (8 * (j - 4))) & 0xffu;
+    }
+    if (has_t && mt) {
+      unpack(make_uint4(prev[4 * j], prev[4 * j + 1], prev[4 * j + 2], prev[4 * j + 3]), nb);
+      sq_acc(at, c, nb, mt);
+    }
+    if (mx) {
+      unpack(lw, nb);
+      sq_acc(ax, c, nb, mx);
+    }
+    if (my) {
+      unpack(uw, nb);
+      sq_acc(ay, c, nb, my);
+    }
+    prev[4 * j] = cw.x, prev[4 * j + 1] = cw.y, prev[4 * j + 2] = cw.z, prev[4 * j + 3] = cw.w;
+  }
 }
 
 template <int D>
@@ -204,34 +282,11 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 2) tr_kernel(const __grid_co
       }
     } else {
       const bool has_t = f > 0;
-      // chunk j+1's three rows are loaded while chunk j is checked
-      uint4 ncw = lds128(swz(box, rc, 0)), nlw = lds128(swz(box, rc - 1, 0)), nuw = lds128(swz(box, rc - kBoxCols, 0));
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 cw = ncw, lw = nlw, uw = nuw;
-        if (j < 7) {
-          ncw = lds128(swz(box, rc, j + 1));
-          nlw = lds128(swz(box, rc - 1, j + 1));
-          nuw = lds128(swz(box, rc - kBoxCols, j + 1));
-        }
-        float2 c[4], nb[4];
-        unpack(cw, c);
-        const uint32_t mt = j < 4 ? (wlo[0] >> (8 * j)) & 0xffu : (whi[0] >> (8 * (j - 4))) & 0xffu;
-        const uint32_t mx = j < 4 ? (wlo[1] >> (8 * j)) & 0xffu : (whi[1] >> (8 * (j - 4))) & 0xffu;
-        const uint32_t my = j < 4 ? (wlo[2] >> (8 * j)) & 0xffu : (whi[2] >> (8 * (j - 4))) & 0xffu;
-        if (has_t && mt) {
-          unpack(make_uint4(prev[4 * j], prev[4 * j + 1], prev[4 * j + 2], prev[4 * j + 3]), nb);
-          sq_acc(at, c, nb, mt);
-        }
-        if (mx) {
-          unpack(lw, nb);
-          sq_acc(ax, c, nb, mx);
-        }
-        if (my) {
-          unpack(uw, nb);
-          sq_acc(ay, c, nb, my);
-        }
-        prev[4 * j] = cw.x, prev[4 * j + 1] = cw.y, prev[4 * j + 2] = cw.z, prev[4 * j + 3] = cw.w;
+      if (p.fixed_windows) {
+        if (half == 0) check_frame<D, 0, true>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
+        else check_frame<D, (L::kHalves > 1 ? 1 : 0), true>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
+      } else {
+        check_frame<D, 0, false>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
       }
     }
     float s[3] = {(at[0].x + at[1].x) + (at[0].y + at[1].y), (ax[0].x + ax[1].x) + (ax[0].y + ax[1].y),
@@ -371,6 +426,9 @@ extern "C" int timeripple_score(const tps_bf16* x, int64_t F, int64_t Hs, int64_
   int err;
   unsigned int* st = device_status(&err);
   if (!st) return err;
+  p.fixed_windows = 1;
+  for (int a = 0; a < 3; ++a)
+    if (p.start[a] != fixed_window(d, a, 0) || p.len[a] != fixed_window(d, a, 1)) p.fixed_windows = 0;
   p.F = static_cast<int>(F), p.Hs = static_cast<int>(Hs), p.Ws = static_cast<int>(Ws), p.H = H;
   p.N = N, p.reuse = reuse, p.delta = delta, p.status = st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
