@@ -61,12 +61,13 @@ def test_attn_random_dense(impl, N, A, H, d, sharp):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
-@pytest.mark.parametrize("growth", ["rising", "falling", "spike"])
+@pytest.mark.parametrize("growth", ["rising", "falling", "spike", "spike_lo", "spike_hi"])
 def test_attn_running_max_moves(impl, growth):
     """Score scales that change along the keys: rising makes later key tiles
     dominate (tile sums far above 2^40 against the first tile's maximum, so the
     kernel must take the slow path, find the new maximum and rescale O);
-    falling keeps the first tile's maximum; spike puts one huge tile mid-way."""
+    falling keeps the first tile's maximum; spike puts one huge tile mid-way;
+    spike_lo / spike_hi put it on keys 0-63 / 64-127 of that tile only."""
     N, A, H, d = 1500, 200, 2, 128
     q = synth.gaussian_bf16((A, H, d), 11)
     k = synth.gaussian_bf16((N, H, d), 12).double()
@@ -77,7 +78,8 @@ def test_attn_running_max_moves(impl, growth):
         g = 25.0 - 24.0 * pos
     else:
         g = torch.ones_like(pos)
-        g[640:768] = 30.0
+        lo, hi = {"spike": (640, 768), "spike_lo": (640, 704), "spike_hi": (704, 768)}[growth]
+        g[lo:hi] = 30.0
     k = (k * g).to(torch.bfloat16)
     v = synth.gaussian_bf16((N, H, d), 13)
     idx = np.sort(np.random.default_rng(5).choice(N, A, replace=False))
