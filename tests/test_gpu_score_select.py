@@ -70,7 +70,7 @@ def test_score_prev_frame_zero_change_and_edges():
 
 
 # --------------------------------------------------------------- select -----
-@pytest.mark.parametrize("N", [1, 7, 1023, 1024, 1025, 5000, 20280, 118800, 300001])
+@pytest.mark.parametrize("N", [1, 7, 1023, 1024, 1025, 5000, 20280, 32768, 32769, 118800, 300001])
 @pytest.mark.parametrize("ties", [False, True])
 def test_select_threshold_and_topk(N, ties):
     s = synth.random_scores(N, N + int(ties), ties=ties, specials=True)
