@@ -200,6 +200,8 @@ TPS_API int tps_gather_rows(void* dst, const void* src, const int32_t* idx, cons
  *   tensor: 0 = K, 1 = V), key (seed mod 2^32, seed div 2^32), q = e div 4 for
  *   flat element e = (n*H + h)*d + c, word e mod 4 mapped to
  *   u = (floor(w/2^9) + 1/2) * 2^-23, Box-Muller over words (0,1) and (2,3).
+ *   eps is computed in fp32 with the hardware log2, sine and cosine: it is
+ *   within about 1e-5 of the exact Box-Muller value, before the bf16 rounding.
  *   The cache is not overwritten by noised rows. idx must be ascending.
  * d in {64, 128}; H*d <= 16384; N < 2^31. */
 typedef struct tps_renoise {

@@ -77,14 +77,32 @@ __global__ void __launch_bounds__(kMoveThreads) rows_move(uint4* __restrict__ d0
 constexpr uint32_t kM0 = 0xD2511F53u, kM1 = 0xCD9E8D57u;  // round multipliers
 constexpr uint32_t kW0 = 0x9E3779B9u, kW1 = 0xBB67AE85u;  // Weyl key increments
 
-__device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
+// The key of round r is (k0 + r*W0, k1 + r*W1) mod 2^32. The schedule is computed
+// once on the host and passed as a __grid_constant__ kernel parameter, so each
+// round reads its key straight from the constant bank as an operand of the XOR.
+struct PhiloxKeys {
+  uint32_t k0[10];
+  uint32_t k1[10];
+};
+
+inline PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys K;
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = k0;
+    K.k1[r] = k1;
+    k0 += kW0;
+    k1 += kW1;
+  }
+  return K;
+}
+
+__device__ __forceinline__ uint4 philox10(uint4 c, const PhiloxKeys& K) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
     const uint32_t hi0 = __umulhi(kM0, c.x), lo0 = kM0 * c.x;
     const uint32_t hi1 = __umulhi(kM1, c.z), lo1 = kM1 * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-    k0 += kW0;
-    k1 += kW1;
+    c = make_uint4(hi1 ^ c.y ^ K.k0[r], lo1, hi0 ^ c.w ^ K.k1[r], lo0);
   }
   return c;
 }
@@ -105,10 +123,22 @@ __device__ __forceinline__ float sqrt_approx(float x) {
 // Box-Muller on one word pair: z0 = r cos(2 pi ub), z1 = r sin(2 pi ub),
 // r = sqrt(-2 ln ua). The angle is taken as 2 pi (ub - 1/2) in (-pi, pi), where
 // the hardware sine/cosine are accurate, and the signs folded back.
+// -2 ln u for u in (0, 1): the hardware base-2 logarithm times -2 ln 2, except
+// for u > 0.995 (t = 1 - u < 0.005, exact in fp32), where the Taylor series of
+// -2 ln(1 - t) = 2t (1 + t/2 + t^2/3 + ...) to the t^2 term is accurate to t^3/4.
+__device__ __forceinline__ float neg2ln(float u) {
+  float l2;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l2) : "f"(u));
+  const float t = 1.0f - u;
+  const float ser = 2.0f * t * fmaf(t, fmaf(t, 0.333333343f, 0.5f), 1.0f);
+  return t < 0.005f ? ser : -1.38629436111989061883f * l2;
+}
+
 __device__ __forceinline__ void box_muller(uint32_t wa, uint32_t wb, float& z0, float& z1) {
   const float ua = uniform01(wa), ub = uniform01(wb);
-  const float r = sqrt_approx(-2.0f * logf(ua));   // hardware sqrt, ~2^-23 relative
-  const float th = 6.28318530717958647692f * (ub - 0.5f);
+  const float r = sqrt_approx(neg2ln(ua));         // hardware sqrt, ~2^-23 relative
+  // 2 pi (ub - 1/2) in one rounding: 2 pi and pi are exact doubles of each other in fp32
+  const float th = fmaf(6.28318530717958647692f, ub, -3.14159265358979323846f);
   float sn, cs;
   __sincosf(th, &sn, &cs);
   z0 = -r * cs;
@@ -116,13 +146,13 @@ __device__ __forceinline__ void box_muller(uint32_t wa, uint32_t wb, float& z0, 
 }
 
 // Eight normals for the flat elements e0 .. e0+7 (e0 % 8 == 0) of tensor t.
-__device__ __forceinline__ void normals8(uint64_t e0, uint32_t step, uint32_t t, uint32_t k0,
-                                         uint32_t k1, float z[8]) {
+__device__ __forceinline__ void normals8(uint64_t e0, uint32_t step, uint32_t t, const PhiloxKeys& K,
+                                         float z[8]) {
   const uint64_t q = e0 >> 2;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint64_t qq = q + h;
-    const uint4 w = philox10(make_uint4(static_cast<uint32_t>(qq), static_cast<uint32_t>(qq >> 32), step, t), k0, k1);
+    const uint4 w = philox10(make_uint4(static_cast<uint32_t>(qq), static_cast<uint32_t>(qq >> 32), step, t), K);
     box_muller(w.x, w.y, z[4 * h + 0], z[4 * h + 1]);
     box_muller(w.z, w.w, z[4 * h + 2], z[4 * h + 3]);
   }
@@ -130,12 +160,14 @@ __device__ __forceinline__ void normals8(uint64_t e0, uint32_t step, uint32_t t,
 
 __device__ __forceinline__ uint4 renoise_vec(uint4 c, float a, float b, const float z[8]) {
   const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+  const float2 a2 = make_float2(a, a), b2 = make_float2(b, b);
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float lo = fmaf(b, z[2 * i], a * bf16lo(cw[i]));
-    const float hi = fmaf(b, z[2 * i + 1], a * bf16hi(cw[i]));
-    o[i] = pack_bf16x2(lo, hi);
+    // a*x, then b*z + (a*x): the same two roundings per element as fmaf(b, z, a * x)
+    const float2 r = __ffma2_rn(b2, make_float2(z[2 * i], z[2 * i + 1]),
+                                __fmul2_rn(a2, make_float2(bf16lo(cw[i]), bf16hi(cw[i]))));
+    o[i] = pack_bf16x2(r.x, r.y);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -148,7 +180,7 @@ constexpr int kRun = 8;
 __global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
     uint4* __restrict__ kc, uint4* __restrict__ vc, const uint4* __restrict__ kf,
     const uint4* __restrict__ vf, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
-    int64_t cap, int64_t N, int vpr, float a, float b, uint32_t k0, uint32_t k1, uint32_t step,
+    int64_t cap, int64_t N, int vpr, float a, float b, const __grid_constant__ PhiloxKeys keys, uint32_t step,
     uint4* __restrict__ ke, uint4* __restrict__ ve, unsigned int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t cnt = active_count(count, cap);
@@ -179,9 +211,9 @@ __global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
           const uint4 y = vc[row + v];
           const uint64_t e0 = static_cast<uint64_t>(n) * epr + static_cast<uint64_t>(v) * 8;
           float z[8];
-          normals8(e0, step, 0u, k0, k1, z);
+          normals8(e0, step, 0u, keys, z);
           ke[row + v] = renoise_vec(x, a, b, z);
-          normals8(e0, step, 1u, k0, k1, z);
+          normals8(e0, step, 1u, keys, z);
           ve[row + v] = renoise_vec(y, a, b, z);
         }
       }
@@ -196,12 +228,12 @@ __global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
   }
 }
 
-__global__ void philox_fill(uint4* out, uint64_t q0, int64_t nq, uint32_t k0, uint32_t k1,
+__global__ void philox_fill(uint4* out, uint64_t q0, int64_t nq, const __grid_constant__ PhiloxKeys keys,
                             uint32_t step, uint32_t t) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nq; i += stride) {
     const uint64_t q = q0 + static_cast<uint64_t>(i);
-    out[i] = philox10(make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), step, t), k0, k1);
+    out[i] = philox10(make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), step, t), keys);
   }
 }
 
@@ -294,8 +326,8 @@ extern "C" int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_f
     kv_sync_renoise<<<move_grid(runs), kMoveThreads, 0, s>>>(
         reinterpret_cast<uint4*>(k_cache), reinterpret_cast<uint4*>(v_cache),
         reinterpret_cast<const uint4*>(k_fresh), reinterpret_cast<const uint4*>(v_fresh), idx, count, cap,
-        N, vpr, rn->a, rn->b, static_cast<uint32_t>(rn->seed), static_cast<uint32_t>(rn->seed >> 32),
-        rn->step, reinterpret_cast<uint4*>(k_eff), reinterpret_cast<uint4*>(v_eff), st);
+        N, vpr, rn->a, rn->b, philox_keys(rn->seed), rn->step, reinterpret_cast<uint4*>(k_eff),
+        reinterpret_cast<uint4*>(v_eff), st);
   }
   if (int e = launch_status("kv_sync")) return e;
   return ok();
@@ -311,8 +343,7 @@ extern "C" int tps_philox_fill(uint32_t* out, uint64_t q0, int64_t nq, uint64_t 
   int64_t g = (nq + 255) / 256;
   if (g > 4096) g = 4096;
   philox_fill<<<static_cast<unsigned int>(g), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<uint4*>(out), q0, nq, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32),
-      step, tensor);
+      reinterpret_cast<uint4*>(out), q0, nq, philox_keys(seed), step, tensor);
   if (int e = launch_status("tps_philox_fill")) return e;
   return ok();
 }
