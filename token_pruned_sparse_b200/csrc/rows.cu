@@ -206,15 +206,25 @@ __global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
         }
         ++p;
       } else {
+        uint4 x = make_uint4(0u, 0u, 0u, 0u), y = x;
+        if (lane < vpr) {
+          x = kc[row + lane];
+          y = vc[row + lane];
+        }
         for (int v = lane; v < vpr; v += 32) {
-          const uint4 x = kc[row + v];
-          const uint4 y = vc[row + v];
+          uint4 xn = x, yn = y;
+          if (v + 32 < vpr) {                       // the next vector's loads overlap this one's math
+            xn = kc[row + v + 32];
+            yn = vc[row + v + 32];
+          }
           const uint64_t e0 = static_cast<uint64_t>(n) * epr + static_cast<uint64_t>(v) * 8;
           float z[8];
           normals8(e0, step, 0u, keys, z);
           ke[row + v] = renoise_vec(x, a, b, z);
           normals8(e0, step, 1u, keys, z);
           ve[row + v] = renoise_vec(y, a, b, z);
+          x = xn;
+          y = yn;
         }
       }
     }
