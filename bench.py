@@ -667,9 +667,9 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
 
 
 def kernel_case(name, dev):
-    """One small, self-contained launch sequence of a single kernel for a
-    detailed counter capture (a few hundred MB on the device, inputs larger than
-    L2): a warm-up launch, then the launch to capture."""
+    """One self-contained launch sequence of a single kernel for a detailed
+    counter capture (inputs larger than L2, at most a few GB on the device): a
+    warm-up launch, then the launch to capture."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
     g.manual_seed(4)
@@ -682,6 +682,18 @@ def kernel_case(name, dev):
         for _ in range(2):
             tps.timeripple_score(x, v.F, v.Hs, v.Ws, synth.timeripple_windows(cfg.d), synth.TR_THETA,
                                  reuse=reuse, score=score)
+    elif name == "renoise":
+        # HSA step at |A| = N/3: K/V caches, fresh rows and K_eff/V_eff (3.4 GB in all)
+        cfg = synth.CONFIGS["hsa"]
+        N, H, d = cfg.video.N, cfg.H, cfg.d
+        A = N // 3
+        idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:A])[0].to(torch.int32)
+        cnt = torch.tensor([A], dtype=torch.int32, device=dev)
+        kc, vc = (torch.randn((N, H, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+        kf, vf = (torch.randn((A, H, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+        ke, ve = torch.empty_like(kc), torch.empty_like(vc)
+        for _ in range(2):
+            tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve)
     else:
         raise SystemExit(f"unknown kernel case {name}")
     torch.cuda.synchronize()
@@ -702,7 +714,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple"], default=None,
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise"], default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
                     help="run each HSA-size stage kernel once, print its table and exit (for counter captures)")
