@@ -300,12 +300,15 @@ int launch(const AttnArgs& a, cudaStream_t st) {
   if (a.cap == 0) return TPS_OK;
   size_t smem = Smem<D>::kBytes;
   if (a.bm) smem += static_cast<size_t>(a.nb) * 2 * sizeof(uint16_t);
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<bool> attr_set[64];   // the attribute is per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev >= 0 && dev < 64 && attr_set[dev].load(std::memory_order_acquire);
+  if (!cached) {
     cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(Smem<D>::kBytes + 4096 * 2 * sizeof(uint16_t)));
     if (e != cudaSuccess) return cuda_status(e, "pruned_attn_mma: smem attribute");
-    attr_set = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_release);
   }
   dim3 grid(static_cast<unsigned int>((a.cap + kBM - 1) / kBM), static_cast<unsigned int>(a.H));
   attn_mma_kernel<D><<<grid, kThreads, smem, st>>>(a, a.scale * kLog2e);

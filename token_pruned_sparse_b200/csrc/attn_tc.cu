@@ -483,13 +483,14 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   constexpr int kSmem = Layout<D>::kAlloc;
-  static bool attr_done[64] = {false};
+  static std::atomic<bool> attr_done[64];   // per device; setting the attribute twice is harmless
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  const bool cached = dev >= 0 && dev < 64 && attr_done[dev].load(std::memory_order_acquire);
+  if (!cached) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return cuda_status(e, "pruned_attn: smem attribute");
-    attr_done[dev] = true;
+    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
   }
   TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part};
   dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),

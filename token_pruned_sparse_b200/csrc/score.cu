@@ -107,16 +107,16 @@ void launch_score(const uint16_t* x, const uint16_t* xr, const uint16_t* xp, int
   constexpr int kThreads = 256;
   const int64_t tok_per_block = (kThreads / 32) * (32 / L);
   int64_t blocks = (N + kG * tok_per_block - 1) / (kG * tok_per_block);
-  static int per_sm[64] = {0};                  // resident blocks per SM (one wave)
+  static std::atomic<int> per_sm[64];           // resident blocks per SM (one wave), per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !per_sm[dev]) {
-    int b = 0;
+  int b = dev >= 0 && dev < 64 ? per_sm[dev].load(std::memory_order_relaxed) : 0;
+  if (!b) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, score_kernel<L, kV, kG>, kThreads, 0) != cudaSuccess || b < 1)
       b = 4;
-    per_sm[dev] = b;
+    if (dev >= 0 && dev < 64) per_sm[dev].store(b, std::memory_order_relaxed);
   }
-  const int64_t cap = static_cast<int64_t>(sm_count()) * (dev >= 0 && dev < 64 ? per_sm[dev] : 4);
+  const int64_t cap = static_cast<int64_t>(sm_count()) * b;
   if (blocks > cap) blocks = cap;
   score_kernel<L, kV, kG><<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(x, xr, xp, HW, C, N, score);
 }

@@ -550,17 +550,19 @@ __global__ void __launch_bounds__(kThreads) select_coop(CoopArgs a, int64_t N, u
 // Max co-resident blocks of a cooperative kernel on the current device (cached).
 template <int kMode>
 int coop_capacity() {
-  static int cap[64] = {0};
+  static std::atomic<int> cap[64];   // per device; two threads may both compute it, to the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (!cap[dev]) {
+  int c = cap[dev].load(std::memory_order_relaxed);
+  if (!c) {
     int per_sm = 0, coop = 0;
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_coop<kMode>, kThreads, 0) != cudaSuccess)
       return 0;
-    cap[dev] = per_sm * sm_count();
+    c = per_sm * sm_count();
+    cap[dev].store(c, std::memory_order_relaxed);
   }
-  return cap[dev];
+  return c;
 }
 
 // Runs the cooperative path when it applies; returns -1 when it does not.

@@ -372,24 +372,25 @@ int launch(const tps_bf16* x, int64_t F, int64_t Hs, int64_t Ws, int H, TrParams
   if (int e = tensor_map_encoder(&enc, "timeripple_score")) return e;
   CUtensorMap tm;
   if (int e = make_map5(enc, &tm, x, F, Hs, Ws, H, D)) return e;
-  static bool attr_done[64] = {false};
-  static int occ[64] = {0};
+  // resident CTAs per SM, per device; nonzero once the smem attribute is set on that device
+  static std::atomic<int> occ[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return fail(TPS_ERR_CUDA, "timeripple_score: device index %d", dev);
-  if (!attr_done[dev]) {
+  int oc = occ[dev].load(std::memory_order_acquire);
+  if (!oc) {
     cudaError_t e = cudaFuncSetAttribute(tr_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return cuda_status(e, "timeripple_score: smem attribute");
     int b = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, tr_kernel<D>, L::kThreads, L::kAlloc);
     if (e != cudaSuccess) return cuda_status(e, "timeripple_score: occupancy");
-    occ[dev] = b > 0 ? b : 1;
-    attr_done[dev] = true;
+    oc = b > 0 ? b : 1;
+    occ[dev].store(oc, std::memory_order_release);
   }
   p.tiles_x = static_cast<int>((Ws + kTX - 1) / kTX);
   p.tiles = p.tiles_x * static_cast<int>((Hs + kTY - 1) / kTY);
   const int64_t per_run = static_cast<int64_t>(p.tiles) * H;
-  p.chunk = choose_chunk(static_cast<int>(F), per_run, static_cast<int64_t>(occ[dev]) * sm_count());
+  p.chunk = choose_chunk(static_cast<int>(F), per_run, static_cast<int64_t>(oc) * sm_count());
   const int64_t runs = (F + p.chunk - 1) / p.chunk;
   const int64_t grid = per_run * runs;
   if (grid > 0x7fffffff) return fail(TPS_ERR_SHAPE, "timeripple_score: %lld work items", (long long)grid);
