@@ -1,0 +1,56 @@
+"""bench.py's reference arm on the host (no GPU): the JSON line it prints for
+the driver, the warm-up floor, and the quiet exit of every rank but 0 under a
+multi-rank launch."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _run(args, **env):
+    e = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    e.update(env)
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, env=e, capture_output=True,
+                          text=True, timeout=600)
+
+
+@pytest.fixture(scope="module")
+def ref_line():
+    r = _run(["--impl", "reference", "--steps", "2", "--warmup", "1"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1, r.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_line_carries_the_contract_keys(ref_line):
+    d = ref_line
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["n_gpus"] == 1 and d["steps"] == 2
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["dtype"] == "f64" and d["data"] == "synthetic"
+    assert "mid" in d["config"]["workload"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_warmup_is_raised_to_three(ref_line):
+    assert ref_line["warmup"] == 3
+
+
+def test_other_ranks_exit_without_work():
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "3"], RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
