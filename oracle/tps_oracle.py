@@ -207,7 +207,11 @@ def renoise_normals(seed: int, step: int, tensor: int, e) -> np.ndarray:
     Element e uses word (e mod 4) of counter block q = e div 4. Each word w
     maps to u = (floor(w / 2^9) + 1/2) * 2^-23 in (0, 1), a value that is
     exact in fp32 as well as fp64. Words (0, 1) and (2, 3) form Box-Muller
-    pairs: r = sqrt(-2 ln u_a), z_a = r cos(2 pi u_b), z_b = r sin(2 pi u_b)."""
+    pairs: r = sqrt(-2 ln u_a), z_a = r cos(2 pi u_b), z_b = r sin(2 pi u_b).
+    Pinned by the radius (z_a^2 + z_b^2 = -2 ln u_a) and angle
+    (atan2(z_b, z_a) = 2 pi u_b) identities read back from the raw words, by
+    within-pair independence, and by planted pairing slips
+    (tests/test_oracle_pins.py)."""
     e = np.asarray(e, np.int64)
     q = (e >> 2).astype(np.uint64)
     j = e & 3

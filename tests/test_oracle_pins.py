@@ -187,6 +187,77 @@ def test_renoise_statistics():
     np.testing.assert_array_equal(ke[idx], kc[idx].double().numpy())
 
 
+def _box_muller_pin_failures(normals):
+    """Names of the Box-Muller pins that `normals(seed, step, tensor, e)` breaks.
+
+    Box & Muller (1958): from two independent uniforms U1, U2 the pair
+    Z0 = sqrt(-2 ln U1) cos(2 pi U2), Z1 = sqrt(-2 ln U1) sin(2 pi U2) is two
+    independent N(0,1) deviates. The raw Philox words fix U1 (word 0 or 2 of
+    a counter block) and U2 (word 1 or 3), so the pins read them back:
+      radius  Z0^2 + Z1^2 = -2 ln U1 (fp64 rounding only),
+      angle   atan2(Z1, Z0) = 2 pi U2 (mod 2 pi),
+      pairing the two members of a pair, and the two pairs of a block, are
+              uncorrelated (|r| < 5/sqrt(n) over n = 2^16 blocks)."""
+    seed, step, tensor = 77, 3, 1
+    nq = 1 << 16
+    q = np.arange(nq)
+    z = normals(seed, step, tensor, np.arange(4 * nq)).reshape(nq, 4)
+    w = O.philox_words(seed, step, tensor, q).astype(np.float64)
+    u = (np.floor(w / 512.0) + 0.5) * 2.0 ** -23          # the word -> (0, 1) map of the oracle's reading
+    bad = []
+    for a, b in ((0, 1), (2, 3)):
+        r2 = z[:, a] ** 2 + z[:, b] ** 2
+        if not np.allclose(r2, -2.0 * np.log(u[:, a]), rtol=1e-12, atol=1e-300):
+            bad.append("radius")
+        ang = np.mod(np.arctan2(z[:, b], z[:, a]), 2 * np.pi)
+        err = np.abs(np.angle(np.exp(1j * (ang - 2 * np.pi * u[:, b]))))
+        if err.max() > 1e-9:
+            bad.append("angle")
+        if abs(np.corrcoef(z[:, a], z[:, b])[0, 1]) >= 5 / math.sqrt(nq):
+            bad.append("pairing")
+    if abs(np.corrcoef(z[:, 0], z[:, 2])[0, 1]) >= 5 / math.sqrt(nq):
+        bad.append("pairing")
+    return sorted(set(bad))
+
+
+def test_box_muller_pairing_radius_and_angle():
+    """The oracle's normals follow the Box-Muller pairing exactly: word 0 (2)
+    gives the radius, word 1 (3) the angle, cosine first, and the two deviates
+    of a pair are independent."""
+    assert _box_muller_pin_failures(O.renoise_normals) == []
+
+
+def _bm_variant(kind):
+    """The oracle's normals with one plausible Box-Muller slip planted."""
+    def fn(seed, step, tensor, e):
+        e = np.asarray(e, np.int64)
+        j = e & 3
+        w = O.philox_words(seed, step, tensor, (e >> 2).astype(np.uint64)).astype(np.float64)
+        u = (np.floor(w / 512.0) + 0.5) * 2.0 ** -23
+        pair = (j >> 1) * 2
+        ua = np.take_along_axis(u, pair[:, None], 1)[:, 0]
+        ub = np.take_along_axis(u, (pair + 1)[:, None], 1)[:, 0]
+        if kind == "same_u":            # both members of a pair from one uniform
+            ub = ua
+        if kind == "swapped_words":     # radius from the second word, angle from the first
+            ua, ub = ub, ua
+        r = np.sqrt(-2.0 * np.log(ua))
+        first = r * np.cos(2 * np.pi * ub)
+        second = r * (np.cos(2 * np.pi * ub) if kind == "cos_twice" else np.sin(2 * np.pi * ub))
+        if kind == "sin_first":
+            first, second = second, first
+        return np.where((j & 1) == 0, first, second)
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["cos_twice", "same_u", "swapped_words", "sin_first"])
+def test_box_muller_pins_catch_planted_mistakes(kind):
+    """Each slip keeps N(0,1) marginals (or nearly), which the moment and KS
+    pins cannot see; the pairing, radius and angle pins catch every one."""
+    assert _box_muller_pin_failures(_bm_variant("none")) == []
+    assert _box_muller_pin_failures(_bm_variant(kind)) != []
+
+
 def test_philox_words_uniform_and_distinct():
     """Raw stream properties beyond the known-answer vectors: uniform bytes
     and distinct streams across counters, steps, tensors and seeds."""
