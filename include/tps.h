@@ -154,9 +154,12 @@ TPS_API int lipar_select(const float* score, int64_t N, int mode, float tau, int
  * that loads the library until exit); larger N returns TPS_ERR_SHAPE. It
  * allocates nothing. The first call on each device looks up the array's
  * device address (with that device current), so make that first call before
- * any stream capture. All calls on a device share the one array: calls that
- * overlap on the GPU (e.g. on two streams without ordering) race; the scratch
- * keeps the last call's contents and is re-initialised by every call. */
+ * any stream capture. Devices numbered 64 and above look the address up on
+ * every call. The cached address does not survive cudaDeviceReset: do not
+ * call this entry point after resetting a device. All calls on a device share
+ * the one array: calls that overlap on the GPU (e.g. on two streams without
+ * ordering) race; the scratch keeps the last call's contents and is
+ * re-initialised by every call. */
 TPS_API int lipar_select_static(const float* score, int64_t N, int mode, float tau, int64_t k,
                                 int32_t* idx, int32_t* count, tps_stream stream);
 

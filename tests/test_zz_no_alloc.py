@@ -38,3 +38,30 @@ def test_static_select_matches_workspace_select_twice(N):
             assert int(cnt.item()) == n_ref, (mode, k, call)
             assert torch.equal(idx[:n_ref], ref_idx[:n_ref]), (mode, k, call)
     tps.tps_check()
+
+
+@pytest.mark.gpu
+def test_static_select_allocates_nothing():
+    """After one warm-up call (which looks up the scratch address), further
+    calls into preallocated outputs leave both the device's free memory and
+    torch's allocator untouched: the entry point itself allocates nothing."""
+    dev = "cuda"
+    N = 118800
+    s = synth.random_scores(N, 99, ties=True, specials=True).to(dev)
+    idx = torch.empty(N, dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    ref_idx, ref_cnt = tps.lipar_select(s, tps.SELECT_TOPK, k=N // 3)
+    tps.lipar_select_static(s, tps.SELECT_TOPK, k=N // 3, idx=idx, count=cnt)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for mode, tau, k in [(tps.SELECT_TOPK, 0.0, N // 3), (tps.SELECT_THRESHOLD, 0.5, 0),
+                         (tps.SELECT_TOPK, 0.0, N // 3)]:
+        tps.lipar_select_static(s, mode, tau=tau, k=k, idx=idx, count=cnt)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
+    n = int(ref_cnt.item())
+    assert int(cnt.item()) == n and torch.equal(idx[:n], ref_idx[:n])
+    tps.tps_check()

@@ -780,20 +780,29 @@ constexpr size_t kStaticBytes =
 static __device__ __align__(256) unsigned char g_select_scratch[kStaticBytes];
 
 // Device address of g_select_scratch on the current device. In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current. Devices 0..kCachedDevices-1 cache it after the first
+// call; a device with a higher index looks it up on every call (still no
+// allocation). The cache is not told about a context that is torn down and
+// recreated (cudaDeviceReset): such a caller must not use this entry point
+// after the reset.
+constexpr int kCachedDevices = 64;
 int static_scratch(void** out) {
-  static void* ptrs[64] = {nullptr};
+  static void* ptrs[kCachedDevices] = {nullptr};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_status(e, "lipar_select_static: cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(TPS_ERR_CUDA, "lipar_select_static: device %d out of range", dev);
+  const bool cacheable = dev >= 0 && dev < kCachedDevices;
   std::lock_guard<std::mutex> lk(mu);
-  if (!ptrs[dev]) {
+  if (!cacheable || !ptrs[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return cuda_status(e, "lipar_select_static: cudaGetSymbolAddress");
+    if (!cacheable) {
+      *out = p;
+      return TPS_OK;
+    }
     ptrs[dev] = p;
   }
   *out = ptrs[dev];
