@@ -1,15 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the token-pruned attention hot path on B200.
 
-One step = one pass of the whole per-layer path over one synthetic batch:
-    lipar_score -> lipar_select -> gather (Q, K, V of the active tokens)
-    -> kv_sync -> pruned_attn -> scatter_out
-on the mid workload (13 x 30x52 = 20280 tokens, 12 heads, d = 128, bf16,
-inter-frame relative-L1 score, top-k keep 30% = 6084 active queries attending
-all 20280 keys). The metric is pruned-attention TFLOP/s (algorithmic
-4*d*H*A*N FLOPs per step over the whole step's time) with active tokens/s per
-layer alongside; a keep-ratio sweep on the Wan-like layer (32760 tokens)
-times the attention kernel alone.
+One step = one pass of the whole per-layer path over one synthetic batch, on
+the largest configuration that fits one GPU: an HSA denoising step of a
+33 x 45x80 = 118800-token latent video, 24 heads, d = 128, bf16 --
+
+    lipar_score (inter-step relative L1 between two velocity tensors)
+    -> lipar_group (rank split into K = 3 groups, budgets 40/20/10 of T = 40)
+    -> lipar_schedule (step i = 1: the reference group only, |A| = N/3 = 39600)
+    -> gather (Q, K, V rows of the active tokens)
+    -> kv_sync (fresh rows into the K/V cache; pruned rows re-noised as
+       a*cache + b*eps with a = 1 - sigma_i, b = sigma_i, Philox normals)
+    -> pruned_attn (39600 active queries x all 118800 keys)
+    -> scatter_out (active rows over the cached outputs).
+
+The metric is pruned-attention TFLOP/s (algorithmic 4*d*H*A*N FLOPs per step
+over the whole step's time) with active tokens/s per layer alongside. The mid
+step (20280 tokens, 12 heads, top-k 30%) is reported as an extra key; a
+keep-ratio sweep on the Wan-like layer (32760 tokens) and per-config kernel
+numbers time the kernels alone.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -39,9 +48,7 @@ from token_pruned_sparse_b200 import synth  # noqa: E402
 METRIC = "pruned-attention TFLOP/s & active tokens/s per layer vs keep ratio; % roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20       # > 2x the 126 MB L2
-# this library's kernels per mid step: top-k select is one cooperative launch
-# (N = 20280 fits it; a cudaMemsetAsync clears its barrier word first)
-LAUNCHES = {"score": 1, "select_topk": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
+ATTN_SOURCES = ("attn_tc.cu", "attn_common.cuh", "tc_ptx.cuh", "tps_internal.cuh", "tma_host.cuh", "trace.cuh")
 
 
 def peaks():
@@ -54,8 +61,10 @@ def peaks():
 
 
 def attn_source_hash() -> str:
+    """Hash of the dense attention kernel's source files (the kernel and every
+    header it includes)."""
     h = hashlib.sha256()
-    for name in ("attn_tc.cu", "attn_common.cuh", "tc_ptx.cuh", "tps_internal.cuh", "tma_host.cuh", "trace.cuh"):
+    for name in ATTN_SOURCES:
         p = os.path.join(ROOT, "token_pruned_sparse_b200", "csrc", name)
         if os.path.exists(p):
             with open(p, "rb") as f:
@@ -63,10 +72,10 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_file: str):
-    """DRAM bytes per launch from the committed ncu summary, or None if the
-    kernel source changed since those counters were taken."""
-    p = os.path.join(ROOT, "profiles", kernel_file)
+def recorded_traffic(profile_file: str):
+    """DRAM bytes per launch from a committed ncu record, or None if the kernel
+    source changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", profile_file)
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -122,66 +131,41 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ------------------------------------------------------------- workload -------
-class MidStep:
-    """Device-resident mid workload and one step of the path."""
+# ------------------------------------------------------------- workloads ------
+HSA_STEP = 1          # an odd step: only the reference group is active, |A| = N/3
 
-    def __init__(self, seed_offset: int, dev, attn: str):
-        from token_pruned_sparse_b200 import tps
-        self.tps = tps
-        cfg = synth.CONFIGS["mid"]
-        spec = cfg.video
-        if seed_offset:
-            spec = synth.VideoSpec(spec.F, spec.Hs, spec.Ws, spec.C, spec.n_obj, spec.obj, spec.pan,
-                                   spec.seed + 1000 * seed_offset)
-        self.cfg, self.spec = cfg, spec
-        self.N, self.H, self.d, self.C = spec.N, cfg.H, cfg.d, spec.C
-        self.k = synth.keep_count(self.N, cfg.keep[0])
-        x, _ = synth.latent_video(spec)
-        xb = synth.to_bf16(x)
-        W = synth.projection_weights(self.C, self.H, self.d, spec.seed)
-        tok = xb.reshape(-1, self.C)
-        q, kf, vf = (synth.project(tok, w, self.H, self.d) for w in W)
-        HW = spec.HW
-        kc = torch.cat([kf[:HW], kf[:-HW]])       # cache = previous frame's projection
-        vc = torch.cat([vf[:HW], vf[:-HW]])
-        self.host = {"x": xb, "q": q, "k": kf, "v": vf}
-        self.x = xb.to(dev)
-        self.q, self.kf, self.vf = q.to(dev), kf.to(dev), vf.to(dev)
-        self.kc, self.vc = kc.to(dev), vc.to(dev)
-        self.o_full = torch.zeros((self.N, self.H, self.d), dtype=torch.bfloat16, device=dev)
-        self.score = torch.empty(self.N, dtype=torch.float32, device=dev)
-        self.idx = torch.empty(self.k, dtype=torch.int32, device=dev)
-        self.cnt = torch.empty(1, dtype=torch.int32, device=dev)
-        self.ws = tps.workspace(tps.OP_SELECT, self.N, 0, dev)
-        shp = (self.k, self.H, self.d)
-        self.q_act = torch.empty(shp, dtype=torch.bfloat16, device=dev)
-        self.k_new = torch.empty(shp, dtype=torch.bfloat16, device=dev)
-        self.v_new = torch.empty(shp, dtype=torch.bfloat16, device=dev)
-        self.o_act = torch.empty(shp, dtype=torch.bfloat16, device=dev)
-        self.scale = 1.0 / math.sqrt(self.d)
-        self.attn_fn = tps.pruned_attn if attn == "tc" else tps.pruned_attn_mma
-        self.flops = 4.0 * self.d * self.H * self.k * self.N
-        self.launches = sum(LAUNCHES.values())
 
-    def _pre(self, inp=None):
-        t = self.tps
-        x, q, kf, vf = (self.x, self.q, self.kf, self.vf) if inp is None else inp
-        t.lipar_score(x, out=self.score)
-        t.lipar_select(self.score, t.SELECT_TOPK, k=self.k, idx=self.idx, count=self.cnt, ws=self.ws)
-        t.tps_gather_rows(self.q_act, q, self.idx, self.cnt)
-        t.tps_gather_rows(self.k_new, kf, self.idx, self.cnt)
-        t.tps_gather_rows(self.v_new, vf, self.idx, self.cnt)
-        t.kv_sync(self.kc, self.vc, self.k_new, self.v_new, self.idx, self.cnt)
+def hsa_config(world: int) -> dict:
+    """The headline workload's description; both arms print this same dict."""
+    cfg = synth.CONFIGS["hsa"]
+    v = cfg.video
+    K, T, budgets = cfg.extra["K"], cfg.extra["T"], cfg.extra["budgets"]
+    A = v.N // K
+    return {"workload": f"HSA step: {v.F}x{v.Hs}x{v.Ws} = {v.N} tokens, {cfg.H} heads, d={cfg.d}, inter-step "
+                        f"rel-L1 score, K={K} rank groups (budgets {'/'.join(map(str, budgets))} of T={T}), "
+                        f"step i={HSA_STEP} active set |A| = N/3 = {A}, re-noised K/V cache sync "
+                        f"(a = 1-sigma_i, b = sigma_i, Philox normals), pruned attention of {A} queries x {v.N} "
+                        f"keys; step = score+group+schedule+gather(Q,K,V)+kv_sync+pruned_attn+scatter_out",
+            "N": v.N, "active": A, "heads": cfg.H, "head_dim": cfg.d, "latent_channels": v.C,
+            "l2": "flushed between timed steps (512 MiB write, then 512 MiB read: L2 left clean)",
+            "parallelism": f"replicas x{world}"}
 
-    def _post(self):
-        self.tps.scatter_out(self.o_full, self.o_act, self.idx, self.cnt)
+
+def project_on(dev, tok: torch.Tensor, W: np.ndarray, H: int, d: int) -> torch.Tensor:
+    """bf16 tokens [N, C] @ W -> bf16 [N, H, d] on `dev` (fp32 product, then
+    RNE): input preparation, untimed."""
+    y = tok.to(dev).float() @ torch.from_numpy(W).to(dev)
+    return y.to(torch.bfloat16).reshape(-1, H, d).contiguous()
+
+
+class PathStep:
+    """A device-resident workload and one step of the path: `_pre` (the stages
+    before attention), `_attn`, `_post` (scatter_out)."""
 
     def capture_graphs(self) -> bool:
-        """Capture the stages before and after attention as two CUDA graphs
-        (score, select, gathers, kv_sync; scatter_out), replayed each step; the
-        attention launch stays outside so its own events time it. Returns False
-        (eager launches) if capture is not possible."""
+        """Capture the stages before and after attention as two CUDA graphs,
+        replayed each step; the attention launch stays outside so its own
+        events time it. Returns False (eager launches) if capture fails."""
         try:
             self.g_pre, self.g_post = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.g_pre):
@@ -203,7 +187,7 @@ class MidStep:
             self._pre()
         if ev_attn:
             ev_attn[0].record()
-        self.attn_fn(self.q_act, self.kc, self.vc, self.idx, self.cnt, self.scale, o_act=self.o_act)
+        self._attn()
         if ev_attn:
             ev_attn[1].record()
         if getattr(self, "graphs", False):
@@ -212,6 +196,206 @@ class MidStep:
             self._post()
 
 
+class HsaStep(PathStep):
+    """HSA step at |A| = N/3 (step i = 1 of T = 40) on the 118800-token video.
+
+    Q/K/V are the projections of the current velocity tensor, the K/V cache
+    holds the previous step's projections, and the output cache starts at
+    zero (the step rewrites the active rows)."""
+
+    # this library's kernels per step: score 1; group 7 (radix init, 4 radix
+    # passes, count, write); schedule 1 (cooperative); gathers 3; kv_sync 2
+    # (cache rows, re-noise); attention 1; scatter 1
+    LAUNCHES = {"score": 1, "group": 7, "schedule": 1, "gather": 3, "kv_sync": 2, "attn": 1, "scatter": 1}
+
+    def __init__(self, seed_offset: int, dev, attn: str):
+        from token_pruned_sparse_b200 import tps
+        self.tps = tps
+        cfg = synth.CONFIGS["hsa"]
+        spec = cfg.video
+        if seed_offset:
+            spec = synth.VideoSpec(spec.F, spec.Hs, spec.Ws, spec.C, spec.n_obj, spec.obj, spec.pan,
+                                   spec.seed + 1000 * seed_offset)
+        self.cfg, self.spec = cfg, spec
+        self.N, self.H, self.d, self.C = spec.N, cfg.H, cfg.d, spec.C
+        self.K, self.T, self.budgets = cfg.extra["K"], cfg.extra["T"], tuple(cfg.extra["budgets"])
+        self.m = cfg.extra["m"]
+        self.i = HSA_STEP
+        sigma = 1.0 - self.i / self.T
+        self.renoise = (1.0 - sigma, sigma, spec.seed, self.i)
+        self.A = self.N // self.K
+        vp, delta = synth.velocity_pair(spec)
+        vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
+        F, HW, C = spec.F, spec.HW, spec.C
+        W = synth.projection_weights(C, self.H, self.d, spec.seed)
+        self.q, self.kf, self.vf = (project_on(dev, vcb, w, self.H, self.d) for w in W)
+        self.kc = project_on(dev, vpb, W[1], self.H, self.d)       # cache = the previous step's K/V
+        self.vc = project_on(dev, vpb, W[2], self.H, self.d)
+        self.host = {"vp": vpb.reshape(F, HW, C), "vc": vcb.reshape(F, HW, C)}
+        self.v_prev, self.v_cur = self.host["vp"].to(dev), self.host["vc"].to(dev)
+        self.ke, self.ve = torch.empty_like(self.kc), torch.empty_like(self.vc)
+        self.o_full = torch.zeros((self.N, self.H, self.d), dtype=torch.bfloat16, device=dev)
+        self.bufs = self.new_buffers(dev)
+        self.scale = 1.0 / math.sqrt(self.d)
+        self.attn_fn = tps.pruned_attn if attn == "tc" else tps.pruned_attn_mma
+        self.flops = 4.0 * self.d * self.H * self.A * self.N
+        self.units = self.A
+        self.launches = sum(self.LAUNCHES.values())
+
+    def new_buffers(self, dev):
+        t = self.tps
+        shp = (self.A, self.H, self.d)
+        z = lambda: torch.empty(shp, dtype=torch.bfloat16, device=dev)    # noqa: E731
+        return {"vp": torch.empty_like(self.v_prev), "vc": torch.empty_like(self.v_cur),
+                "score": torch.empty(self.N, dtype=torch.float32, device=dev),
+                "group": torch.empty(self.N, dtype=torch.int8, device=dev),
+                "idx": torch.empty(self.N, dtype=torch.int32, device=dev),
+                "cnt": torch.empty(1, dtype=torch.int32, device=dev),
+                "ws_g": t.workspace(t.OP_GROUP, self.N, self.K, dev),
+                "ws_s": t.workspace(t.OP_SCHEDULE, self.N, self.K, dev),
+                "q": z(), "k": z(), "v": z(), "o": z()}
+
+    def front(self, X, vp, vc, q, kf, vf):
+        """score -> group -> schedule -> gathers into buffer set X."""
+        t = self.tps
+        t.lipar_score(vc, vp, out=X["score"])
+        t.lipar_group(X["score"], self.K, group=X["group"], ws=X["ws_g"])
+        t.lipar_schedule(X["group"], self.K, self.budgets, self.T, self.i, self.m, idx=X["idx"], count=X["cnt"],
+                         ws=X["ws_s"])
+        t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
+        t.tps_gather_rows(X["k"], kf, X["idx"], X["cnt"])
+        t.tps_gather_rows(X["v"], vf, X["idx"], X["cnt"])
+
+    def sync(self, X):
+        self.tps.kv_sync(self.kc, self.vc, X["k"], X["v"], X["idx"], X["cnt"], renoise=self.renoise,
+                         k_eff=self.ke, v_eff=self.ve)
+
+    def attend(self, X):
+        self.attn_fn(X["q"], self.ke, self.ve, X["idx"], X["cnt"], self.scale, o_act=X["o"])
+
+    def _pre(self):
+        X = self.bufs
+        self.front(X, self.v_prev, self.v_cur, self.q, self.kf, self.vf)
+        self.sync(X)
+
+    def _attn(self):
+        self.attend(self.bufs)
+
+    def _post(self):
+        X = self.bufs
+        self.tps.scatter_out(self.o_full, X["o"], X["idx"], X["cnt"])
+
+    def active_count(self) -> int:
+        return int(self.bufs["cnt"].item())
+
+    # ---- end to end: the step's inputs in pinned host memory ------------------
+    def host_inputs(self):
+        """Pinned host copies of the step's inputs: the two velocity tensors and
+        the Q/K/V projections (the gathers read only the active rows of these)."""
+        return {"vp": self.host["vp"].pin_memory(), "vc": self.host["vc"].pin_memory(),
+                "q": self.q.cpu().pin_memory(), "k": self.kf.cpu().pin_memory(), "v": self.vf.cpu().pin_memory()}
+
+    def e2e_bytes(self, host):
+        R = self.H * self.d * 2
+        h2d = sum(host[k].numel() * host[k].element_size() for k in ("vp", "vc")) + 3 * self.A * R
+        return h2d, self.A * R
+
+    def e2e_front(self, X, host):
+        X["vp"].copy_(host["vp"], non_blocking=True)
+        X["vc"].copy_(host["vc"], non_blocking=True)
+        self.front(X, X["vp"], X["vc"], host["q"], host["k"], host["v"])     # gathers read rows over PCIe
+
+
+class MidStep(PathStep):
+    """Mid step: 13 x 30x52 = 20280 tokens, 12 heads, inter-frame score, top-k
+    30% = 6084 active queries; the K/V cache holds the previous frame's
+    projections."""
+
+    LAUNCHES = {"score": 1, "select_topk": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
+
+    def __init__(self, seed_offset: int, dev, attn: str):
+        from token_pruned_sparse_b200 import tps
+        self.tps = tps
+        cfg = synth.CONFIGS["mid"]
+        spec = cfg.video
+        if seed_offset:
+            spec = synth.VideoSpec(spec.F, spec.Hs, spec.Ws, spec.C, spec.n_obj, spec.obj, spec.pan,
+                                   spec.seed + 1000 * seed_offset)
+        self.cfg, self.spec = cfg, spec
+        self.N, self.H, self.d, self.C = spec.N, cfg.H, cfg.d, spec.C
+        self.k = synth.keep_count(self.N, cfg.keep[0])
+        self.A = self.k
+        x, _ = synth.latent_video(spec)
+        xb = synth.to_bf16(x)
+        W = synth.projection_weights(self.C, self.H, self.d, spec.seed)
+        tok = xb.reshape(-1, self.C)
+        q, kf, vf = (synth.project(tok, w, self.H, self.d) for w in W)
+        HW = spec.HW
+        kc = torch.cat([kf[:HW], kf[:-HW]])       # cache = previous frame's projection
+        vc = torch.cat([vf[:HW], vf[:-HW]])
+        self.host = {"x": xb, "q": q, "k": kf, "v": vf}
+        self.x = xb.to(dev)
+        self.q, self.kf, self.vf = q.to(dev), kf.to(dev), vf.to(dev)
+        self.kc, self.vc = kc.to(dev), vc.to(dev)
+        self.o_full = torch.zeros((self.N, self.H, self.d), dtype=torch.bfloat16, device=dev)
+        self.bufs = self.new_buffers(dev)
+        self.scale = 1.0 / math.sqrt(self.d)
+        self.attn_fn = tps.pruned_attn if attn == "tc" else tps.pruned_attn_mma
+        self.flops = 4.0 * self.d * self.H * self.k * self.N
+        self.units = self.k
+        self.launches = sum(self.LAUNCHES.values())
+
+    def new_buffers(self, dev):
+        t = self.tps
+        shp = (self.k, self.H, self.d)
+        z = lambda: torch.empty(shp, dtype=torch.bfloat16, device=dev)    # noqa: E731
+        return {"x": torch.empty_like(self.x), "score": torch.empty(self.N, dtype=torch.float32, device=dev),
+                "idx": torch.empty(self.k, dtype=torch.int32, device=dev),
+                "cnt": torch.empty(1, dtype=torch.int32, device=dev),
+                "ws": t.workspace(t.OP_SELECT, self.N, 0, dev), "q": z(), "k": z(), "v": z(), "o": z()}
+
+    def front(self, X, x, q, kf, vf):
+        t = self.tps
+        t.lipar_score(x, out=X["score"])
+        t.lipar_select(X["score"], t.SELECT_TOPK, k=self.k, idx=X["idx"], count=X["cnt"], ws=X["ws"])
+        t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
+        t.tps_gather_rows(X["k"], kf, X["idx"], X["cnt"])
+        t.tps_gather_rows(X["v"], vf, X["idx"], X["cnt"])
+
+    def sync(self, X):
+        self.tps.kv_sync(self.kc, self.vc, X["k"], X["v"], X["idx"], X["cnt"])
+
+    def attend(self, X):
+        self.attn_fn(X["q"], self.kc, self.vc, X["idx"], X["cnt"], self.scale, o_act=X["o"])
+
+    def _pre(self):
+        X = self.bufs
+        self.front(X, self.x, self.q, self.kf, self.vf)
+        self.sync(X)
+
+    def _attn(self):
+        self.attend(self.bufs)
+
+    def _post(self):
+        X = self.bufs
+        self.tps.scatter_out(self.o_full, X["o"], X["idx"], X["cnt"])
+
+    def active_count(self) -> int:
+        return int(self.bufs["cnt"].item())
+
+    def host_inputs(self):
+        return {k: v.pin_memory() for k, v in self.host.items()}
+
+    def e2e_bytes(self, host):
+        R = self.H * self.d * 2
+        return host["x"].numel() * host["x"].element_size() + 3 * self.k * R, self.k * R
+
+    def e2e_front(self, X, host):
+        X["x"].copy_(host["x"], non_blocking=True)
+        self.front(X, X["x"], host["q"], host["k"], host["v"])
+
+
+# ---------------------------------------------------------------- timing ------
 def rank_seed_offset(rank: int) -> int:
     """Each rank runs an independent layer: rank r shifts the video seed by r."""
     return rank
@@ -249,16 +433,12 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.sink)
 
 
-def flush_l2(flush):
-    flush()
-
-
-def timed_steps(fn, steps, flush_buf, with_attn=False):
+def timed_steps(fn, steps, flush, with_attn=False):
     """Per-step CUDA events on the launching stream, L2 flushed between steps."""
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     attn_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i in range(steps):
-        flush_l2(flush_buf)
+        flush()
         evs[i][0].record()
         fn(attn_evs[i] if with_attn else None)
         evs[i][1].record()
@@ -268,6 +448,125 @@ def timed_steps(fn, steps, flush_buf, with_attn=False):
     return step_ms, attn_ms
 
 
+def _time(fn, flush, reps=5, warm=2):
+    ms = []
+    for i in range(warm + reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= warm:
+            ms.append(a.elapsed_time(b))
+    return float(np.median(ms))
+
+
+def run_path(st, steps, warmup, world, use_graphs, flush, dev):
+    """Warm-up, then `steps` timed steps of a PathStep; returns (total ms and
+    mean attention ms, both max over ranks)."""
+    st.step()                     # first eager step: one-time setup (status word, occupancy queries)
+    torch.cuda.synchronize()
+    if use_graphs:
+        st.capture_graphs()
+    for _ in range(warmup):
+        st.step()
+    torch.cuda.synchronize()
+    st.tps.tps_check()
+    if st.active_count() != st.units:          # correctness guard on the timed configuration
+        raise RuntimeError(f"active count {st.active_count()} != {st.units}")
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, attn_ms = timed_steps(st.step, steps, flush, with_attn=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st.tps.tps_check()
+    total_ms, attn_avg = max_over_ranks([np.sum(step_ms), np.mean(attn_ms)], world, dev)
+    return total_ms, attn_avg
+
+
+# ------------------------------------------------------------------ e2e -------
+def e2e_leg(st, dev, steps, world):
+    """The same metric through the C ABI with the step's data in pinned host
+    memory and the result written back into host memory.
+
+    The library's kernels address pinned host memory directly (unified
+    addressing, checked with tps_pointer_is_device_accessible): the inputs the
+    step copies whole (velocity or latent tensors) are copied to the device,
+    the gathers read only the active rows of Q/K/V from host memory, and
+    scatter_out writes only the active rows of the caller's host-side output.
+    Step i+1's copy, score, selection and gathers run on a second stream
+    beside step i's kv_sync and attention; step i's scatter_out runs on a
+    third stream beside step i+1's attention."""
+    tps = st.tps
+    host = st.host_inputs()
+    o_host = torch.zeros((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory()
+    if not all(tps.pointer_is_device_accessible(t) for t in list(host.values()) + [o_host]):
+        return {"unavailable": "pinned host memory is not device-accessible here"}
+    h2d, d2h = st.e2e_bytes(host)
+    sets = [st.new_buffers(dev), st.new_buffers(dev)]
+    comp = torch.cuda.current_stream()
+    s_pre, s_post = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()           # noqa: E731
+    pre_done, attn_done, free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in free:
+        e.record(comp)
+
+    def pre(i):
+        b = i & 1
+        with torch.cuda.stream(s_pre):
+            s_pre.wait_event(free[b])
+            st.e2e_front(sets[b], host)
+            pre_done[b].record(s_pre)
+
+    def main(i):
+        b = i & 1
+        X = sets[b]
+        comp.wait_event(pre_done[b])
+        st.sync(X)
+        st.attend(X)
+        attn_done[b].record(comp)
+        with torch.cuda.stream(s_post):
+            s_post.wait_event(attn_done[b])
+            tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])          # rows written over PCIe
+            free[b].record(s_post)
+
+    def run(n):
+        pre(0)
+        for i in range(n):
+            if i + 1 < n:
+                pre(i + 1)
+            main(i)
+        comp.wait_stream(s_post)
+
+    run(2)
+    torch.cuda.synchronize()
+    tps.tps_check()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    s_pre.wait_event(a)
+    run(steps)
+    b.record(comp)
+    torch.cuda.synchronize()
+    tps.tps_check()
+    ms = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
+    # the host-side output must equal the device-resident path's (same inputs, same kernels)
+    st.step()
+    torch.cuda.synchronize()
+    if not torch.equal(o_host, st.o_full.cpu()):
+        raise RuntimeError("e2e: host-side output differs from the device-resident step")
+    return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": round(ms / steps, 4),
+            "mode": "pinned host data; whole velocity/latent tensors copied in, gathers read and scatter_out "
+                    "writes only the active rows over PCIe; step i+1's front end and step i-1's scatter overlap "
+                    "step i's attention"}
+
+
+# ------------------------------------------------------- kernel sweeps --------
 def keep_sweep(dev, attn, reps=5):
     """Wan-like layer (32760 tokens, 12 heads): attention kernel alone per keep ratio."""
     from token_pruned_sparse_b200 import tps
@@ -284,241 +583,16 @@ def keep_sweep(dev, attn, reps=5):
         idx = torch.from_numpy(np.sort(np.random.default_rng(304).choice(N, A, replace=False)).astype(np.int32)).to(dev)
         cnt = torch.tensor([A], dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
-        ms = []
-        for i in range(reps + 2):
-            flush_l2(flush)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o)
-            b.record()
-            torch.cuda.synchronize()
-            if i >= 2:
-                ms.append(a.elapsed_time(b))
-        t = float(np.median(ms))
+        t = _time(lambda: fn(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o), flush, reps=reps)
         fl = 4.0 * d * H * A * N
         # the same call through pruned_attn_ws (key-range splits when the grid is thin)
         ws, nws = tps.attn_workspace(A, N, H, d, dev)
-        ms = []
-        for i in range(reps + 2):
-            flush_l2(flush)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            tps.pruned_attn_ws(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o, ws=ws)
-            b.record()
-            torch.cuda.synchronize()
-            if i >= 2:
-                ms.append(a.elapsed_time(b))
-        tw = float(np.median(ms))
+        tw = _time(lambda: tps.pruned_attn_ws(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o, ws=ws), flush,
+                   reps=reps)
         out.append({"keep": r, "active": A, "attn_ms": round(t, 4), "tflops": round(fl / t / 1e9, 1),
                     "active_tokens_per_s": round(A / t * 1e3, 1), "attn_ws_ms": round(tw, 4),
                     "tflops_ws": round(fl / tw / 1e9, 1), "ws_bytes": nws})
     return out
-
-
-# -------------------------------------------------------- CPU oracle leg ------
-class OracleStep:
-    """The fp64 oracle on the mid step, inputs prepared once (untimed).
-
-    ``linear()`` times score, select, gather, kv_sync and scatter over all
-    tokens; ``attn(rows)`` times the attention of `rows` sampled active rows x
-    all heads. A full step is extrapolated as linear + attn * (k / rows)."""
-
-    def __init__(self):
-        import oracle as O
-        self.O = O
-        try:
-            from threadpoolctl import threadpool_info
-            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        except Exception:  # pragma: no cover
-            self.threads = 1
-        cfg = synth.CONFIGS["mid"]
-        spec = cfg.video
-        x, _ = synth.latent_video(spec)
-        self.xb = synth.to_bf16(x)
-        W = synth.projection_weights(spec.C, cfg.H, cfg.d, spec.seed)
-        tok = self.xb.reshape(-1, spec.C)
-        self.q, self.kf, self.vf = (synth.project(tok, w, cfg.H, cfg.d) for w in W)
-        HW = spec.HW
-        self.kc = torch.cat([self.kf[:HW], self.kf[:-HW]])
-        self.vc = torch.cat([self.vf[:HW], self.vf[:-HW]])
-        self.k = synth.keep_count(spec.N, cfg.keep[0])
-        self.N, self.H, self.d = spec.N, cfg.H, cfg.d
-        self.flops = 4.0 * self.d * self.H * self.k * self.N
-        self.rng = np.random.default_rng(7)
-        self.state = None
-
-    def linear(self):
-        O = self.O
-        t0 = time.perf_counter()
-        s = O.lipar_score(self.xb)
-        idx = O.select_topk(s, self.k)
-        q_act = O.gather_rows(self.q, idx)
-        kc2, vc2, _, _ = O.kv_sync(self.kc, self.vc, self.kf[idx], self.vf[idx], idx)
-        O.scatter_out(torch.zeros_like(self.kc), q_act, idx)
-        # exact fp64 widening of the attention inputs, once per step, head-major
-        # so that every head's K/V is one contiguous matrix (views of [N, H, d])
-        hm = lambda t: np.ascontiguousarray(O.f64(t).transpose(1, 0, 2)).transpose(1, 0, 2)
-        self.state = (idx, hm(q_act), hm(kc2), hm(vc2))
-        return time.perf_counter() - t0
-
-    def attn(self, rows):
-        idx, q_act, kc2, vc2 = self.state
-        r = self.rng.choice(self.k, rows, replace=False)
-        t0 = time.perf_counter()
-        self.O.pruned_attn(q_act, kc2, vc2, idx, 1 / math.sqrt(self.d), rows=r)
-        return time.perf_counter() - t0
-
-    def fit(self, r1=64, r2=256):
-        """Fixed cost per attention call (the per-head fp64 widening of K and V):
-        t(rows) = a + b * rows from two sample sizes."""
-        self.attn(r1)                                    # warm
-        t1, t2 = self.attn(r1), self.attn(r2)
-        b = max((t2 - t1) / (r2 - r1), 1e-9)
-        self.a = max(t1 - b * r1, 0.0)
-        return self.a
-
-    def full_step(self, t_lin, t_attn, rows):
-        a = getattr(self, "a", 0.0)
-        return t_lin + a + max(t_attn - a, 0.0) * self.k / rows
-
-    def describe(self, rows):
-        return (f"mid step: score/select/gather/kv_sync/scatter over all {self.N} tokens plus attention for "
-                f"{rows} sampled of {self.k} active rows x {self.H} heads (fp64, numpy/BLAS); the full step is "
-                f"extrapolated as linear stages + per-call cost + per-row cost x {self.k} (per-call and per-row "
-                f"costs fitted from 64- and 256-row samples)")
-
-
-def oracle_baseline():
-    """cpu_baseline of the GPU arm: one complete mid step through the fp64
-    oracle (every active row, every head), timed on the host cores."""
-    o = OracleStep()
-    t_lin = o.linear()
-    t_att = o.attn(o.k)
-    full = t_lin + t_att
-    return {"value": round(o.flops / full / 1e12, 6), "unit": "TFLOP/s", "cores": o.threads, "kind": "oracle",
-            "sample": f"one complete mid step (score/select/gather/kv_sync/scatter over {o.N} tokens, attention "
-                      f"of all {o.k} active rows x {o.H} heads in fp64 numpy/BLAS)",
-            "seconds": round(full, 2)}
-
-
-# ------------------------------------------------------- per-config sweep ------
-def oracle_config_baselines(rows: int = 128):
-    """The fp64 oracle on every config, each a bounded sample, reported beside the
-    GPU numbers (a baseline, not a target). Per config and step size: the O(N)
-    stages (score, select or HSA groups/schedule, gather, kv_sync -- re-noise on
-    one head at the HSA size -- and scatter) run over all tokens; attention runs
-    for `rows` sampled active rows of one head, and the layer step is
-    extrapolated as O(N) stages + per-(row, head) attention cost x |A| x H."""
-    import oracle as O
-    out = {}
-    rng = np.random.default_rng(11)
-
-    def tm(fn):
-        t0 = time.perf_counter()
-        r = fn()
-        return time.perf_counter() - t0, r
-
-    def attn_cost(q, k, v, idx, scale, bm=None):
-        """(per-head fixed cost, per-(row, head) cost) from samples of rows/2 and 2*rows rows"""
-        ts = []
-        for n in (rows // 2, 2 * rows):
-            r = rng.choice(len(idx), min(n, len(idx)), replace=False)
-            t, _ = tm(lambda: O.pruned_attn(q, k, v, idx, scale, blockmask=bm, rows=r, heads=[0]))
-            ts.append((len(r), t))
-        (n1, t1), (n2, t2) = ts
-        b = max((t2 - t1) / max(n2 - n1, 1), 1e-9)
-        return max(t1 - b * n1, 0.0), b
-
-    def report(name, t_lin, cost, A, H, N, d, flops, sampled):
-        step = t_lin + H * (cost[0] + cost[1] * A)
-        out[name] = {"seconds_per_step": round(step, 4), "tflops_alg": round(flops / step / 1e12, 6),
-                     "active_tokens_per_s": round(A / step, 1), "measured_linear_seconds": round(sampled, 3),
-                     "active": int(A), "tokens": int(N)}
-
-    def qkv(tok, cfg):
-        W = synth.projection_weights(cfg.video.C, cfg.H, cfg.d, cfg.video.seed)
-        return [synth.project(tok, w, cfg.H, cfg.d) for w in W]
-
-    # tiny: the complete step, all rows and heads
-    cfg = synth.CONFIGS["tiny"]
-    x, _ = synth.latent_video(cfg.video)
-    xb = synth.to_bf16(x)
-    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
-    t_all, _ = tm(lambda: O.pruned_attn(q, kf, vf, O.select_threshold(O.lipar_score(xb), cfg.tau),
-                                        1 / math.sqrt(cfg.d)))
-    A = len(O.select_threshold(O.lipar_score(xb), cfg.tau))
-    report("tiny", t_all, (0.0, 0.0), A, cfg.H, cfg.video.N, cfg.d, O.attn_flops(A, cfg.video.N, cfg.H, cfg.d),
-           t_all)
-
-    # Wan, inter-step score, keep 10/30/50/100%
-    cfg = synth.CONFIGS["wan"]
-    vp, delta = synth.velocity_pair(cfg.video)
-    vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
-    N, H, d = cfg.video.N, cfg.H, cfg.d
-    q, kf, vf = qkv(vcb, cfg)
-    t_score, s = tm(lambda: O.lipar_score(vcb[None], vpb[None]))
-    for ratio in cfg.keep:
-        k = synth.keep_count(N, ratio)
-        t_sel, idx = tm(lambda: O.select_topk(s, k))
-        t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.kv_sync(kf, vf, kf[idx], vf[idx], idx),
-                                O.scatter_out(q, q[idx], idx)))
-        per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d))
-        report(f"wan_keep{int(ratio * 100)}", t_score + t_sel + t_rows, per, k, H, N, d,
-               O.attn_flops(k, N, H, d), t_score + t_sel + t_rows)
-
-    # HSA: groups + schedule, re-noise, attention at |A| = N/3 (odd steps)
-    cfg = synth.CONFIGS["hsa"]
-    vp, delta = synth.velocity_pair(cfg.video)
-    vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
-    N, H, d = cfg.video.N, cfg.H, cfg.d
-    K, T, budgets = cfg.extra["K"], cfg.extra["T"], cfg.extra["budgets"]
-    q, kf, vf = qkv(vcb, cfg)
-    t_score, s = tm(lambda: O.lipar_score(vcb[None], vpb[None]))
-    t_grp, g = tm(lambda: O.group_split(s, K))
-    t_sch, idx = tm(lambda: O.schedule_active(g, K, budgets, T, 1, 0))
-    t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.scatter_out(q, q[idx], idx)))
-    t_rn, _ = tm(lambda: O.kv_sync(kf, vf, kf[idx], vf[idx], idx, renoise=(0.025, 0.975, 4, 1), heads=[0]))
-    per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d))
-    A = len(idx)
-    t_lin = t_score + t_grp + t_sch + t_rows + t_rn * H
-    report("hsa_step_A_N/3", t_lin, per, A, H, N, d, O.attn_flops(A, N, H, d),
-           t_score + t_grp + t_sch + t_rows + t_rn)
-
-    # block-sparse: inter-frame top-k 40%, 139 of 929 key blocks per query block
-    cfg = synth.CONFIGS["block"]
-    x, _ = synth.latent_video(cfg.video)
-    xb = synth.to_bf16(x)
-    N, H, d = cfg.video.N, cfg.H, cfg.d
-    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
-    t_score, s = tm(lambda: O.lipar_score(xb))
-    kk = synth.keep_count(N, cfg.keep[0])
-    t_sel, idx = tm(lambda: O.select_topk(s, kk))
-    bm = synth.block_mask_band_random(cfg.video, 128, cfg.extra["kept_per_row"], cfg.video.seed)
-    per = attn_cost(q[idx], kf, vf, idx, 1 / math.sqrt(d), bm=bm)
-    keys = bm.numpy()[np.asarray(idx) // 128].sum(axis=1) * 128.0
-    report("block_sparse", t_score + t_sel, per, kk, H, N, d, O.attn_flops(kk, N, H, d, keys),
-           t_score + t_sel)
-    for v in out.values():
-        v["sample"] = (f"O(N) stages over all tokens (HSA re-noise on one head, x H); attention timed for "
-                       f"{rows // 2} and {2 * rows} sampled active rows of one head, split into a per-head and "
-                       f"a per-row cost, and extrapolated to all rows and heads")
-    return out
-
-
-def _time(fn, flush, reps=5, warm=2):
-    ms = []
-    for i in range(warm + reps):
-        flush_l2(flush)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        fn()
-        b.record()
-        torch.cuda.synchronize()
-        if i >= warm:
-            ms.append(a.elapsed_time(b))
-    return float(np.median(ms))
-
-
 def executed_key_tiles(idx: np.ndarray, N: int, nb_mask=None, rows_per_cta=256):
     """Key tiles the attention kernel runs per CTA (dense: all; masked: the
     union of the mask rows of the query blocks a CTA spans)."""
@@ -666,17 +740,25 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     return out
 
 
+
+
 def kernel_case(name, dev):
-    """One self-contained launch sequence of a single kernel for a detailed
-    counter capture (inputs larger than L2, at most a few GB on the device): a
-    warm-up launch, then the launch to capture."""
+    """One self-contained launch sequence of a single kernel for a counter
+    capture (inputs larger than L2, at most a few GB on the device): a warm-up
+    launch, then the launch to capture.
+
+    attn_mid: one mid-size attention launch (6084 queries x 20280 keys, 12
+    heads). attn_hsa_h4: the HSA step's attention (39600 queries x 118800
+    keys) on 4 of its 24 heads; heads are independent units of the grid, so a
+    full launch moves 6x these bytes."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
     g.manual_seed(4)
+    rnd = lambda *shape: torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)   # noqa: E731
     if name == "timeripple":
         cfg = synth.CONFIGS["hsa"]
         v = cfg.video
-        x = torch.randn((v.N, cfg.H, cfg.d), generator=g, device=dev).to(torch.bfloat16)   # 730 MB
+        x = rnd(v.N, cfg.H, cfg.d)                                      # 730 MB
         reuse = torch.empty((v.N, cfg.H), dtype=torch.uint8, device=dev)
         score = torch.empty(v.N, dtype=torch.float32, device=dev)
         for _ in range(2):
@@ -689,11 +771,24 @@ def kernel_case(name, dev):
         A = N // 3
         idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:A])[0].to(torch.int32)
         cnt = torch.tensor([A], dtype=torch.int32, device=dev)
-        kc, vc = (torch.randn((N, H, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
-        kf, vf = (torch.randn((A, H, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+        kc, vc = rnd(N, H, d), rnd(N, H, d)
+        kf, vf = rnd(A, H, d), rnd(A, H, d)
         ke, ve = torch.empty_like(kc), torch.empty_like(vc)
         for _ in range(2):
             tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve)
+    elif name in ("attn_mid", "attn_hsa_h4"):
+        if name == "attn_mid":
+            cfg = synth.CONFIGS["mid"]
+            N, H, d, A = cfg.video.N, cfg.H, cfg.d, synth.keep_count(cfg.video.N, cfg.keep[0])
+        else:
+            cfg = synth.CONFIGS["hsa"]
+            N, H, d, A = cfg.video.N, 4, cfg.d, cfg.video.N // 3
+        idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:A])[0].to(torch.int32)
+        cnt = torch.tensor([A], dtype=torch.int32, device=dev)
+        q, k, v = rnd(A, H, d), rnd(N, H, d), rnd(N, H, d)
+        o = torch.empty_like(q)
+        for _ in range(2):
+            tps.pruned_attn(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o)
     else:
         raise SystemExit(f"unknown kernel case {name}")
     torch.cuda.synchronize()
@@ -701,20 +796,268 @@ def kernel_case(name, dev):
     return {"kernel_case": name, "ok": True}
 
 
+# -------------------------------------------------------- CPU oracle leg ------
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        return 1
+
+
+class OracleHsaSlice:
+    """The fp64 oracle on the HSA step, timed as proportional slices.
+
+    Setup (untimed): the step's inputs; the full score, group and schedule (the
+    step's active set; those two global rank steps take about 0.05 s of a full
+    step that takes tens of minutes, and are not part of the slices); head 0's
+    projections and its re-noised K_eff/V_eff (the oracle's kv_sync with
+    re-noise, that head only), widened once to fp64.
+
+    slice(r) runs one bounded sample holding the share phi = r / (A*H) of every
+    per-row and per-token stage of the step: attention of r sampled active rows
+    of head 0 against all N keys, the score of ceil(phi*N) tokens, kv_sync with
+    re-noise over ceil(phi*N) rows of all heads, and the gather and scatter of
+    ceil(phi*A) active rows. It returns its own seconds; the attention FLOPs it
+    performs are 4*d*r*N."""
+
+    def __init__(self):
+        import oracle as O
+        self.O = O
+        self.threads = _threads()
+        cfg = synth.CONFIGS["hsa"]
+        spec = cfg.video
+        self.N, self.H, self.d, self.C = spec.N, cfg.H, cfg.d, spec.C
+        K, T, budgets = cfg.extra["K"], cfg.extra["T"], cfg.extra["budgets"]
+        sigma = 1.0 - HSA_STEP / T
+        self.renoise = (1.0 - sigma, sigma, spec.seed, HSA_STEP)
+        vp, delta = synth.velocity_pair(spec)
+        self.vpb, self.vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
+        s = O.lipar_score(self.vcb[None], self.vpb[None])
+        g = O.group_split(s, K)
+        self.idx = O.schedule_active(g, K, budgets, T, HSA_STEP, cfg.extra["m"])
+        self.A = len(self.idx)
+        W = synth.projection_weights(self.C, self.H, self.d, spec.seed)
+        d = self.d
+        # head 0 over all tokens (embedded in full-width tensors, so the re-noise
+        # element indices are those of the full layer)
+        def head0(tok, w):
+            out = torch.zeros((self.N, self.H, d), dtype=torch.bfloat16)
+            out[:, 0] = (tok.float() @ torch.from_numpy(np.ascontiguousarray(w[:, :d]))).to(torch.bfloat16)
+            return out
+        q0, kf0, vf0 = (head0(self.vcb, w) for w in W)
+        kc0, vc0 = head0(self.vpb, W[1]), head0(self.vpb, W[2])
+        _, _, ke, ve = O.kv_sync(kc0, vc0, kf0[self.idx], vf0[self.idx], self.idx, renoise=self.renoise,
+                                 heads=[0])
+        self.ke, self.ve = ke, ve                                      # fp64 [N, 1, d]
+        self.q0 = O.f64(q0[torch.as_tensor(self.idx)][:, :1])          # fp64 [A, 1, d]
+        del q0, kf0, vf0, kc0, vc0
+        # all heads for a pool of tokens (the O(N) slices)
+        self.pool = 4096
+        tok_c, tok_p = self.vcb[: self.pool], self.vpb[: self.pool]
+        self.pq, self.pkf, self.pvf = (synth.project(tok_c, w, self.H, d) for w in W)
+        self.pkc, self.pvc = synth.project(tok_p, W[1], self.H, d), synth.project(tok_p, W[2], self.H, d)
+        self.rng = np.random.default_rng(7)
+        self.flops_per_row = 4.0 * d * self.N
+
+    def slice(self, r: int) -> float:
+        O = self.O
+        phi = r / (self.A * self.H)
+        n = min(self.pool, max(1, math.ceil(phi * self.N)))
+        m = min(n, max(1, math.ceil(phi * self.A)))
+        t0n = int(self.rng.integers(0, self.N - n + 1))
+        rows = self.rng.choice(self.A, r, replace=False)
+        local = np.arange(0, n, 3)[:m]                                 # active rows inside the token slice
+        t0 = time.perf_counter()
+        O.lipar_score(self.vcb[t0n:t0n + n][None], self.vpb[t0n:t0n + n][None])
+        fresh = [O.gather_rows(t, local) for t in (self.pq, self.pkf, self.pvf)]
+        O.kv_sync(self.pkc[:n], self.pvc[:n], fresh[1], fresh[2], local, renoise=self.renoise)
+        O.pruned_attn(self.q0, self.ke, self.ve, self.idx, 1 / math.sqrt(self.d), rows=rows)
+        O.scatter_out(self.pq[:n], fresh[0], local)
+        return time.perf_counter() - t0
+
+    def describe(self, r: int) -> str:
+        phi = r / (self.A * self.H)
+        return (f"HSA step (N={self.N}, |A|={self.A}, {self.H} heads): proportional slice phi = r/(A*H) with "
+                f"r = {r} sampled active rows of one head attending all {self.N} keys, plus phi of every O(N) "
+                f"stage (score of ceil(phi*N) tokens, re-noised kv_sync of ceil(phi*N) rows x all heads, gather "
+                f"and scatter of ceil(phi*A) rows); phi = {phi:.2e}; fp64 numpy/BLAS. The group and schedule "
+                f"rank steps (about 0.05 s per full step) run once at setup")
+
+
+def oracle_baseline(rows: int = 8192):
+    """cpu_baseline of the GPU arm: one proportional slice of the HSA step
+    through the fp64 oracle on the host cores (about 10 s)."""
+    o = OracleHsaSlice()
+    o.slice(64)                                                        # warm
+    t = o.slice(rows)
+    return {"value": round(o.flops_per_row * rows / t / 1e12, 6), "unit": "TFLOP/s", "cores": o.threads,
+            "kind": "oracle", "sample": o.describe(rows), "seconds": round(t, 2)}
+
+
+def attn_cost_fit(O, q, k, v, idx, scale, bm=None, counts=(32, 128, 512), reps=3, seed=11):
+    """The oracle's attention cost on one config, fitted once: head 0's Q/K/V
+    are widened to fp64 once, then t(rows) = a + b*rows is fitted by least
+    squares to the median of `reps` timings at each row count. Returns
+    (a seconds per head-call, b seconds per (row, head), worst relative residual)."""
+    rng = np.random.default_rng(seed)
+    qh, kh, vh = O.f64(q[:, :1]), O.f64(k[:, :1]), O.f64(v[:, :1])
+    counts = [min(c, len(idx)) for c in counts]
+    med = []
+    for c in counts:
+        ts = []
+        for _ in range(reps):
+            r = rng.choice(len(idx), c, replace=False)
+            t0 = time.perf_counter()
+            O.pruned_attn(qh, kh, vh, idx, scale, blockmask=bm, rows=r)
+            ts.append(time.perf_counter() - t0)
+        med.append(float(np.median(ts)))
+    if len(set(counts)) > 1:
+        b, a = np.polyfit(np.asarray(counts, float), np.asarray(med), 1)
+    else:
+        a, b = 0.0, med[0] / counts[0]
+    a, b = max(float(a), 0.0), max(float(b), 1e-12)
+    resid = max(abs(m - (a + b * c)) / m for m, c in zip(med, counts))
+    return a, b, resid
+
+
+def oracle_config_baselines():
+    """The fp64 oracle on the other configs, reported beside the GPU numbers (a
+    baseline, not a target). The O(N) stages (score, selection, gather,
+    kv_sync, scatter) run over all tokens; the attention cost per (row, head)
+    is fitted once per config (attn_cost_fit: it depends on N, d and the mask,
+    not on |A|) and the step is extrapolated as O(N) stages + H * (a + b*|A|)."""
+    import oracle as O
+    out = {}
+
+    def tm(fn):
+        t0 = time.perf_counter()
+        r = fn()
+        return time.perf_counter() - t0, r
+
+    def report(name, t_lin, fit, A, H, N, flops):
+        a, b, resid = fit
+        step = t_lin + H * (a + b * A)
+        out[name] = {"seconds_per_step_extrapolated": round(step, 3), "tflops_alg": round(flops / step / 1e12, 6),
+                     "active_tokens_per_s": round(A / step, 1), "o_n_stages_seconds": round(t_lin, 3),
+                     "attn_fit": {"per_head_s": round(a, 5), "per_row_head_s": round(b, 7),
+                                  "worst_rel_residual": round(resid, 3)},
+                     "active": int(A), "tokens": int(N)}
+
+    def qkv(tok, cfg):
+        W = synth.projection_weights(cfg.video.C, cfg.H, cfg.d, cfg.video.seed)
+        return [synth.project(tok, w, cfg.H, cfg.d) for w in W]
+
+    # tiny: the complete step, all rows and heads
+    cfg = synth.CONFIGS["tiny"]
+    x, _ = synth.latent_video(cfg.video)
+    xb = synth.to_bf16(x)
+    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
+    t_all, idx = tm(lambda: O.select_threshold(O.lipar_score(xb), cfg.tau))
+    t_att, _ = tm(lambda: O.pruned_attn(q[idx], kf, vf, idx, 1 / math.sqrt(cfg.d)))
+    out["tiny"] = {"seconds_per_step": round(t_all + t_att, 4), "active": int(len(idx)), "tokens": cfg.video.N,
+                   "tflops_alg": round(O.attn_flops(len(idx), cfg.video.N, cfg.H, cfg.d) / (t_all + t_att) / 1e12, 6),
+                   "sample": "the complete step"}
+
+    # mid: inter-frame top-k 30%
+    cfg = synth.CONFIGS["mid"]
+    x, _ = synth.latent_video(cfg.video)
+    xb = synth.to_bf16(x)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
+    k = synth.keep_count(N, cfg.keep[0])
+    t_lin, idx = tm(lambda: O.select_topk(O.lipar_score(xb), k))
+    t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.kv_sync(kf, vf, kf[idx], vf[idx], idx),
+                            O.scatter_out(q, q[idx], idx)))
+    report("mid", t_lin + t_rows, attn_cost_fit(O, q[idx], kf, vf, idx, 1 / math.sqrt(d)), k, H, N,
+           O.attn_flops(k, N, H, d))
+
+    # Wan, inter-step score, keep 10/30/50/100%: one attention fit for all ratios
+    cfg = synth.CONFIGS["wan"]
+    vp, delta = synth.velocity_pair(cfg.video)
+    vpb, vcb = synth.to_bf16(vp), synth.to_bf16(vp + delta)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    q, kf, vf = qkv(vcb, cfg)
+    t_score, s = tm(lambda: O.lipar_score(vcb[None], vpb[None]))
+    fit = None
+    for ratio in cfg.keep:
+        k = synth.keep_count(N, ratio)
+        t_sel, idx = tm(lambda: O.select_topk(s, k))
+        t_rows, _ = tm(lambda: (O.gather_rows(q, idx), O.kv_sync(kf, vf, kf[idx], vf[idx], idx),
+                                O.scatter_out(q, q[idx], idx)))
+        if fit is None:
+            fit = attn_cost_fit(O, q[idx], kf, vf, idx, 1 / math.sqrt(d))
+        report(f"wan_keep{int(ratio * 100)}", t_score + t_sel + t_rows, fit, k, H, N, O.attn_flops(k, N, H, d))
+
+    # block-sparse: inter-frame top-k 40%, 139 of 929 key blocks per query block
+    cfg = synth.CONFIGS["block"]
+    x, _ = synth.latent_video(cfg.video)
+    xb = synth.to_bf16(x)
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    q, kf, vf = qkv(xb.reshape(-1, cfg.video.C), cfg)
+    kk = synth.keep_count(N, cfg.keep[0])
+    t_lin, idx = tm(lambda: O.select_topk(O.lipar_score(xb), kk))
+    bm = synth.block_mask_band_random(cfg.video, 128, cfg.extra["kept_per_row"], cfg.video.seed)
+    keys = bm.numpy()[np.asarray(idx) // 128].sum(axis=1) * 128.0
+    report("block_sparse", t_lin, attn_cost_fit(O, q[idx], kf, vf, idx, 1 / math.sqrt(d), bm=bm), kk, H, N,
+           O.attn_flops(kk, N, H, d, keys))
+    for v in out.values():
+        v.setdefault("sample", "O(N) stages over all tokens; attention cost per (row, head) fitted once per config "
+                               "from 32, 128 and 512 sampled rows of head 0 (median of 3 timings each) and "
+                               "extrapolated to all rows and heads")
+    return out
+
+
+# ------------------------------------------------------------- reference ------
+def reference_arm(a, rank, world):
+    """The reference arm is the fp64 CPU oracle (the pages ship no code), timed
+    on the host cores on the headline workload, metric and unit. Every step is
+    one proportional slice of the HSA step (OracleHsaSlice: r sampled active
+    rows of one head plus the same share of every O(N) stage); the line reports
+    the slices' own measured time and the attention FLOPs they perform. Under
+    torchrun only rank 0 runs."""
+    if rank != 0:
+        return 0
+    rows = 256
+    o = OracleHsaSlice()
+    for _ in range(a.warmup):
+        o.slice(rows)
+    times = [o.slice(rows) for _ in range(a.steps)]
+    per_step = float(np.mean(times))
+    value = o.flops_per_row * rows / per_step / 1e12
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(per_step * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": hsa_config(world),
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": o.threads, "kind": "oracle",
+                             "sample": "each step: " + o.describe(rows)},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ main ------
+def roofline_block(flops, attn_ms, peak, peak_kind, traffic, kernel):
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": traffic, "kernel": kernel,
+            "flops_per_launch": flops, "avg_launch_ms": round(attn_ms, 4)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--attn", choices=["tc", "mma"], default="tc", help="attention kernel (mma = legacy baseline)")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-mid", action="store_true", help="skip the mid step")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple", "renoise"], default=None,
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h4"], default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
                     help="run each HSA-size stage kernel once, print its table and exit (for counter captures)")
@@ -747,52 +1090,52 @@ def main():
         tps.tps_check()
         print(json.dumps(res["stages_hsa"]), flush=True)
         return 0
-    st = MidStep(rank_seed_offset(rank), dev, a.attn)
+    pk, pk_kind = peaks()
     flush = L2Flush(dev)
-    st.step()                     # first eager step: one-time setup (status word, occupancy queries)
-    torch.cuda.synchronize()
-    if not a.no_graph:
-        st.capture_graphs()
-    for _ in range(a.warmup):
-        st.step()
-    torch.cuda.synchronize()
-    tps.tps_check()
-    # correctness guard on the timed configuration: the active count
-    assert int(st.cnt.item()) == st.k
 
+    # ---- headline: the HSA step ------------------------------------------------------
+    st = HsaStep(rank_seed_offset(rank), dev, a.attn)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    step_ms, attn_ms = timed_steps(st.step, a.steps, flush, with_attn=True)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    total_ms, attn_avg = run_path(st, a.steps, a.warmup, world, not a.no_graph, flush, dev)
     clocks = sampler.stop()
-    tps.tps_check()
-
-    total_ms, attn_avg = max_over_ranks([np.sum(step_ms), np.mean(attn_ms)], world, dev)
     ms_per_step = total_ms / a.steps
     value = job_throughput(st.flops, world, a.steps, total_ms) / 1e12
-    tok_s = job_throughput(st.k, world, a.steps, total_ms)
+    tok_s = job_throughput(st.units, world, a.steps, total_ms)
+    kernel = "pruned_attn" if a.attn == "tc" else "pruned_attn_mma"
+    roofline = roofline_block(st.flops, attn_avg, float(pk["bf16_tflops_sustained"]),
+                              f"bf16 dense sustained ({pk_kind}; the launch runs ~{attn_avg:.0f} ms inside a long "
+                              f"step)", recorded_traffic("pruned_attn_hsa.json") if a.attn == "tc" else None, kernel)
+    roofline["frac_of_burst"] = round(roofline["achieved"] / float(pk["bf16_tflops"]), 4)
+    e2e = None if a.no_e2e else e2e_leg(st, dev, max(3, min(a.steps, 20)), world)
+    graphs = bool(getattr(st, "graphs", False))
+    del st
+    torch.cuda.empty_cache()
 
-    # ---- end to end through the public API: pinned host inputs -> result on host
-    e2e = None if a.no_e2e else e2e_leg(st, dev, max(3, min(a.steps, 50)), world)
+    # ---- extra: the mid step -----------------------------------------------------------
+    mid = None
+    if not a.no_mid:
+        ms = MidStep(rank_seed_offset(rank), dev, a.attn)
+        msteps = max(a.steps, 100)
+        m_total, m_attn = run_path(ms, msteps, a.warmup, world, not a.no_graph, flush, dev)
+        mid = {"workload": "mid: 13x30x52 = 20280 tokens, 12 heads, d=128, inter-frame rel-L1 score, top-k 30% = "
+                           "6084 active queries x 20280 keys; step = score+select+gather+kv_sync+pruned_attn+"
+                           "scatter_out",
+               "steps": msteps, "ms_per_step": round(m_total / msteps, 4),
+               "value": round(job_throughput(ms.flops, world, msteps, m_total) / 1e12, 2), "unit": "TFLOP/s",
+               "active_tokens_per_s": round(job_throughput(ms.units, world, msteps, m_total), 1),
+               "roofline": roofline_block(ms.flops, m_attn, float(pk["bf16_tflops"]), f"bf16 dense burst ({pk_kind})",
+                                          recorded_traffic("pruned_attn_mid.json") if a.attn == "tc" else None,
+                                          kernel)}
+        if not a.no_e2e:
+            mid["e2e"] = e2e_leg(ms, dev, max(3, min(msteps, 50)), world)
+        del ms
+        torch.cuda.empty_cache()
 
-    sweep = None if a.no_sweep else keep_sweep(dev, a.attn)
-    pk, pk_kind = peaks()
-    achieved = st.flops / (attn_avg * 1e-3) / 1e12
-    peak = float(pk["bf16_tflops"])
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "peak_kind": f"bf16 dense burst ({pk_kind})",
-                "traffic": recorded_traffic("pruned_attn_mid.json") if a.attn == "tc" else None,
-                "kernel": "pruned_attn" if a.attn == "tc" else "pruned_attn_mma",
-                "flops_per_launch": st.flops, "avg_launch_ms": round(attn_avg, 4)}
-
-    configs = None if (a.no_configs or world > 1) else config_sweep(dev, peak, float(pk["hbm_gbs"]))
+    sweep = None if (a.no_sweep or world > 1) else keep_sweep(dev, a.attn)
+    configs = None if (a.no_configs or world > 1) else config_sweep(dev, float(pk["bf16_tflops"]),
+                                                                   float(pk["hbm_gbs"]))
     cpu = cpu_configs = None
     if rank == 0 and world == 1 and not a.no_cpu:
         cpu = oracle_baseline()
@@ -807,209 +1150,15 @@ def main():
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded latent video: static background + jitter, moving objects, pan strip)",
-        "config": {"workload": "mid: 13x30x52 = 20280 tokens, 12 heads, d=128, inter-frame rel-L1 score, "
-                               "top-k 30% = 6084 active queries x 20280 keys; step = score+select+gather+"
-                               "kv_sync+pruned_attn+scatter_out",
-                   "N": st.N, "active": st.k, "heads": st.H, "head_dim": st.d,
-                   "l2": "flushed between timed steps (512 MiB write, then 512 MiB read: L2 left clean)",
-                   "parallelism": f"replicas x{world}",
-                   "attn_kernel": roofline["kernel"],
-                   "cuda_graphs": bool(getattr(st, "graphs", False))},
+        "data": "synthetic (seeded velocity pair of a latent video: static background + jitter, moving objects, "
+                "pan strip; step delta N(0,0.05) on background, N(0,1) on moving tokens)",
+        "config": hsa_config(world),
+        "impl_details": {"attn_kernel": kernel, "cuda_graphs": graphs},
         "active_tokens_per_s": round(tok_s, 1),
-        "gpu_launches": st.launches * a.steps,
+        "gpu_launches": sum(HsaStep.LAUNCHES.values()) * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
-        "keep_sweep_wan": sweep, "configs": configs, "cpu_baseline_configs": cpu_configs,
+        "mid": mid, "keep_sweep_wan": sweep, "configs": configs, "cpu_baseline_configs": cpu_configs,
     }
-    print(json.dumps(line), flush=True)
-    return 0
-
-
-def e2e_leg(st, dev, steps, world):
-    """Same metric through the C ABI with the step's data in pinned host memory.
-
-    When the library's kernels can address pinned host memory (unified
-    addressing; checked with tps_pointer_is_device_accessible), the gathers read
-    only the active rows of Q/K/V straight from host memory and scatter_out
-    writes only the active rows of the caller's host-side output, so each step
-    moves the latents plus 3 x |A| rows in and |A| rows out over PCIe. The next
-    step's host-side work (latent copy, score, select, gathers) runs on a second
-    stream beside this step's kv_sync, attention and scatter. Otherwise the
-    copy-based leg below runs."""
-    tps = st.tps
-    host = {k: v.pin_memory() for k, v in st.host.items()}
-    o_host = torch.zeros_like(st.o_full, device="cpu").pin_memory()   # cached outputs: zeros, as on the device
-    if not all(tps.pointer_is_device_accessible(t) for t in (host["q"], host["k"], host["v"], o_host)):
-        return e2e_leg_copies(st, dev, steps, world)
-    R = st.H * st.d * 2
-    h2d = host["x"].numel() * host["x"].element_size() + 3 * st.k * R
-    d2h = st.k * R
-    shp = (st.k, st.H, st.d)
-
-    def new_set():
-        z = lambda dt=torch.bfloat16: torch.empty(shp, dtype=dt, device=dev)    # noqa: E731
-        return {"x": torch.empty_like(st.x), "score": torch.empty_like(st.score), "idx": torch.empty_like(st.idx),
-                "cnt": torch.empty_like(st.cnt), "ws": torch.empty_like(st.ws), "q": z(), "k": z(), "v": z(),
-                "o": z()}
-    sets = [new_set(), new_set()]
-    comp = torch.cuda.current_stream()
-    s_pre = torch.cuda.Stream()
-    pre_done = [torch.cuda.Event(), torch.cuda.Event()]
-    main_done = [torch.cuda.Event(), torch.cuda.Event()]
-    for e in main_done:
-        e.record(comp)
-
-    def pre(i):
-        b = i & 1
-        X = sets[b]
-        with torch.cuda.stream(s_pre):
-            s_pre.wait_event(main_done[b])
-            X["x"].copy_(host["x"], non_blocking=True)
-            tps.lipar_score(X["x"], out=X["score"])
-            tps.lipar_select(X["score"], tps.SELECT_TOPK, k=st.k, idx=X["idx"], count=X["cnt"], ws=X["ws"])
-            for key in ("q", "k", "v"):
-                tps.tps_gather_rows(X[key], host[key], X["idx"], X["cnt"])    # rows read over PCIe
-            pre_done[b].record(s_pre)
-
-    def main(i):
-        b = i & 1
-        X = sets[b]
-        comp.wait_event(pre_done[b])
-        tps.kv_sync(st.kc, st.vc, X["k"], X["v"], X["idx"], X["cnt"])
-        st.attn_fn(X["q"], st.kc, st.vc, X["idx"], X["cnt"], st.scale, o_act=X["o"])
-        tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])                    # rows written over PCIe
-        main_done[b].record(comp)
-
-    def run(n):
-        pre(0)
-        for i in range(n):
-            if i + 1 < n:
-                pre(i + 1)
-            main(i)
-
-    run(2)
-    torch.cuda.synchronize()
-    tps.tps_check()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(comp)
-    s_pre.wait_event(a)
-    run(steps)
-    b.record(comp)
-    torch.cuda.synchronize()
-    tps.tps_check()
-    ms = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
-    # the host-side output must equal the device-resident path's (same inputs, same kernels)
-    st.step()
-    torch.cuda.synchronize()
-    if not torch.equal(o_host, st.o_full.cpu()):
-        raise RuntimeError("e2e: host-side output differs from the device-resident step")
-    return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": round(ms / steps, 4),
-            "mode": "pinned host data; gathers read and scatter_out writes only the active rows over PCIe; "
-                    "step i+1's latent copy, score, select and gathers overlap step i's attention"}
-
-
-def e2e_leg_copies(st, dev, steps, world):
-    """Same metric through the C ABI with host buffers: each step copies the
-    step's inputs (latents + Q/K/V projections) from pinned host memory and
-    reads the full output back; copies are inside the timed region.
-
-    The copies overlap the computation on separate streams, as a serving loop
-    would run them: step i+1's inputs stream in (into the second of two device
-    input sets) while step i computes, and step i's output is copied to a
-    device staging buffer and read back while step i+1 runs."""
-    host_in = {k: v.pin_memory() for k, v in st.host.items()}
-    host_out = [torch.empty((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = host_out[0].numel() * host_out[0].element_size()
-    sets = [(st.x, st.q, st.kf, st.vf),
-            tuple(torch.empty_like(t) for t in (st.x, st.q, st.kf, st.vf))]
-    stage = [torch.empty_like(st.o_full) for _ in range(2)]
-    comp = torch.cuda.current_stream()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()            # noqa: E731
-    in_ready, in_free = [ev(), ev()], [ev(), ev()]
-    out_ready, out_free = [ev(), ev()], [ev(), ev()]
-    for e in in_free + out_free:
-        e.record(comp)
-
-    def copy_in(i):
-        b = i & 1
-        with torch.cuda.stream(s_in):
-            s_in.wait_event(in_free[b])
-            for dst, key in zip(sets[b], ("x", "q", "k", "v")):
-                dst.copy_(host_in[key], non_blocking=True)
-            in_ready[b].record(s_in)
-
-    def run(n):
-        copy_in(0)
-        for i in range(n):
-            b = i & 1
-            if i + 1 < n:
-                copy_in(i + 1)
-            comp.wait_event(in_ready[b])
-            st._pre(sets[b])
-            in_free[b].record(comp)
-            st.attn_fn(st.q_act, st.kc, st.vc, st.idx, st.cnt, st.scale, o_act=st.o_act)
-            st._post()
-            comp.wait_event(out_free[b])
-            stage[b].copy_(st.o_full, non_blocking=True)
-            out_ready[b].record(comp)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(out_ready[b])
-                host_out[b].copy_(stage[b], non_blocking=True)
-                out_free[b].record(s_out)
-        comp.wait_stream(s_out)
-
-    run(2)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(comp)
-    s_in.wait_event(a)
-    run(steps)
-    b.record(comp)
-    torch.cuda.synchronize()
-    ms = max_over_ranks([a.elapsed_time(b)], world, dev)[0]
-    return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": round(ms / steps, 4),
-            "overlap": "H2D of step i+1 and D2H of step i-1 run beside step i on two copy streams"}
-
-
-def reference_arm(a, rank, world):
-    """The reference arm is the fp64 CPU oracle (the pages ship no code), timed
-    on the host cores on the same workload and metric. Each step is a bounded
-    sample: attention for 16 sampled active rows x all heads; the O(N) stages
-    (score, select, gather, kv_sync, scatter) are re-timed every 16th step and
-    their latest time is added to every step. Under torchrun only rank 0 runs."""
-    if rank != 0:
-        return 0
-    rows = 16
-    o = OracleStep()
-    t_lin = o.linear()
-    o.fit()
-    times, spent = [], t_lin
-    for i in range(a.warmup + a.steps):
-        if i % 16 == 0 and i:
-            t_lin = o.linear()
-            spent += t_lin
-        t_att = o.attn(rows)
-        spent += t_att
-        if i >= a.warmup:
-            times.append(o.full_step(t_lin, t_att, rows))
-    per_step = float(np.mean(times))
-    value = o.flops / per_step / 1e12
-    line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
-            "warmup": a.warmup, "ms_per_step": round(per_step * 1e3, 2), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": "mid: 13x30x52 = 20280 tokens, 12 heads, d=128, inter-frame rel-L1 score, "
-                                   "top-k 30% = 6084 active queries x 20280 keys; step = score+select+gather+"
-                                   "kv_sync+pruned_attn+scatter_out (fp64 CPU oracle)"},
-            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": o.threads, "kind": "oracle",
-                             "sample": o.describe(rows), "seconds_spent": round(spent, 2)},
-            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 

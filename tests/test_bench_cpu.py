@@ -38,7 +38,8 @@ def test_reference_line_carries_the_contract_keys(ref_line):
     assert d["n_gpus"] == 1 and d["steps"] == 2
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["dtype"] == "f64" and d["data"] == "synthetic"
-    assert "mid" in d["config"]["workload"]
+    assert d["config"] == bench.hsa_config(1)          # the GPU arm prints this same dict
+    assert "HSA step" in d["config"]["workload"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e2e = d["e2e"]
