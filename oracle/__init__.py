@@ -11,8 +11,10 @@ Parity status per function (see each docstring for the pins):
   lipar_score, select_threshold, select_topk, group_split, schedule_active,
   kv_sync, pruned_attn, scatter_out  -- pinned by tests/test_oracle_pins.py
   euler_update, lse_merge, lipar_score_motion,
-  timeripple_delta/_reuse/_token_score/_theta -- pinned likewise (hand-worked
-                                         fixtures, closed forms, invariants)
+  timeripple_delta/_reuse/_token_score/_theta,
+  rope_rotate, kv_rerotate             -- pinned likewise (hand-worked
+                                         fixtures, closed forms, invariants,
+                                         complex-number form)
   philox4x32_10 raw stream            -- pinned by the published
                                          known-answer vectors (Salmon et al.,
                                          SC'11), and its normals statistically.

@@ -40,6 +40,7 @@ __all__ = [
     "philox_words", "renoise_normals", "pruned_attn", "scatter_out", "gather_rows",
     "attn_flops", "euler_update", "lse_merge", "lipar_score_motion",
     "timeripple_delta", "timeripple_reuse", "timeripple_token_score", "timeripple_theta",
+    "rope_rotate", "kv_rerotate",
 ]
 
 
@@ -469,3 +470,52 @@ def timeripple_theta(step: int, theta_lo: float, theta_hi: float, i0: int = 11, 
     if step >= i1:
         return float(theta_hi)
     return float(theta_lo) + (float(theta_hi) - float(theta_lo)) * (step - i0) / float(i1 - i0)
+
+
+# ---------------------------------------------------------------------------
+# Attention recovery: re-rotation of keys duplicated across frames
+# ---------------------------------------------------------------------------
+def rope_rotate(k, dims, shift, base: float = 10000.0) -> np.ndarray:
+    """Rotary position offset of keys ([LIPAR] 2.C, Dutch summary: the K/V of a
+    pruned token are approximated from the previous frame's cache, taking the
+    RoPE rotations into account; [TR] Metodologia 1: the rotary channels of a
+    head form temporal, x and y groups).
+
+    Reading: a head's d channels are the contiguous groups [t | x | y] of
+    sizes dims = (d_t, d_x, d_y) (all even, summing to d). Inside group a
+    (channel offset o_a, size d_a) the adjacent channels (o_a + 2j,
+    o_a + 2j + 1) form pair j with frequency theta = base^(-2j / d_a); a
+    position offset shift = (s_t, s_x, s_y) rotates that pair by phi = s_a *
+    theta:  (x, y) -> (x cos phi - y sin phi, x sin phi + y cos phi).
+    k is [..., d] (bf16 tensor or array); returns float64 of the same shape.
+    Pinned by a hand-worked example (tests/golden/rope_worked.json), the
+    complex-number form z * exp(i phi) (numpy), composition of offsets, norm
+    preservation, relative-offset invariance of q . k, and planted slips."""
+    x = f64(k)
+    out = x.copy()
+    o = 0
+    for a in range(3):
+        da = int(dims[a])
+        j = np.arange(da // 2)
+        phi = float(shift[a]) * base ** (-2.0 * j / da)
+        c, s = np.cos(phi), np.sin(phi)
+        ev, od = x[..., o + 2 * j], x[..., o + 2 * j + 1]
+        out[..., o + 2 * j] = ev * c - od * s
+        out[..., o + 2 * j + 1] = ev * s + od * c
+        o += da
+    return out
+
+
+def kv_rerotate(k_cache, idx, dims, shift, base: float = 10000.0) -> np.ndarray:
+    """K_eff for attention when pruned tokens reuse cached keys of the previous
+    frame ([LIPAR] 2.C): the row of an active token (in idx) is its cache row
+    (already the fresh key after kv_sync); the row of a pruned token is its
+    cache row moved to the token's own position, rope_rotate(row, shift) --
+    the configured reading is shift = (1, 0, 0), one frame later. k_cache is
+    [N, H, d]; returns float64 [N, H, d]."""
+    out = f64(k_cache)
+    N = out.shape[0]
+    pruned = np.setdiff1d(np.arange(N), np.asarray(idx, np.int64))
+    if len(pruned):
+        out[pruned] = rope_rotate(out[pruned], dims, shift, base)
+    return out

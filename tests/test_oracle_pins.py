@@ -551,3 +551,97 @@ def test_philox_known_answer_vectors():
         out = O.philox4x32_10(*c, k[0], k[1])
         got = [int(np.asarray(o).reshape(-1)[0]) for o in out]
         assert got == [int(v, 16) for v in case["out"]]
+
+
+# ------------------------------------------------- RoPE re-rotation ([LIPAR] 2.C) ---
+def test_rope_worked_examples():
+    for c in _gold("rope_worked.json")["cases"]:
+        got = O.rope_rotate(np.array(c["k"], float), c["dims"], c["shift"], c["base"])
+        np.testing.assert_allclose(got, np.array(c["out"], float), rtol=0, atol=1e-15)
+
+
+def _rope_complex(k, dims, shift, base=10000.0):
+    """The same offset as complex multiplication: pair (x, y) is z = x + iy and
+    moves to z * exp(i phi) (numpy's complex arithmetic)."""
+    x = np.asarray(k, float)
+    out = x.copy()
+    o = 0
+    for a, da in enumerate(dims):
+        j = np.arange(da // 2)
+        z = x[..., o + 2 * j] + 1j * x[..., o + 2 * j + 1]
+        z = z * np.exp(1j * shift[a] * base ** (-2.0 * j / da))
+        out[..., o + 2 * j], out[..., o + 2 * j + 1] = z.real, z.imag
+        o += da
+    return out
+
+
+def test_rope_complex_form_composition_norm_and_relative_offset():
+    dims = synth.rope_dims(128)
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((64, 3, 128))
+    q = rng.standard_normal((64, 3, 128))
+    s1, s2 = (1, -2, 3), (4, 5, -1)
+    r1 = O.rope_rotate(k, dims, s1)
+    np.testing.assert_allclose(r1, _rope_complex(k, dims, s1), rtol=0, atol=1e-12)
+    # R(a) R(b) = R(a + b)
+    np.testing.assert_allclose(O.rope_rotate(r1, dims, s2), O.rope_rotate(k, dims, np.add(s1, s2)),
+                               rtol=0, atol=1e-12)
+    # every pair keeps its length
+    pn = lambda x: np.hypot(x[..., 0::2], x[..., 1::2])                 # noqa: E731
+    np.testing.assert_allclose(pn(r1), pn(k), rtol=1e-13)
+    # (R(p) q) . (R(p + delta) k) depends on the offset delta only
+    ref = np.sum(q * O.rope_rotate(k, dims, (1, 0, 0)), axis=-1)
+    for p in ((0, 0, 0), (5, 0, 0), (-7, 3, 2)):
+        got = np.sum(O.rope_rotate(q, dims, p) * O.rope_rotate(k, dims, np.add(p, (1, 0, 0))), axis=-1)
+        np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-10)
+    # no offset is the identity, bit for bit
+    assert np.array_equal(O.rope_rotate(k, dims, (0, 0, 0)), k)
+
+
+def test_kv_rerotate_rows():
+    kc = synth.gaussian_bf16((40, 2, 64), 71)
+    idx = np.array([0, 3, 4, 17, 39])
+    dims = synth.rope_dims(64)
+    ke = O.kv_rerotate(kc, idx, dims, (1, 0, 0))
+    np.testing.assert_array_equal(ke[idx], kc[idx].double().numpy())      # active rows: the cache row
+    pruned = np.setdiff1d(np.arange(40), idx)
+    np.testing.assert_array_equal(ke[pruned], O.rope_rotate(kc[pruned], dims, (1, 0, 0)))
+    assert not np.allclose(ke[pruned], kc[pruned].double().numpy())
+    np.testing.assert_array_equal(O.kv_rerotate(kc, idx, dims, (0, 0, 0)), kc.double().numpy())
+
+
+def _rope_variant(kind):
+    """The oracle's rotation with one plausible slip planted."""
+    def fn(k, dims, shift, base=10000.0):
+        x = np.asarray(k, float)
+        out = x.copy()
+        o = 0
+        order = (1, 2, 0) if kind == "groups_rotated" else (0, 1, 2)
+        for a in order:
+            da = int(dims[a])
+            j = np.arange(da // 2)
+            denom = x.shape[-1] if kind == "freq_over_d" else da
+            phi = float(shift[a]) * base ** (-2.0 * j / denom) * (-1.0 if kind == "sign" else 1.0)
+            if kind == "half_split":                   # pairs (j, j + d_a/2) instead of adjacent channels
+                i0, i1 = o + j, o + da // 2 + j
+            else:
+                i0, i1 = o + 2 * j, o + 2 * j + 1
+            c, s = np.cos(phi), np.sin(phi)
+            out[..., i0] = x[..., i0] * c - x[..., i1] * s
+            out[..., i1] = x[..., i0] * s + x[..., i1] * c
+            o += da
+        return out
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["sign", "half_split", "freq_over_d", "groups_rotated"])
+def test_rope_pins_catch_planted_mistakes(kind):
+    """Composition, norm and relative-offset pins hold for any consistent
+    rotation; the hand-worked examples fix the sign, the pairing, the
+    frequencies and the group order."""
+    def worked_ok(fn):
+        return all(np.allclose(fn(np.array(c["k"], float), c["dims"], c["shift"], c["base"]),
+                               np.array(c["out"], float), rtol=0, atol=1e-12)
+                   for c in _gold("rope_worked.json")["cases"])
+    assert worked_ok(_rope_variant("none"))
+    assert not worked_ok(_rope_variant(kind))

@@ -37,7 +37,7 @@ import torch
 __all__ = [
     "VideoSpec", "CONFIGS", "latent_video", "velocity_pair", "projection_weights",
     "project", "to_bf16", "random_scores", "block_mask_band_random", "gaussian_bf16",
-    "timeripple_windows", "TR_THETA",
+    "timeripple_windows", "TR_THETA", "rope_dims",
 ]
 
 
@@ -106,6 +106,14 @@ def timeripple_windows(d: int):
     g = 2 * (d // 6)
     dt = d - 2 * g
     return ((dt, 2 * g), (dt + g, dt + g), (0, dt + g))
+
+
+def rope_dims(d: int):
+    """Channel counts (t, x, y) of a head's rotary groups, contiguous in that
+    order: (d - 4*(d//6), 2*(d//6), 2*(d//6)), each even (the same split as the
+    Timeripple windows above). Configuration, not arithmetic."""
+    g = 2 * (d // 6)
+    return (d - 2 * g, g, g)
 
 
 # Threshold schedule of the per-axis checks (t, x, y): theta rises from 0 at
