@@ -669,6 +669,10 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     o_full, o_act = rnd(N, H, d), rnd(A, H, d)
     t = timer(lambda: tps.scatter_out(o_full, o_act, idx, cnt), flush)
     stages["scatter_out"] = (t, 2 * R * A)
+    # keys of the pruned rows turned one frame forward (RoPE re-rotation), active rows copied
+    rope_dims = synth.rope_dims(d)
+    t = timer(lambda: tps.kv_rerotate(kc, idx, cnt, rope_dims, (1, 0, 0), k_eff=ke), flush)
+    stages["kv_rerotate"] = (t, 2 * R * N + 4 * A)
     # attention-recovery merge of two partial results for the A active rows
     lse_a, lse_b, lse_o = (torch.randn(A, H, generator=g, device=dev) for _ in range(3))
     o_b = rnd(A, H, d)

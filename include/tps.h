@@ -8,6 +8,7 @@
  *   lipar_group / lipar_schedule -> HSA step groups and per-step active list
  *   tps_gather_rows -> the active tokens' rows (input of the QKV projection)
  *   kv_sync       -> fresh K/V rows into the layer cache (+ noise-aware re-noise)
+ *   kv_rerotate   -> cached keys of pruned tokens turned to their own RoPE position
  *   pruned_attn   -> active queries attend all N cached keys (optional key-block mask)
  *   scatter_out   -> active outputs written back over the cached outputs
  *
@@ -219,6 +220,36 @@ TPS_API int kv_sync(tps_bf16* k_cache, tps_bf16* v_cache, const tps_bf16* k_fres
             const tps_bf16* v_fresh, const int32_t* idx, const int32_t* count, int64_t cap,
             int64_t N, int H, int d, const tps_renoise* rn /* HOST, may be NULL */,
             tps_bf16* k_eff, tps_bf16* v_eff, tps_stream stream);
+
+/* ---- attention recovery: keys reused across frames ([LIPAR] 2.C) -----------
+ * "Training-free Latent Inter-Frame Pruning with Attention Recovery", Dutch
+ * summary 2.C: the K/V of pruned tokens are approximated by the cached K/V of
+ * the previous frame, taking the RoPE rotations into account; "Timeripple",
+ * Metodologia 1: a head's rotary channels form temporal, x and y groups.
+ * Writes k_eff [N, H, d] (bf16, may alias k_cache) from k_cache [N, H, d]:
+ *   active rows n = idx[j], j < min(*count, cap): k_eff[n] = k_cache[n] (bit
+ *     copy: after kv_sync these hold the fresh keys);
+ *   every other row: k_cache[n] turned to its own position. Per head, the
+ *     channels are the contiguous groups [t | x | y] of dims[0], dims[1],
+ *     dims[2] channels (each even, summing to d); in group a the adjacent
+ *     channels (o_a + 2j, o_a + 2j + 1) are rotated by
+ *     phi = shift[a] * base^(-2j / dims[a]):
+ *       (x, y) -> (x cos phi - y sin phi, x sin phi + y cos phi),
+ *     computed in fp32 from an fp32 (cos, sin) table rounded from double
+ *     precision, then rounded to bf16 (RNE).
+ * A key cached at frame f-1 for the token at frame f takes shift = (1, 0, 0).
+ * V needs no rotation (RoPE acts on Q and K only). idx must be ascending;
+ * entries outside [0, N) or out of order raise TPS_ERR_BOUNDS at tps_check.
+ * d in {64, 128}; H*d <= 16384; |shift[a]| <= 2^20; rope is a HOST pointer. */
+typedef struct tps_rope {
+  int32_t dims[3];   /* channels of the t, x and y rotary groups        */
+  int32_t shift[3];  /* position offset: frames, columns, rows           */
+  float   base;      /* frequency base (10000 in common video DiTs)      */
+  int32_t pad_;
+} tps_rope;
+
+TPS_API int kv_rerotate(const tps_bf16* k_cache, const int32_t* idx, const int32_t* count, int64_t cap,
+                        int64_t N, int H, int d, const tps_rope* rope, tps_bf16* k_eff, tps_stream stream);
 
 /* ---- step 5: pruned attention ([HSA] 2.2 (3)-(4); [SVOO] part 2; [TR]) ------
  * For every active row j < min(*count, cap) and head h:

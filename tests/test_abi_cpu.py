@@ -138,3 +138,22 @@ def test_workspace_min_size_is_a_lower_bound():
     F = C.c_void_p(0x1000)
     need = tps.workspace_min_size(tps.OP_SELECT, 100000)
     assert tps.lib().lipar_select(F, 100000, tps.SELECT_TOPK, 0.0, 5, F, F, F, need - 1, NULL) == tps.WORKSPACE
+
+
+def test_rerotate_validation():
+    l = tps.lib()
+    P = lambda r: C.cast(C.byref(r), C.c_void_p)               # noqa: E731
+    good = tps.Rope((C.c_int32 * 3)(24, 20, 20), (C.c_int32 * 3)(1, 0, 0), 10000.0, 0)
+    odd = tps.Rope((C.c_int32 * 3)(23, 21, 20), (C.c_int32 * 3)(1, 0, 0), 10000.0, 0)
+    short = tps.Rope((C.c_int32 * 3)(24, 20, 18), (C.c_int32 * 3)(1, 0, 0), 10000.0, 0)
+    far = tps.Rope((C.c_int32 * 3)(24, 20, 20), (C.c_int32 * 3)((1 << 20) + 1, 0, 0), 10000.0, 0)
+    nobase = tps.Rope((C.c_int32 * 3)(24, 20, 20), (C.c_int32 * 3)(1, 0, 0), 0.0, 0)
+    assert _err(l.kv_rerotate(F, F, F, 10, 100, 2, 64, P(odd), F, NULL))[0] == tps.INVALID_ARG
+    code, msg = _err(l.kv_rerotate(F, F, F, 10, 100, 2, 64, P(short), F, NULL))
+    assert code == tps.INVALID_ARG and "sum to 62" in msg
+    assert l.kv_rerotate(F, F, F, 10, 100, 2, 64, P(far), F, NULL) == tps.INVALID_ARG
+    assert l.kv_rerotate(F, F, F, 10, 100, 2, 64, P(nobase), F, NULL) == tps.INVALID_ARG
+    assert l.kv_rerotate(F, F, F, 10, 100, 2, 64, NULL, F, NULL) == tps.INVALID_ARG
+    assert l.kv_rerotate(F, F, F, 10, 100, 2, 96, P(good), F, NULL) == tps.INVALID_ARG
+    assert l.kv_rerotate(MIS, F, F, 10, 100, 2, 64, P(good), F, NULL) == tps.ALIGN
+    assert l.kv_rerotate(F, F, F, 10, 0, 2, 64, P(good), F, NULL) == tps.SHAPE

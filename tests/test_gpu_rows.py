@@ -201,3 +201,52 @@ def test_philox_known_answer_vectors_on_gpu():
         words = tps.tps_philox_fill(c[0] | (c[1] << 32), 1, k[0] | (k[1] << 32), c[2], c[3])
         got = words.cpu().numpy().view(np.uint32).tolist()
         assert got == [int(v, 16) for v in case["out"]]
+
+
+def _rope_tol(ref, src):
+    # one bf16 rounding of the result (one ulp of slack) plus the fp32 table and
+    # arithmetic (a few 2^-24 relative of the pair's magnitude)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+    pair = np.abs(src).reshape(*src.shape[:-1], -1, 2).sum(-1).repeat(2, axis=-1)
+    return ulp + 1e-6 * pair + 1e-30
+
+
+@pytest.mark.parametrize("N,H,d,A,shift,base", [(256, 2, 64, 100, (1, 0, 0), 10000.0),
+                                                (4099, 12, 128, 1500, (1, 0, 0), 10000.0),
+                                                (3001, 3, 128, 1000, (-3, 2, 5), 500.0),
+                                                (517, 24, 128, 0, (2, -1, 0), 10000.0),
+                                                (777, 4, 64, 777, (1, 0, 0), 10000.0)])
+def test_kv_rerotate_parity(N, H, d, A, shift, base):
+    kc, _, _, _, idx = _case(N, H, d, A, 7 * N + A)
+    dims = synth.rope_dims(d)
+    di, dc = _dev_idx(idx)
+    ke = tps.kv_rerotate(kc.to(DEV), di, dc, dims, shift, base, cap=max(A, 1)).cpu()
+    ref = O.kv_rerotate(kc, idx, dims, shift, base)
+    assert torch.equal(ke[torch.from_numpy(idx).long()], kc[torch.from_numpy(idx).long()])   # active: bit copies
+    pruned = np.setdiff1d(np.arange(N), idx)
+    got = ke[torch.from_numpy(pruned)].double().numpy()
+    err = np.abs(got - ref[pruned])
+    assert np.all(err <= _rope_tol(ref[pruned], kc[torch.from_numpy(pruned)].double().numpy()))
+    tps.tps_check()
+
+
+def test_kv_rerotate_zero_shift_in_place_and_full_size():
+    # no offset: every row is copied bit for bit (cos 0 = 1, sin 0 = 0), here in place
+    kc, _, _, _, idx = _case(1000, 3, 128, 400, 91)
+    kcd = kc.to(DEV)
+    di, dc = _dev_idx(idx)
+    tps.kv_rerotate(kcd, di, dc, synth.rope_dims(128), (0, 0, 0), k_eff=kcd)
+    assert torch.equal(kcd.cpu(), kc)
+    # the HSA size with the step's schedule-like list: sampled rows against the oracle
+    cfg = synth.CONFIGS["hsa"]
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    kc = synth.gaussian_bf16((N, H, d), 92)
+    idx = np.arange(0, N, 3, dtype=np.int32)
+    di, dc = _dev_idx(idx)
+    dims = synth.rope_dims(d)
+    ke = tps.kv_rerotate(kc.to(DEV), di, dc, dims, (1, 0, 0)).cpu()
+    rows = np.sort(np.random.default_rng(93).choice(N, 3000, replace=False))
+    ref = O.kv_rerotate(kc[torch.from_numpy(rows)], np.flatnonzero(rows % 3 == 0), dims, (1, 0, 0))
+    got = ke[torch.from_numpy(rows)].double().numpy()
+    assert np.all(np.abs(got - ref) <= _rope_tol(ref, kc[torch.from_numpy(rows)].double().numpy()))
+    tps.tps_check()

@@ -33,6 +33,7 @@ SIGNATURES = {
     "lipar_schedule": (_INT, [_P, _I64, _INT, _P, _INT, _INT, _INT, _P, _P, _P, C.c_size_t, _P]),
     "tps_gather_rows": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "kv_sync": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P, _P, _P]),
+    "kv_rerotate": (_INT, [_P, _P, _P, _I64, _I64, _INT, _INT, _P, _P, _P]),
     "pruned_attn": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "pruned_attn_ws": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P,
                               C.c_size_t, _P]),
@@ -200,6 +201,23 @@ def kv_sync(k_cache, v_cache, k_fresh, v_fresh, idx, count, cap=None, renoise=No
                        cap, N, H, d, None if rn is None else C.cast(C.byref(rn), _P), _ptr(k_eff), _ptr(v_eff),
                        _stream(stream)))
     return k_eff, v_eff
+
+
+class Rope(C.Structure):
+    """tps_rope: rotary groups (t, x, y), the offset given to pruned rows, base."""
+    _fields_ = [("dims", C.c_int32 * 3), ("shift", C.c_int32 * 3), ("base", C.c_float), ("pad_", C.c_int32)]
+
+
+def kv_rerotate(k_cache, idx, count, dims, shift, base=10000.0, k_eff=None, cap=None, stream=None):
+    """k_eff [N, H, d]: active rows copied, pruned rows turned by `shift`."""
+    N, H, d = k_cache.shape
+    cap = idx.shape[0] if cap is None else cap
+    if k_eff is None:
+        k_eff = torch.empty_like(k_cache)
+    r = Rope((C.c_int32 * 3)(*[int(v) for v in dims]), (C.c_int32 * 3)(*[int(v) for v in shift]), float(base), 0)
+    _chk(lib().kv_rerotate(_ptr(k_cache), _ptr(idx), _ptr(count), cap, N, H, d, C.cast(C.byref(r), _P),
+                           _ptr(k_eff), _stream(stream)))
+    return k_eff
 
 
 def _attn(fn, q_act, k, v, idx, count, scale, blockmask, block, o_act, lse, cap, stream):
