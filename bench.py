@@ -593,20 +593,17 @@ def keep_sweep(dev, attn, reps=5):
                     "active_tokens_per_s": round(A / t * 1e3, 1), "attn_ws_ms": round(tw, 4),
                     "tflops_ws": round(fl / tw / 1e9, 1), "ws_bytes": nws})
     return out
-def executed_key_tiles(idx: np.ndarray, N: int, nb_mask=None, rows_per_cta=256):
-    """Key tiles the attention kernel runs per CTA (dense: all; masked: the
-    union of the mask rows of the query blocks a CTA spans)."""
+def executed_flops(idx: np.ndarray, N: int, H: int, d: int, nb_mask=None) -> float:
+    """FLOPs the attention kernel executes, padding rows and whole 128-key
+    tiles included. Dense: ceil(A/256) CTAs of two 128-row tiles, every key
+    tile. Masked: one 128-row tile per original query block holding an active
+    row, the key tiles that block keeps."""
     nkt = -(-N // 128)
     A = len(idx)
-    ctas = -(-A // rows_per_cta)
     if nb_mask is None:
-        return ctas * nkt, ctas
-    tot = 0
-    for c in range(ctas):
-        r0, r1 = c * rows_per_cta, min(A, (c + 1) * rows_per_cta) - 1
-        qb0, qb1 = idx[r0] // 128, idx[r1] // 128
-        tot += int(np.any(nb_mask[qb0:qb1 + 1] != 0, axis=0).sum())
-    return tot, ctas
+        return 4.0 * d * H * 256 * 128 * (-(-A // 256)) * nkt
+    blocks = np.unique(np.asarray(idx) // 128)
+    return 4.0 * d * H * 128 * 128 * float(nb_mask[blocks].astype(np.int64).sum())
 
 
 def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
@@ -714,8 +711,7 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
         o = torch.empty_like(q)
         t = timer(lambda: tps.pruned_attn(q, ke, ve, ii, cc, scale, o_act=o), flush, reps=3, warm=1)
         alg = 4.0 * d * H * Aq * N
-        tiles, ctas = executed_key_tiles(np.arange(Aq), N)
-        exe = 4.0 * d * H * 256 * 128 * tiles
+        exe = executed_flops(np.arange(Aq), N, H, d)
         att[name] = {"ms": round(t, 3), "tflops_alg": round(alg / t / 1e9, 1), "tflops_exec": round(exe / t / 1e9, 1),
                      "frac_peak_exec": round(exe / t / 1e9 / peak_tflops, 3)}
         del q, o
@@ -735,8 +731,7 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     bm_h = bm.numpy()
     alg = 4.0 * d * H * 128 * float(bm_h[bidx_h // 128].sum())
     alg -= 4.0 * d * H * float(np.sum(bm_h[bidx_h // 128][:, -1])) * (128 - (N - (bm_h.shape[0] - 1) * 128))
-    tiles, ctas = executed_key_tiles(bidx_h, N, bm_h)
-    exe = 4.0 * d * H * 256 * 128 * tiles
+    exe = executed_flops(bidx_h, N, H, d, bm_h)
     att["block_sparse"] = {"ms": round(t, 3), "tflops_alg": round(alg / t / 1e9, 1),
                            "tflops_exec": round(exe / t / 1e9, 1), "frac_peak_exec": round(exe / t / 1e9 / peak_tflops, 3),
                            "exec_over_alg": round(exe / alg, 2)}

@@ -119,6 +119,42 @@ def test_attn_blockmask(impl, N, A):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_blockmask_query_block_edges(impl, d):
+    """Masked mode runs one tile per original query block: full blocks (128
+    active rows), single-row and empty blocks, key lists of very different
+    lengths within one CTA (all blocks vs one), a block whose row keeps nothing,
+    an odd number of blocks (the last CTA has one tile), a running-max spike in
+    a kept tile, and a count below cap (rows past the count stay untouched)."""
+    N, H = 2000, 2                                          # nb = 16
+    rng = np.random.default_rng(40 + d)
+    sel = [np.arange(0, 128), np.array([130]), np.arange(384, 512), np.arange(512, 640, 3),
+           np.array([700, 701, 830]), np.arange(1920, 2000)]
+    idx = np.unique(np.concatenate(sel + [rng.choice(np.arange(896, 1900), 300, replace=False)]))
+    A = len(idx)
+    q = synth.gaussian_bf16((A, H, d), 41)
+    k = synth.gaussian_bf16((N, H, d), 42).double()
+    k[1000:1100] *= 20.0                                    # spike inside key block 7
+    k = k.to(torch.bfloat16)
+    v = synth.gaussian_bf16((N, H, d), 43)
+    nb = -(-N // 128)
+    bm = torch.from_numpy((rng.random((nb, nb)) < 0.3).astype(np.uint8))
+    bm[0] = 1                                               # block 0 keeps every key block
+    bm[1] = 0
+    bm[1, 15] = 1                                           # block 1 keeps only the ragged last one
+    bm[3] = 0                                               # block 3 keeps nothing
+    bm[:, 7] = 1
+    o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm)
+    _check(o, lse, o_ref, lse_ref)
+    c = A - 77
+    o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm, count=c)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm, rows=np.arange(c))
+    _check(o[:c], lse[:c], o_ref, lse_ref)
+    assert torch.all(o[c:].float() == 7.0) and np.all(lse[c:] == 7.0)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
 def test_attn_count_below_cap_leaves_tail(impl):
     N, A, H, d = 700, 300, 2, 64
     q = synth.gaussian_bf16((A, H, d), 20)

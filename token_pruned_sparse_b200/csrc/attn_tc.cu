@@ -6,11 +6,15 @@
 // valid rows for skipped ones), so the attention costs O(|A_i| * N).
 // Key-block sparsity ([SVOO] part 2, co-clustering -> block-sparse attention;
 // [TR] skipping of reusable work): with a mask, a query attends only the
-// 128-key blocks its ORIGINAL 128-token block keeps; whole key tiles that no
-// query of a CTA needs are never loaded.
+// 128-key blocks its ORIGINAL 128-token block keeps.
 //
-// One CTA = 256 compacted active queries of one head, as two 128-row tiles
-// (t = 0, 1) that share every K/V tile and take turns on the tensor cores:
+// Dense mode: one CTA = 256 compacted active queries of one head, as two
+// 128-row tiles (t = 0, 1) that share every K/V tile. Block mode (a mask is
+// given): tile t of CTA x holds the active rows of original query block
+// 2x + t (at most 128; the rest of the tile is padding) and streams only the
+// key tiles that block keeps, so every loaded key tile is work for every row
+// of its tile; the two tiles' loads interleave in one K ring and one V ring.
+// In both modes the two tiles take turns on the tensor cores:
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r of
 //              its tile (= TMEM lane r). Loads S from TMEM, online softmax in
 //              the log2 domain, writes P (bf16) back over the first half of
@@ -24,6 +28,7 @@
 //              freed when the last S MMA reading it completes and a V stage
 //              when the last P V MMA does, so the next K tile streams in about
 //              one tile period earlier than a shared K/V stage would allow.
+//              (Block mode: each stage has one reader, its own tile.)
 //   warp 9     MMA issuer and TMEM owner. Per key tile j and tile t:
 //              O_t += P_t(j) V_j (A operand read from TMEM), then
 //              S_t(j+1) = Q_t K_{j+1}^T; completion via tcgen05.commit.
@@ -62,9 +67,9 @@ struct Layout {
   static constexpr int kQ = 0;                           // [tile][sub]
   static constexpr int kK = kQ + kQT * kSub * kSubBytes; // [stage][sub]
   static constexpr int kV = kK + kStages * kSub * kSubBytes;
-  static constexpr int kList = kV + kStages * kSub * kSubBytes;   // uint16 kept key blocks
+  static constexpr int kList = kV + kStages * kSub * kSubBytes;   // uint16 kept key blocks, per tile
   static constexpr int kListMax = 4096;
-  static constexpr int kBar = kList + kListMax * 2;      // mbarriers (Bars)
+  static constexpr int kBar = kList + kQT * kListMax * 2;   // mbarriers (Bars)
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
 };
@@ -112,27 +117,61 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return r;
 }
 
-template <int D>
+template <int D, bool kBlk>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams prm) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
-  __shared__ int s_ntiles;
+  __shared__ int s_ntiles[kQT];
+  __shared__ int s_nrows[kQT];
+  __shared__ int s_row0[kQT];
   __shared__ volatile int s_abort;
-  __shared__ unsigned int s_wcnt[kWarps];
+  __shared__ unsigned int s_wcnt[kQT][kWarps];
 
   const AttnArgs& p = prm.a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int64_t rows = active_count(p.count, p.cap);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
-  if (row0 >= rows) return;   // whole CTA exits before touching TMEM or barriers
+
+  // ---- the query rows of each tile ------------------------------------------------------
+  // Dense: tile t = compacted rows [256 bx + 128 t, +128). Block mode: tile t =
+  // the active rows of original query block qb = 2 bx + t, i.e. the run of the
+  // ascending idx inside [128 qb, 128 qb + 128): every row of a tile then keeps
+  // the same key blocks, so every key tile a tile loads is work for all its rows.
+  if constexpr (kBlk) {
+    if (warp == 0) {
+      // lane 2t: first row of tile t; lane 2t + 1: one past its last row (lower bounds in idx)
+      const int64_t key = (2 * static_cast<int64_t>(blockIdx.x) + (lane >> 1) + (lane & 1)) * 128;
+      int64_t lo = 0, hi = rows;
+      while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (p.idx[mid] < key) lo = mid + 1;
+        else hi = mid;
+      }
+      const int64_t end = __shfl_down_sync(0xffffffffu, lo, 1);
+      if (lane < 2 * kQT && (lane & 1) == 0) {
+        const int64_t n = end - lo;
+        s_row0[lane >> 1] = static_cast<int>(lo);
+        s_nrows[lane >> 1] = static_cast<int>(n < 0 ? 0 : (n > kBM ? kBM : n));
+      }
+    }
+    __syncthreads();
+    if (s_nrows[0] == 0 && s_nrows[1] == 0) return;   // uniform: before TMEM or barriers
+  } else {
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
+    if (base >= rows) return;                          // whole CTA exits before touching TMEM or barriers
+    if (tid < kQT) {
+      const int64_t n = rows - (base + tid * kBM);
+      s_row0[tid] = static_cast<int>(base + tid * kBM);
+      s_nrows[tid] = static_cast<int>(n < 0 ? 0 : (n > kBM ? kBM : n));
+    }
+  }
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
-  uint16_t* sList = reinterpret_cast<uint16_t*>(gbase + L::kList);
+  uint16_t* sList = reinterpret_cast<uint16_t*>(gbase + L::kList);   // [tile][kListMax]
   const uint32_t bar0 = sbase + L::kBar;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int nkt_all = static_cast<int>((p.N + kBN - 1) / kBN);   // key tiles = key blocks
@@ -140,7 +179,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int kt0 = static_cast<int>((static_cast<int64_t>(nkt_all) * blockIdx.z) / prm.nsplit);
   const int nkt = static_cast<int>((static_cast<int64_t>(nkt_all) * (blockIdx.z + 1)) / prm.nsplit) - kt0;
 
-  // ---- setup: barriers, TMEM, key-tile list ---------------------------------------------
+  // ---- setup: barriers, TMEM, key-tile lists ------------------------------------------
   if (tid == 0) {
     s_abort = 0;
     for (int t = 0; t < kQT; ++t) {
@@ -164,76 +203,104 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (p.bm) {
-    const int64_t rlast = row0 + kQT * kBM - 1 < rows ? row0 + kQT * kBM - 1 : rows - 1;
-    int qb0 = p.idx[row0] / 128, qb1 = p.idx[rlast] / 128;
-    qb0 = qb0 < 0 ? 0 : (qb0 >= p.nb ? p.nb - 1 : qb0);
-    qb1 = qb1 < qb0 ? qb0 : (qb1 >= p.nb ? p.nb - 1 : qb1);
-    int base = 0;
+  if constexpr (kBlk) {
+    // tile t's key list: the key blocks its query block keeps, ascending
+    __syncthreads();                                   // s_nrows visible to every warp
+    int base[kQT] = {0, 0};
+    const uint8_t* mrow[kQT];
+    for (int t = 0; t < kQT; ++t)
+      mrow[t] = p.bm + (2 * static_cast<int64_t>(blockIdx.x) + t) * p.nb;
     for (int kb0 = 0; kb0 < p.nb; kb0 += kThreads) {
       const int kb = kb0 + tid;
-      bool keep = false;
-      if (kb < p.nb)
-        for (int qb = qb0; qb <= qb1 && !keep; ++qb) keep = p.bm[static_cast<int64_t>(qb) * p.nb + kb] != 0;
-      const unsigned int m = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0) s_wcnt[warp] = __popc(m);
-      __syncthreads();
-      int off = base, tot = 0;
-      for (int i = 0; i < kWarps; ++i) {
-        off += i < warp ? s_wcnt[i] : 0;
-        tot += s_wcnt[i];
+      unsigned int m[kQT];
+      for (int t = 0; t < kQT; ++t) {
+        const bool keep = s_nrows[t] > 0 && kb < p.nb && mrow[t][kb] != 0;
+        m[t] = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) s_wcnt[t][warp] = __popc(m[t]);
       }
-      if (keep) sList[off + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb);
-      base += tot;
+      __syncthreads();
+      for (int t = 0; t < kQT; ++t) {
+        int off = base[t], tot = 0;
+        for (int i = 0; i < kWarps; ++i) {
+          off += i < warp ? s_wcnt[t][i] : 0;
+          tot += s_wcnt[t][i];
+        }
+        if ((m[t] >> lane) & 1u)
+          sList[t * L::kListMax + off + __popc(m[t] & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb);
+        base[t] += tot;
+      }
       __syncthreads();
     }
-    if (tid == 0) s_ntiles = base;
-  } else if (tid == 0) {
-    s_ntiles = nkt;
+    if (tid < kQT) s_ntiles[tid] = base[tid];
+  } else if (tid < kQT) {
+    s_ntiles[tid] = nkt;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int ntiles = s_ntiles;
   const uint32_t tmem = s_tmem;
   auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
-  auto tile_kb = [&](int j) -> int { return p.bm ? static_cast<int>(sList[j]) : kt0 + j; };
+  auto tile_kb = [&](int t, int j) -> int {
+    if constexpr (kBlk) return static_cast<int>(sList[t * L::kListMax + j]);
+    else return kt0 + j;
+  };
+  const int n0 = s_ntiles[0], n1 = s_ntiles[1];
+  // Position of (tile t, key step j) in the K and V load sequence. Dense: both
+  // tiles read the one tile of step j. Block mode: loads go (j,0), (j,1), (j+1,0),
+  // ... skipping a tile whose list has ended.
+  auto seq_of = [&](int j, int t) -> int {
+    if constexpr (kBlk) return (j < n0 ? j : n0) + (j < n1 ? j : n1) + (t == 1 && j < n0 ? 1 : 0);
+    else return j;
+  };
 
   if (warp == kTmaWarp) {
     // ================================ TMA producer =====================================
     if (lane == 0) {
       int issued_k = 0, issued_v = 0;
+      bool q_issued[kQT];
       for (int t = 0; t < kQT; ++t) {
+        q_issued[t] = s_ntiles[t] > 0;
+        if (!q_issued[t]) continue;
         mbar_expect_tx(bar(Bars::q_full + t), L::kSub * kSubBytes);
         for (int s = 0; s < L::kSub; ++s)
-          tma_load_3d(sbase + L::kQ + (t * L::kSub + s) * kSubBytes, &tmQ, 64 * s, h,
-                      static_cast<int>(row0 + t * kBM), bar(Bars::q_full + t));
+          tma_load_3d(sbase + L::kQ + (t * L::kSub + s) * kSubBytes, &tmQ, 64 * s, h, s_row0[t],
+                      bar(Bars::q_full + t));
       }
       // K and V stages are freed separately: a K stage as soon as the last S MMA
       // reading it completes (about one period before its PV stage), so the next
       // K tile streams in while the current P.V products still run.
-      for (int j = 0; j < ntiles; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = ((j / kStages) - 1) & 1;
-        const int key0 = tile_kb(j) * kBN;
-        if (j >= kStages && !mbar_wait(bar(Bars::k_empty + st), ph, &s_abort, prm.status)) break;
-        mbar_expect_tx(bar(Bars::k_full + st), L::kSub * kSubBytes);
-        for (int s = 0; s < L::kSub; ++s)
-          tma_load_3d(sbase + L::kK + (st * L::kSub + s) * kSubBytes, &tmK, 64 * s, h, key0, bar(Bars::k_full + st));
-        issued_k = j + 1;
-        if (j >= kStages && !mbar_wait(bar(Bars::v_empty + st), ph, &s_abort, prm.status)) break;
-        mbar_expect_tx(bar(Bars::v_full + st), L::kSub * kSubBytes);
-        for (int s = 0; s < L::kSub; ++s)
-          tma_load_3d(sbase + L::kV + (st * L::kSub + s) * kSubBytes, &tmV, 64 * s, h, key0, bar(Bars::v_full + st));
-        issued_v = j + 1;
+      const int jmax = n0 > n1 ? n0 : n1;
+      const int ntl = kBlk ? kQT : 1;                   // loads per key step
+      bool ok = true;
+      for (int j = 0; ok && j < jmax; ++j) {
+        for (int t = 0; ok && t < ntl; ++t) {
+          if (j >= s_ntiles[t]) continue;
+          const int q = seq_of(j, t);
+          const int st = q % kStages;
+          const uint32_t ph = ((q / kStages) - 1) & 1;
+          const int key0 = tile_kb(t, j) * kBN;
+          if (q >= kStages && !mbar_wait(bar(Bars::k_empty + st), ph, &s_abort, prm.status)) ok = false;
+          if (!ok) break;
+          mbar_expect_tx(bar(Bars::k_full + st), L::kSub * kSubBytes);
+          for (int s = 0; s < L::kSub; ++s)
+            tma_load_3d(sbase + L::kK + (st * L::kSub + s) * kSubBytes, &tmK, 64 * s, h, key0, bar(Bars::k_full + st));
+          issued_k = q + 1;
+          if (q >= kStages && !mbar_wait(bar(Bars::v_empty + st), ph, &s_abort, prm.status)) ok = false;
+          if (!ok) break;
+          mbar_expect_tx(bar(Bars::v_full + st), L::kSub * kSubBytes);
+          for (int s = 0; s < L::kSub; ++s)
+            tma_load_3d(sbase + L::kV + (st * L::kSub + s) * kSubBytes, &tmV, 64 * s, h, key0, bar(Bars::v_full + st));
+          issued_v = q + 1;
+        }
       }
       // drain: every load issued above must land before the CTA may exit
-      for (int t = 0; t < kQT; ++t) drain_wait(bar(Bars::q_full + t), 0);
-      for (int j = issued_k > kStages ? issued_k - kStages : 0; j < issued_k; ++j)
-        drain_wait(bar(Bars::k_full + j % kStages), (j / kStages) & 1);
-      for (int j = issued_v > kStages ? issued_v - kStages : 0; j < issued_v; ++j)
-        drain_wait(bar(Bars::v_full + j % kStages), (j / kStages) & 1);
+      for (int t = 0; t < kQT; ++t)
+        if (q_issued[t]) drain_wait(bar(Bars::q_full + t), 0);
+      for (int q = issued_k > kStages ? issued_k - kStages : 0; q < issued_k; ++q)
+        drain_wait(bar(Bars::k_full + q % kStages), (q / kStages) & 1);
+      for (int q = issued_v > kStages ? issued_v - kStages : 0; q < issued_v; ++q)
+        drain_wait(bar(Bars::v_full + q % kStages), (q / kStages) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ================================ MMA issuer =======================================
@@ -241,7 +308,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, false, false);  // Q K^T: both K-major
       constexpr uint32_t kIdescO = idesc_bf16(kBM, D, false, true);     // P V: V is MN-major
       auto issue_s = [&](int t, int j) {
-        const int st = j % kStages;
+        const int st = seq_of(j, t) % kStages;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;   // 16 bf16 along d
@@ -250,20 +317,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_f16_ss(tS(t), da, db, kIdescS, kk > 0);
         }
         mma_commit(bar(Bars::s_full + t));
-        if (t == kQT - 1) mma_commit(bar(Bars::k_empty + st));   // last reader of this K stage
+        if (kBlk || t == kQT - 1) mma_commit(bar(Bars::k_empty + st));   // last reader of this K stage
       };
-      bool ok = ntiles > 0;
-      if (ok) ok = mbar_wait(bar(Bars::k_full), 0, &s_abort, prm.status);
+      // K stage of (t, j) full: dense tiles share step j's stage and wait once (t = 0)
+      auto wait_k = [&](int t, int j) -> bool {
+        if (!kBlk && t != 0) return true;
+        const int q = seq_of(j, t);
+        const bool r = mbar_wait(bar(Bars::k_full + q % kStages), (q / kStages) & 1, &s_abort, prm.status);
+        tc_fence_after();
+        return r;
+      };
+      bool ok = true;
       for (int t = 0; ok && t < kQT; ++t) {
-        ok = mbar_wait(bar(Bars::q_full + t), 0, &s_abort, prm.status);
+        if (s_ntiles[t] == 0) continue;
+        ok = wait_k(t, 0) && mbar_wait(bar(Bars::q_full + t), 0, &s_abort, prm.status);
         tc_fence_after();
         if (ok) issue_s(t, 0);
       }
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j % kStages;
+      const int jmax = n0 > n1 ? n0 : n1;
+      for (int j = 0; ok && j < jmax; ++j) {
         for (int t = 0; ok && t < kQT; ++t) {
+          if (j >= s_ntiles[t]) continue;
+          const int q = seq_of(j, t);
+          const int st = q % kStages;
           ok = mbar_wait(bar(Bars::p_full + t), j & 1, &s_abort, prm.status);
-          if (ok && t == 0) ok = mbar_wait(bar(Bars::v_full + st), (j / kStages) & 1, &s_abort, prm.status);
+          if (ok && (kBlk || t == 0)) ok = mbar_wait(bar(Bars::v_full + st), (q / kStages) & 1, &s_abort, prm.status);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -275,14 +353,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mma_f16_ts(tO(t), tS(t) + 8 * kk, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(Bars::pv_done + t));
-          if (t == kQT - 1) mma_commit(bar(Bars::v_empty + st));   // last reader of this V stage
-          if (j + 1 < ntiles) {
+          if (kBlk || t == kQT - 1) mma_commit(bar(Bars::v_empty + st));   // last reader of this V stage
+          if (j + 1 < s_ntiles[t]) {
             // S_t(j+1) overwrites the columns P_t(j) was read from: tcgen05.mma
             // operations of one thread execute in issue order.
-            if (t == 0) {
-              ok = mbar_wait(bar(Bars::k_full + (j + 1) % kStages), ((j + 1) / kStages) & 1, &s_abort, prm.status);
-              tc_fence_after();
-            }
+            ok = wait_k(t, j + 1);
             if (ok) issue_s(t, j + 1);
           }
         }
@@ -293,14 +368,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ================================ softmax warps ====================================
     const int t = warp >> 2;                      // query tile of this warpgroup
     const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
-    const int64_t row = row0 + t * kBM + r;
-    const bool valid = row < rows;
+    const int64_t row = static_cast<int64_t>(s_row0[t]) + r;
+    const bool valid = r < s_nrows[t];
+    const int ntiles = s_ntiles[t];
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int qb = 0;
-    if (p.bm) {
-      qb = p.idx[valid ? row : rows - 1] / 128;
-      qb = qb < 0 ? 0 : (qb >= p.nb ? p.nb - 1 : qb);
-    }
     const float sl2 = prm.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_run = -INFINITY, l_run = 0.f;
@@ -312,10 +383,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      const int kb = tile_kb(j);
-      const int64_t key0 = static_cast<int64_t>(kb) * kBN;
-      const bool row_ok = !p.bm || p.bm[static_cast<int64_t>(qb) * p.nb + kb] != 0;
-      const int nvalid = row_ok ? static_cast<int>(p.N - key0 < kBN ? p.N - key0 : kBN) : 0;
+      const int64_t key0 = static_cast<int64_t>(tile_kb(t, j)) * kBN;
+      // a row outside the tile's query rows takes no key (its S is whatever the
+      // padding rows held); keys past N are masked
+      const int nvalid = valid ? static_cast<int>(p.N - key0 < kBN ? p.N - key0 : kBN) : 0;
       uint32_t sr[kBN];
       auto load_s = [&]() {
         tmem_ld128(tS(t) + lane_off, sr);
@@ -424,15 +495,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (valid) prm.lse_part[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       } else {
         uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < D; c += 32) {
           float o[32];
           if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
           else
-  #pragma unroll
+#pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = 0.f;
           if (valid) {
-  #pragma unroll
+#pragma unroll
             for (int q = 0; q < 4; ++q)
               orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
                                            pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
@@ -470,6 +541,26 @@ int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, 
   return TPS_OK;
 }
 
+// Sets the kernel's dynamic shared-memory limit once per device (setting it
+// twice is harmless; devices numbered 64 and above set it on every launch).
+template <int D, bool kBlk>
+int smem_attribute() {
+  static std::atomic<bool> done[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire);
+  if (!cached) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kBlk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Layout<D>::kAlloc);
+    if (e != cudaSuccess) return cuda_status(e, "pruned_attn: smem attribute");
+    if (dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_release);
+  }
+  return TPS_OK;
+}
+
+// Dense: ceil(cap/256) x H x nsplit CTAs of two 128-row tiles of compacted rows.
+// Masked (block mode): ceil(nb/2) x H CTAs, CTA x holding the active rows of
+// query blocks 2x and 2x+1, each tile with its own key list.
 template <int D>
 int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr) {
   if (a.cap == 0) return TPS_OK;
@@ -483,19 +574,17 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   constexpr int kSmem = Layout<D>::kAlloc;
-  static std::atomic<bool> attr_done[64];   // per device; setting the attribute twice is harmless
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const bool cached = dev >= 0 && dev < 64 && attr_done[dev].load(std::memory_order_acquire);
-  if (!cached) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return cuda_status(e, "pruned_attn: smem attribute");
-    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
-  }
   TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part};
-  dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
-            static_cast<unsigned int>(nsplit));
-  attn_tc_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+  if (a.bm) {
+    if (int e = smem_attribute<D, true>()) return e;
+    dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
+    attn_tc_kernel<D, true><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+  } else {
+    if (int e = smem_attribute<D, false>()) return e;
+    dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
+              static_cast<unsigned int>(nsplit));
+    attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+  }
   return launch_status("pruned_attn");
 }
 
