@@ -263,7 +263,12 @@ TPS_API int kv_rerotate(const tps_bf16* k_cache, const int32_t* idx, const int32
  *          logits. A row with no allowed key gets o = 0 and lse = -inf.
  * scale must be finite and > 0 (typically 1/sqrt(d)).
  * bf16 inputs, fp32 accumulation and softmax, tcgen05 tensor cores.
- * d in {64, 128}; 1 <= H <= 256; N < 2^31; pointers 16-byte aligned. */
+ * d in {64, 128}; 1 <= H <= 256; N < 2^31; pointers 16-byte aligned.
+ * Dense launches that would fill the GPU poorly (few 256-row query tiles x
+ * heads, e.g. a low keep ratio) split the key range S <= 4 ways over a
+ * thread-block cluster whose CTAs merge their partial results over
+ * distributed shared memory (S from tps_attn_split; no workspace). Results
+ * agree with the unsplit kernel within the attention tolerance. */
 TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
                 const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
                 float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
@@ -282,6 +287,10 @@ TPS_API int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tps_b
                            float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
                            void* ws, size_t ws_bytes, tps_stream stream);
 TPS_API size_t tps_attn_workspace_size(int64_t cap, int64_t N, int H, int d);
+
+/* The key-range split S (1..4) a dense pruned_attn call of this shape runs
+ * with on the current device (1 = unsplit). HOST query, no launch. */
+TPS_API int tps_attn_split(int64_t cap, int64_t N, int H, int d);
 
 /* Same contract as pruned_attn, computed with the legacy warp-level
  * mma.sync tensor-core path (kept as the baseline the tcgen05 kernel is

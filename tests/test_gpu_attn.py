@@ -402,3 +402,50 @@ def test_attn_ws_wan_keep10_sampled():
 def test_attn_ws_no_split_when_grid_is_full():
     # 24 x 12 = 288 CTAs fill 148 SMs twice at 97%: no split, no workspace
     assert tps.lib().tps_attn_workspace_size(6084, 20280, 12, 128) == 0
+
+
+# ------------------------------- split-key attention merged inside a cluster -----
+@pytest.mark.parametrize("N,S", [(1100, 2), (1600, 3), (4099, 4)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_cluster_split_matches_oracle(N, S, d):
+    """One query tile pair x one head fills one SM: pruned_attn splits the keys
+    over a cluster of S CTAs (S bounded by 4 key tiles per split) that merge
+    over distributed shared memory. A score spike confined to one split's key
+    range gives the partials very different maxima; a count below cap leaves
+    the tail rows untouched."""
+    A, H = 200, 1
+    assert tps.attn_split(A, N, H, d) == S
+    q = synth.gaussian_bf16((A, H, d), N + S)
+    k = synth.gaussian_bf16((N, H, d), N + S + 1).double()
+    k[N - 300:N - 200] *= 25.0                              # inside the last split only
+    k = k.to(torch.bfloat16)
+    v = synth.gaussian_bf16((N, H, d), N + S + 2)
+    idx = np.sort(np.random.default_rng(S).choice(N, A, replace=False))
+    for scale in (1 / math.sqrt(d), 0.35):
+        o, lse = _run("pruned_attn", q, k, v, idx, scale)
+        o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
+        _check(o, lse, o_ref, lse_ref)
+    o, lse = _run("pruned_attn", q, k, v, idx, 0.2, count=150)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 0.2, rows=np.arange(150))
+    _check(o[:150], lse[:150], o_ref, lse_ref)
+    assert torch.all(o[150:].float() == 7.0) and np.all(lse[150:] == 7.0)
+
+
+def test_attn_cluster_split_wan_keep10_sampled():
+    """The Wan-like layer at keep 10% (3276 queries x 32760 keys, 12 heads:
+    156 CTAs on 148 SMs) through pruned_attn: the cluster split is chosen and
+    matches the oracle on sampled rows."""
+    Q, K, V = qkv("wan")
+    N, H, d = Q.shape
+    idx = oracle_idx("wan", 0)
+    A = len(idx)
+    assert tps.attn_split(A, N, H, d) > 1
+    o, lse = _run("pruned_attn", Q[idx], K, V, idx, 1 / math.sqrt(d))
+    rows = _sample(A, 192, 6)
+    o_ref, lse_ref = O.pruned_attn(Q[idx], K, V, idx, 1 / math.sqrt(d), rows=rows)
+    _check(o, lse, o_ref, lse_ref, rows=rows)
+
+
+def test_attn_no_cluster_split_when_grid_is_full():
+    assert tps.attn_split(6084, 20280, 12, 128) == 1
+    assert tps.attn_split(39600, 118800, 24, 128) == 1

@@ -84,7 +84,8 @@ struct Bars {  // mbarrier indices inside the barrier block (8 bytes each)
   static constexpr int p_full = s_full + kQT;          // + tile
   static constexpr int pv_done = p_full + kQT;         // + tile
   static constexpr int drain = pv_done + kQT;          // last commit of the MMA thread
-  static constexpr int count = drain + 1;
+  static constexpr int merge = drain + 1;              // cluster leader: every partner's partials staged
+  static constexpr int count = merge + 1;
 };
 static_assert(Bars::count * 8 <= 256, "barrier block");
 
@@ -93,9 +94,12 @@ struct TcParams {
   float scale_log2;
   unsigned int* status;
   int nsplit;          // key-range splits (blockIdx.z); 1 = whole key range
-  float* o_part;       // nsplit > 1: normalised partial outputs, fp32 [nsplit][cap][H][D]
-  float* lse_part;     // nsplit > 1: partial log-sum-exp, fp32 [nsplit][cap][H]
+  float* o_part;       // nsplit > 1, workspace merge: normalised partial outputs, fp32 [nsplit][cap][H][D]
+  float* lse_part;     // nsplit > 1, workspace merge: partial log-sum-exp, fp32 [nsplit][cap][H]
+  int cluster;         // > 1: the nsplit CTAs of a cluster merge their partials over distributed
+                       // shared memory (no workspace); 1 otherwise
 };
+constexpr int kMaxCluster = 4;
 
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -195,6 +199,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(Bars::v_empty + s), 1);
     }
     mbar_init(bar(Bars::drain), 1);
+    if (prm.cluster > 1) mbar_init(bar(Bars::merge), kSoftmaxThreads * (prm.cluster - 1));
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc<kTmemCols>(smem_u32(&s_tmem));
@@ -238,6 +243,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // cluster merge: every CTA of the cluster runs and has its barriers initialised
+  // before any CTA arrives on a peer's barrier
+  if (prm.cluster > 1) cluster_sync_all();
   const uint32_t tmem = s_tmem;
   auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
@@ -473,7 +481,87 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && ntiles > 0) ok = mbar_wait(bar(Bars::pv_done + t), (ntiles - 1) & 1, &s_abort, prm.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    if (ok) {
+    if (ok && prm.cluster > 1) {
+      // Split-key partials merged inside the cluster over distributed shared
+      // memory: a partner stages its unnormalised O rows and (m, l) in its own
+      // K/V ring region (free once its last P V has completed: the K ring holds
+      // tile 0's rows, the V ring tile 1's) and arrives on the leader's merge
+      // barrier; the leader reads every partner's rows and writes the output.
+      constexpr int kChunks = D / 4;                                   // float4 chunks per row
+      const int srow = t * kBM + r;
+      float4* stage = reinterpret_cast<float4*>(gbase + L::kK);       // [256][kChunks], chunk rotated by row
+      float2* ml = reinterpret_cast<float2*>(gbase + L::kList);       // [256] (m_run, l_run)
+      const uint32_t crank = cluster_ctarank();
+      if (crank != 0) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            stage[srow * kChunks + (c / 4 + q + r) % kChunks] =
+                make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        }
+        ml[srow] = make_float2(m_run, l_run);
+        mbar_arrive_remote(map_to_rank(bar(Bars::merge), 0));
+      } else if (__all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::merge), 0, &s_abort, prm.status))) {
+        const int np = prm.cluster - 1;
+        float mk[kMaxCluster - 1], ak[kMaxCluster - 1];
+        uint32_t rbase[kMaxCluster - 1];
+        float M = m_run;
+#pragma unroll
+        for (int k = 0; k < kMaxCluster - 1; ++k) {
+          mk[k] = -INFINITY;
+          ak[k] = 0.f;
+          rbase[k] = 0u;
+          if (k < np) {
+            const float2 v = ld_cluster_f2(map_to_rank(smem_u32(&ml[srow]), k + 1));
+            mk[k] = v.x;
+            ak[k] = v.y;                                                // l of partner k, for now
+            rbase[k] = map_to_rank(smem_u32(stage), k + 1);
+            M = fmaxf(M, v.x);
+          }
+        }
+        const float a0 = m_run == -INFINITY ? 0.f : fast_exp2(m_run - M);
+        float l = a0 * l_run;
+#pragma unroll
+        for (int k = 0; k < kMaxCluster - 1; ++k) {
+          const float lk = ak[k];
+          ak[k] = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - M);
+          l += ak[k] * lk;
+        }
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= a0;
+#pragma unroll
+          for (int k = 0; k < kMaxCluster - 1; ++k) {
+            if (k >= np) break;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 x = ld_cluster_f4(rbase[k] + static_cast<uint32_t>(srow * kChunks + (c / 4 + q + r) % kChunks) * 16u);
+              o[4 * q] = fmaf(ak[k], x.x, o[4 * q]);
+              o[4 * q + 1] = fmaf(ak[k], x.y, o[4 * q + 1]);
+              o[4 * q + 2] = fmaf(ak[k], x.z, o[4 * q + 2]);
+              o[4 * q + 3] = fmaf(ak[k], x.w, o[4 * q + 3]);
+            }
+          }
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
+                                           pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                           pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                           pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+          }
+        }
+        if (valid && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
+      }
+    } else if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       if (prm.nsplit > 1) {
         // partial result of this key range: normalised fp32 row + its log-sum-exp
@@ -521,6 +609,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // a partner's shared memory stays valid until the leader has read it
+  if (prm.cluster > 1) cluster_sync_all();
   if (warp == kMmaWarp) {
     __syncwarp();
     tmem_dealloc<kTmemCols>(tmem);
@@ -574,7 +664,7 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   constexpr int kSmem = Layout<D>::kAlloc;
-  TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part};
+  TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1};
   if (a.bm) {
     if (int e = smem_attribute<D, true>()) return e;
     dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
@@ -585,6 +675,105 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
               static_cast<unsigned int>(nsplit));
     attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   }
+  return launch_status("pruned_attn");
+}
+
+// CTAs of the dense kernel resident at once when launched in clusters of S
+// along z: cudaOccupancyMaxActiveClusters x S (the SM count for S = 1),
+// cached per device; 0 if clusters of S cannot be scheduled.
+template <int D>
+int cluster_slots(int S) {
+  if (S <= 1) return sm_count();
+  static std::atomic<int> cache[64][kMaxCluster + 1];   // 0 = not yet queried; stored as slots + 1
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cacheable = dev >= 0 && dev < 64;
+  if (cacheable) {
+    const int v = cache[dev][S].load(std::memory_order_acquire);
+    if (v > 0) return v - 1;
+  }
+  if (smem_attribute<D, false>()) return 0;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(1, 1, static_cast<unsigned int>(S));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<D>::kAlloc;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned int>(S);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<D, false>, &cfg) != cudaSuccess) {
+    cudaGetLastError();                 // a failed query leaves its error in the last-error slot
+    n = 0;
+  }
+  const int slots = n * S;
+  if (cacheable) cache[dev][S].store(slots + 1, std::memory_order_release);
+  return slots;
+}
+
+// Key-range splits merged inside a thread-block cluster, for a dense launch
+// that would fill the GPU poorly: ceil(cap/256) x H CTAs that leave most of
+// their last wave empty run as S <= 4 key-range splits, the S CTAs of one
+// (query tile pair, head) forming a cluster along z that merges its partials
+// over distributed shared memory. S is chosen by wave efficiency against the
+// CTAs the GPU keeps resident in clusters of S; >= 4 key tiles per split.
+template <int D>
+int choose_cluster_split(int64_t cap, int H, int64_t N) {
+  const int64_t units = ((cap + kQT * kBM - 1) / (kQT * kBM)) * H;
+  const int64_t nkt = (N + kBN - 1) / kBN;
+  if (units <= 0) return 1;
+  const int64_t sms = sm_count();
+  if (static_cast<double>(units) / static_cast<double>(((units + sms - 1) / sms) * sms) >= 0.9) return 1;
+  // time in units of one unsplit CTA: waves of S-split CTAs, each doing 1/S of the keys
+  auto cost = [&](int S) -> double {
+    const int64_t slots = cluster_slots<D>(S);
+    if (slots <= 0) return 1e30;
+    return static_cast<double>((units * S + slots - 1) / slots) / S;
+  };
+  int best = 1;
+  double bc = cost(1);
+  for (int S = 2; S <= kMaxCluster; ++S) {
+    if (nkt < 4 * S) break;
+    const double c = cost(S);
+    if (c < 0.98 * bc) {
+      best = S;
+      bc = c;
+    }
+  }
+  return best;
+}
+
+template <int D>
+int launch_cluster(const AttnArgs& a, cudaStream_t st, int S) {
+  EncodeTiledFn enc;
+  if (int e = tensor_map_encoder(&enc, "pruned_attn")) return e;
+  int err;
+  unsigned int* status = device_status(&err);
+  if (!status) return err;
+  CUtensorMap mq, mk, mv;
+  if (int e = make_map(enc, &mq, a.q, a.cap, a.H, a.d)) return e;
+  if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
+  if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
+  if (int e = smem_attribute<D, false>()) return e;
+  TcParams prm{a, a.scale * kLog2e, status, S, nullptr, nullptr, S};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
+                     static_cast<unsigned int>(S));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<D>::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned int>(S);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, false>, mq, mk, mv, prm);
+  if (e != cudaSuccess) return cuda_status(e, "pruned_attn: cluster launch");
   return launch_status("pruned_attn");
 }
 
@@ -661,6 +850,12 @@ extern "C" int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tp
   return e ? e : ok();
 }
 
+extern "C" int tps_attn_split(int64_t cap, int64_t N, int H, int d) {
+  using namespace tps;
+  if (cap <= 0 || N <= 0 || H <= 0 || (d != 64 && d != 128)) return 1;
+  return d == 64 ? choose_cluster_split<64>(cap, H, N) : choose_cluster_split<128>(cap, H, N);
+}
+
 extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
                            const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,
                            const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse, tps_stream stream) {
@@ -671,6 +866,10 @@ extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_b
                             lse, &a))
     return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int e = d == 64 ? launch<64>(a, st) : launch<128>(a, st);
+  int e;
+  const int S = blockmask || cap == 0 ? 1 : (d == 64 ? choose_cluster_split<64>(cap, H, N)
+                                                     : choose_cluster_split<128>(cap, H, N));
+  if (S > 1) e = d == 64 ? launch_cluster<64>(a, st, S) : launch_cluster<128>(a, st, S);
+  else e = d == 64 ? launch<64>(a, st) : launch<128>(a, st);
   return e ? e : ok();
 }

@@ -38,6 +38,7 @@ SIGNATURES = {
     "pruned_attn_ws": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P,
                               C.c_size_t, _P]),
     "tps_attn_workspace_size": (C.c_size_t, [_I64, _I64, _INT, _INT]),
+    "tps_attn_split": (_INT, [_I64, _I64, _INT, _INT]),
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
     "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
@@ -238,6 +239,11 @@ def pruned_attn(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act
 def attn_workspace(cap, N, H, d, device=None):
     n = int(lib().tps_attn_workspace_size(cap, N, H, d))
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda"), n
+
+
+def attn_split(cap, N, H, d) -> int:
+    """Key-range split a dense pruned_attn call of this shape uses (1 = none)."""
+    return int(lib().tps_attn_split(int(cap), int(N), int(H), int(d)))
 
 
 def pruned_attn_ws(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None, cap=None,
