@@ -203,10 +203,10 @@ class HsaStep(PathStep):
     holds the previous step's projections, and the output cache starts at
     zero (the step rewrites the active rows)."""
 
-    # this library's kernels per step: score 1; group 7 (radix init, 4 radix
-    # passes, count, write); schedule 1 (cooperative); gathers 3; kv_sync 2
-    # (cache rows, re-noise); attention 1; scatter 1
-    LAUNCHES = {"score": 1, "group": 7, "schedule": 1, "gather": 3, "kv_sync": 2, "attn": 1, "scatter": 1}
+    # this library's kernels per step: score + group split 1 (one cooperative
+    # launch); schedule 1 (cooperative); gathers 3; kv_sync 2 (cache rows,
+    # re-noise); attention 1; scatter 1
+    LAUNCHES = {"score_group": 1, "schedule": 1, "gather": 3, "kv_sync": 2, "attn": 1, "scatter": 1}
 
     def __init__(self, seed_offset: int, dev, attn: str):
         from token_pruned_sparse_b200 import tps
@@ -251,15 +251,14 @@ class HsaStep(PathStep):
                 "group": torch.empty(self.N, dtype=torch.int8, device=dev),
                 "idx": torch.empty(self.N, dtype=torch.int32, device=dev),
                 "cnt": torch.empty(1, dtype=torch.int32, device=dev),
-                "ws_g": t.workspace(t.OP_GROUP, self.N, self.K, dev),
+                "ws_g": t.workspace(t.OP_FRONT, self.N, self.K, dev),
                 "ws_s": t.workspace(t.OP_SCHEDULE, self.N, self.K, dev),
                 "q": z(), "k": z(), "v": z(), "o": z()}
 
     def front(self, X, vp, vc, q, kf, vf):
         """score -> group -> schedule -> gathers into buffer set X."""
         t = self.tps
-        t.lipar_score(vc, vp, out=X["score"])
-        t.lipar_group(X["score"], self.K, group=X["group"], ws=X["ws_g"])
+        t.lipar_front(vc, t.FRONT_GROUP, x_ref=vp, K=self.K, group=X["group"], ws=X["ws_g"])
         t.lipar_schedule(X["group"], self.K, self.budgets, self.T, self.i, self.m, idx=X["idx"], count=X["cnt"],
                          ws=X["ws_s"])
         t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
@@ -311,7 +310,7 @@ class MidStep(PathStep):
     30% = 6084 active queries; the K/V cache holds the previous frame's
     projections."""
 
-    LAUNCHES = {"score": 1, "select_topk": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
+    LAUNCHES = {"score_topk": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
 
     def __init__(self, seed_offset: int, dev, attn: str):
         from token_pruned_sparse_b200 import tps
@@ -352,12 +351,11 @@ class MidStep(PathStep):
         return {"x": torch.empty_like(self.x), "score": torch.empty(self.N, dtype=torch.float32, device=dev),
                 "idx": torch.empty(self.k, dtype=torch.int32, device=dev),
                 "cnt": torch.empty(1, dtype=torch.int32, device=dev),
-                "ws": t.workspace(t.OP_SELECT, self.N, 0, dev), "q": z(), "k": z(), "v": z(), "o": z()}
+                "ws": t.workspace(t.OP_FRONT, self.N, 0, dev), "q": z(), "k": z(), "v": z(), "o": z()}
 
     def front(self, X, x, q, kf, vf):
         t = self.tps
-        t.lipar_score(x, out=X["score"])
-        t.lipar_select(X["score"], t.SELECT_TOPK, k=self.k, idx=X["idx"], count=X["cnt"], ws=X["ws"])
+        t.lipar_front(x, t.FRONT_TOPK, k=self.k, idx=X["idx"], count=X["cnt"], ws=X["ws"])
         t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
         t.tps_gather_rows(X["k"], kf, X["idx"], X["cnt"])
         t.tps_gather_rows(X["v"], vf, X["idx"], X["cnt"])
@@ -653,6 +651,16 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
                                          ws=wss), flush)
     A = int(cnt.item())
     stages["schedule"] = (t, N + A * 4)
+    # fused front end: score + top-k N/3, and score + group split, one cooperative launch each
+    wsf = tps.workspace(tps.OP_FRONT, N, K, dev)
+    idx_f = torch.empty(N, dtype=torch.int32, device=dev)
+    cnt_f = torch.empty(1, dtype=torch.int32, device=dev)
+    grp_f = torch.empty(N, dtype=torch.int8, device=dev)
+    t = timer(lambda: tps.lipar_front(v_cur, tps.FRONT_TOPK, x_ref=v_prev, k=k3, idx=idx_f, count=cnt_f, ws=wsf),
+              flush)
+    stages["front_score_topk"] = (t, N * (4 * C + 4) + k3 * 4)
+    t = timer(lambda: tps.lipar_front(v_cur, tps.FRONT_GROUP, x_ref=v_prev, K=K, group=grp_f, ws=wsf), flush)
+    stages["front_score_group"] = (t, N * (4 * C + 1))
     idx = idx_all[:A].clone()
     kc, vc = rnd(N, H, d), rnd(N, H, d)
     kf, vf = rnd(A, H, d), rnd(A, H, d)

@@ -164,6 +164,27 @@ TPS_API int lipar_select(const float* score, int64_t N, int mode, float tau, int
 TPS_API int lipar_select_static(const float* score, int64_t N, int mode, float tau, int64_t k,
                                 int32_t* idx, int32_t* count, tps_stream stream);
 
+/* ---- fused front end: steps 1-3 in one launch ([LIPAR] 2.B; [HSA] 2.1) ------
+ * Exactly lipar_score(x, x_ref, x_prev_frame, F, HW, C) followed by
+ *   mode TPS_FRONT_THRESHOLD / TPS_FRONT_TOPK: lipar_select (tau / k, idx,
+ *     count as there), or
+ *   mode TPS_FRONT_GROUP: lipar_group (K groups into group[N]).
+ * score: NULL, or float32 [N] that also receives the scores.
+ * For C in {64, 128} and N <= 524,288 this runs as ONE cooperative launch:
+ * each block scores its own tokens (the same arithmetic as lipar_score, so
+ * the scores are bit-identical) into shared memory and the selection or rank
+ * split reads them there; otherwise the separate kernels run, with identical
+ * results. ws: tps_workspace_size(TPS_OP_FRONT, N, K) bytes (K ignored except
+ * for groups), 16-byte aligned; its contents need no initialisation. Calls
+ * that share one workspace must be ordered on the GPU. */
+#define TPS_FRONT_THRESHOLD 0
+#define TPS_FRONT_TOPK      1
+#define TPS_FRONT_GROUP     2
+TPS_API int lipar_front(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame,
+                        int64_t F, int64_t HW, int64_t C, int mode, float tau, int64_t k, int K,
+                        float* score, int32_t* idx, int32_t* count, int8_t* group,
+                        void* ws, size_t ws_bytes, tps_stream stream);
+
 /* ---- HSA group assignment ([HSA] 2.1, dynamic token selection) -------------
  * Ranks tokens by score descending (ties to the lower index, NaN last) and
  * splits the ranks into K contiguous groups of N/K (the remainder joins the
@@ -337,6 +358,7 @@ TPS_API int hsa_euler_update(float* x, tps_bf16* v_cache, const tps_bf16* v_fres
 #define TPS_OP_SELECT   0
 #define TPS_OP_GROUP    1
 #define TPS_OP_SCHEDULE 2
+#define TPS_OP_FRONT    3
 /* Workspace bytes for lipar_select / lipar_group / lipar_schedule (0 on bad op). */
 TPS_API size_t tps_workspace_size(int op, int64_t N, int K);
 

@@ -157,3 +157,20 @@ def test_rerotate_validation():
     assert l.kv_rerotate(F, F, F, 10, 100, 2, 96, P(good), F, NULL) == tps.INVALID_ARG
     assert l.kv_rerotate(MIS, F, F, 10, 100, 2, 64, P(good), F, NULL) == tps.ALIGN
     assert l.kv_rerotate(F, F, F, 10, 0, 2, 64, P(good), F, NULL) == tps.SHAPE
+
+
+def test_front_validation():
+    l = tps.lib()
+    need = tps.workspace_min_size(tps.OP_FRONT, 100, 3)
+    assert need >= 400 and tps.workspace_size(tps.OP_FRONT, 100, 3) >= need
+    args = lambda mode, k=5, K=3, ws=F, nws=1 << 20, x=F: (x, NULL, NULL, 4, 25, 128, mode, 0.5, k, K, NULL,   # noqa: E731
+                                                          F, F, F, ws, nws, NULL)
+    assert l.lipar_front(*args(3)) == tps.INVALID_ARG
+    assert l.lipar_front(*args(1, k=101)) == tps.INVALID_ARG
+    assert l.lipar_front(*args(2, K=9)) == tps.INVALID_ARG
+    assert l.lipar_front(*args(0, x=NULL)) == tps.INVALID_ARG
+    assert l.lipar_front(*args(0, x=MIS)) == tps.ALIGN
+    code, msg = _err(l.lipar_front(*args(1, nws=16)))
+    assert code == tps.WORKSPACE and "required" in msg
+    assert l.lipar_front(F, F, F, 4, 25, 128, 0, 0.5, 5, 3, NULL, F, F, F, F, 1 << 20, NULL) == tps.INVALID_ARG
+    assert l.lipar_front(F, NULL, NULL, 4, 25, 100, 0, 0.5, 5, 3, NULL, F, F, F, F, 1 << 20, NULL) == tps.SHAPE

@@ -177,3 +177,84 @@ def test_select_multi_launch_path_matches_oracle(N):
             idx, cnt = tps.lipar_select(sd, tps.SELECT_THRESHOLD, tau=tau, ws=ws)
             assert np.array_equal(_idx(idx, cnt), O.select_threshold(sn, tau)), (N, tau, ws.numel())
     tps.tps_check()
+
+
+@pytest.mark.parametrize("N,K", [(1000, 2), (118800, 3), (600000, 4)])
+def test_group_cooperative_and_multi_launch_paths(N, K):
+    """lipar_group runs as one cooperative launch with the recommended
+    workspace (N within one launch) and as the multi-launch radix path with the
+    minimum workspace; both equal the oracle's rank split, ties included."""
+    s = synth.random_scores(N, 300 + N, ties=True, specials=True)
+    ref = O.group_split(s.numpy(), K)
+    sd = s.to(DEV)
+    for ws in (tps.workspace(tps.OP_GROUP, N, K, DEV), tps.workspace(tps.OP_GROUP, N, K, DEV, minimal=True)):
+        g = tps.lipar_group(sd, K, ws=ws).cpu().numpy()
+        assert np.array_equal(g, ref), ws.numel()
+    tps.tps_check()
+
+
+# ------------------------------------------------- fused front end ----------
+@pytest.mark.parametrize("name", ["tiny", "mid", "block"])
+def test_front_interframe_matches_separate_stages(name):
+    """lipar_front = lipar_score + lipar_select: the same scores bit for bit
+    and the oracle's index list."""
+    cfg, xb, k = frame_case(name)
+    x = xb.to(DEV)
+    ref_s = tps.lipar_score(x).cpu()
+    s = torch.full((cfg.video.N,), 7.0, device=DEV)
+    if k is None:
+        idx, cnt = tps.lipar_front(x, tps.FRONT_THRESHOLD, tau=cfg.tau, score=s)
+    else:
+        idx, cnt = tps.lipar_front(x, tps.FRONT_TOPK, k=k, score=s)
+    assert torch.equal(s.cpu(), ref_s)
+    assert np.array_equal(_idx(idx, cnt), oracle_idx(name))
+    tps.tps_check()
+
+
+def test_front_interstep_keep_sweep_and_hsa_groups():
+    cfg, vpb, vc, _ = step_case("wan")
+    F, HW, C = cfg.video.F, cfg.video.HW, cfg.video.C
+    cur, prev = vc.reshape(F, HW, C).to(DEV), vpb.reshape(F, HW, C).to(DEV)
+    ws = tps.workspace(tps.OP_FRONT, cfg.video.N, 0, DEV)
+    for i, r in enumerate(cfg.keep):
+        k = synth.keep_count(cfg.video.N, r)
+        idx, cnt = tps.lipar_front(cur, tps.FRONT_TOPK, x_ref=prev, k=k, ws=ws)
+        assert np.array_equal(_idx(idx, cnt), oracle_idx("wan", i))
+    cfg, vpb, vc, _ = step_case("hsa")
+    F, HW, C = cfg.video.F, cfg.video.HW, cfg.video.C
+    K = cfg.extra["K"]
+    cur, prev = vc.reshape(F, HW, C).to(DEV), vpb.reshape(F, HW, C).to(DEV)
+    s = torch.empty(cfg.video.N, device=DEV)
+    g = tps.lipar_front(cur, tps.FRONT_GROUP, x_ref=prev, K=K, score=s).cpu().numpy()
+    assert torch.equal(s.cpu(), tps.lipar_score(cur, prev).cpu())
+    assert np.array_equal(g, O.group_split(O.lipar_score(vc[None], vpb[None]), K))
+    tps.tps_check()
+
+
+@pytest.mark.parametrize("F,HW,C", [(3, 700, 64), (2, 70000, 128), (5, 130000, 128), (4, 33, 96)])
+def test_front_sizes_prev_frame_and_fallback(F, HW, C):
+    """Both cooperative tilings (N <= 131072 and larger), the separate-kernel
+    path (N beyond one cooperative launch, or C outside {64, 128}), the
+    streaming case with a previous frame, and zero change."""
+    x = synth.gaussian_bf16((F, HW, C), F * HW + C)
+    prev = synth.gaussian_bf16((HW, C), 5)
+    N = F * HW
+    xd, pd = x.to(DEV), prev.to(DEV)
+    for xp in (None, pd):
+        s_ref = tps.lipar_score(xd, x_prev_frame=xp)
+        for k in (1, N // 3, N):
+            idx, cnt = tps.lipar_front(xd, tps.FRONT_TOPK, x_prev_frame=xp, k=k)
+            ridx, rcnt = tps.lipar_select(s_ref, tps.SELECT_TOPK, k=k)
+            n = int(rcnt.item())
+            assert int(cnt.item()) == n and torch.equal(idx[:n], ridx[:n]), (xp is None, k)
+        idx, cnt = tps.lipar_front(xd, tps.FRONT_THRESHOLD, x_prev_frame=xp, tau=1.0)
+        ridx, rcnt = tps.lipar_select(s_ref, tps.SELECT_THRESHOLD, tau=1.0)
+        n = int(rcnt.item())
+        assert int(cnt.item()) == n and torch.equal(idx[:n], ridx[:n])
+        for K in (1, 3):
+            g = tps.lipar_front(xd, tps.FRONT_GROUP, x_prev_frame=xp, K=K)
+            assert torch.equal(g, tps.lipar_group(s_ref, K))
+    same = x[:1].expand(F, HW, C).contiguous().to(DEV)
+    idx, cnt = tps.lipar_front(same, tps.FRONT_THRESHOLD, x_prev_frame=same[0], tau=1e-6)
+    assert int(cnt.item()) == 0
+    tps.tps_check()

@@ -362,40 +362,58 @@ __global__ void __launch_bounds__(kThreads) group_write(const float* __restrict_
   }
 }
 
-// ---- single-launch cooperative path (threshold, top-k, schedule) ----------------------
-// For N up to 256 blocks of 2048 elements the whole selection runs as ONE
+// ---- single-launch cooperative path (threshold, top-k, schedule, group) -------------
+// For N up to 256 blocks of 256*kItems elements the whole selection runs as ONE
 // cooperative launch (all blocks co-resident, guaranteed by the launch): each
-// block keeps its 2048 keys in registers; the four radix passes and the final
-// compaction are separated by grid barriers. A barrier is a counter in the
-// workspace (zeroed before the launch) that thread 0 of every block increments
-// and then polls; each poll loop is bounded by clock64 and, if it expires, sets
-// the device status word (TPS_ERR_TIMEOUT) and the block leaves without
-// writing results.
+// block keeps its keys in registers; the four radix passes and the final
+// compaction (or, for groups, the tie ranking) are separated by grid barriers.
+// A barrier is a counter in the workspace (zeroed before the launch) that
+// thread 0 of every block increments and then polls; each poll loop is bounded
+// by clock64 and, if it expires, sets the device status word (TPS_ERR_TIMEOUT)
+// and the block leaves without writing results.
+//
+// With kV > 0 the launch also computes the scores (the fused front end,
+// lipar_front): every block first scores its own tokens -- the relative L1
+// change, with the same lane layout and summation order as lipar_score, so
+// the scores are bit-identical -- into shared memory, and the selection reads
+// them from there: the scores never make a round trip through global memory
+// between the two stages.
 constexpr int kCoopItems = 8;
-constexpr int kCoopTile = kThreads * kCoopItems;   // elements per block
 constexpr int kCoopMaxBlocks = 256;
 constexpr long long kGridWaitCycles = 2000000000LL; // ~1 s
 constexpr int kCoopHdrWords = 64;                   // barrier counter + padding
 
-enum CoopMode { kCoopThresh = 0, kCoopTopk = 1, kCoopSched = 2 };
+enum CoopMode { kCoopThresh = 0, kCoopTopk = 1, kCoopSched = 2, kCoopGroup = 3 };
 
 struct CoopArgs {
-  const float* s;
+  const float* s;          // scores (kV == 0)
   float tau;
-  const int8_t* g;
+  const int8_t* g;         // groups (schedule)
   unsigned int act;
   int K;
   unsigned int k;          // top-k target (>= 1)
+  int nbound;              // group: rank cuts (K - 1)
+  unsigned int cuts[kMaxBound];
+  int8_t* group;           // group: output
+  const uint16_t* x;       // kV > 0: the tokens to score (as lipar_score)
+  const uint16_t* xref;
+  const uint16_t* xprev;
+  int64_t HW;
+  float* score_out;        // kV > 0: optional copy of the scores
 };
 
-inline int64_t coop_blocks(int64_t N) { return (N + kCoopTile - 1) / kCoopTile; }
-// Workspace: header (barrier counter), one 256-bin histogram per radix pass
-// (summed with atomics; zeroed together with the header before the launch),
-// then two counts per block.
-constexpr int kCoopZeroWords = kCoopHdrWords + 4 * 256;
-inline size_t coop_bytes(int64_t N, int mode) {
-  (void)mode;
-  return kCoopZeroWords * 4 + coop_blocks(N) * 2 * 4;
+inline int64_t coop_blocks(int64_t N, int items = kCoopItems) {
+  return (N + kThreads * items - 1) / (kThreads * items);
+}
+// Workspace: header (barrier counter), the radix histograms (one 256-bin
+// histogram per pass and cut, summed with atomics; zeroed with the header
+// before the launch), then the per-block count columns.
+__host__ __device__ inline int coop_zero_words(int mode, int nbound) {
+  return kCoopHdrWords + (mode == kCoopGroup ? 4 * nbound * 256 : 4 * 256);
+}
+inline int coop_cols(int mode, int nbound) { return mode == kCoopGroup ? nbound : 2; }
+inline size_t coop_bytes(int64_t G, int mode, int nbound) {
+  return static_cast<size_t>(coop_zero_words(mode, nbound)) * 4 + static_cast<size_t>(G) * coop_cols(mode, nbound) * 4;
 }
 
 __device__ __forceinline__ bool grid_sync(unsigned int* bar, unsigned int target, unsigned int* status,
@@ -418,80 +436,221 @@ __device__ __forceinline__ bool grid_sync(unsigned int* bar, unsigned int target
   return *s_fail == 0;
 }
 
-template <int kMode>
+// Scores of this block's tokens into s_sc (fused front end). Eight lanes per
+// token, 16-byte vectors, the same per-lane order and xor-shuffle reduction as
+// score_kernel<8, kV, *>, hence the same fp32 result.
+template <int kItems, int kV>
+__device__ __forceinline__ void score_tile(const CoopArgs& a, int64_t N, float* s_sc) {
+  constexpr int L = 8, kTokW = 32 / L, C = kV * 8;
+  constexpr int kTileC = kThreads * kItems;
+  constexpr int kSteps = kTileC / (kWarps * kTokW);
+  constexpr int kG = 4;
+  static_assert(kSteps % kG == 0, "score steps");
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, sub = lane & (L - 1);
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileC;
+  for (int s0 = 0; s0 < kSteps; s0 += kG) {
+    const uint16_t* cur[kG];
+    const uint16_t* ref[kG];
+    int jj[kG];
+    bool valid[kG];
+#pragma unroll
+    for (int q = 0; q < kG; ++q) {
+      const int j = ((s0 + q) * kWarps + w) * kTokW + lane / L;
+      const int64_t t = t0 + j;
+      jj[q] = j;
+      valid[q] = t < N;
+      ref[q] = nullptr;
+      cur[q] = a.x + (valid[q] ? t : 0) * C;
+      if (valid[q]) {
+        if (a.xref) ref[q] = a.xref + t * C;
+        else if (t >= a.HW) ref[q] = a.x + (t - a.HW) * C;
+        else if (a.xprev) ref[q] = a.xprev + t * C;
+      }
+    }
+    float num[kG], den[kG];
+#pragma unroll
+    for (int q = 0; q < kG; ++q) num[q] = 0.f, den[q] = 0.f;
+#pragma unroll
+    for (int v = sub; v < kV; v += L) {
+      uint4 ca[kG], cb[kG];
+#pragma unroll
+      for (int q = 0; q < kG; ++q)
+        if (ref[q]) {
+          ca[q] = ld16(cur[q] + v * 8);
+          cb[q] = ld16(ref[q] + v * 8);
+        }
+#pragma unroll
+      for (int q = 0; q < kG; ++q)
+        if (ref[q]) {
+          const uint32_t aw[4] = {ca[q].x, ca[q].y, ca[q].z, ca[q].w};
+          const uint32_t bw[4] = {cb[q].x, cb[q].y, cb[q].z, cb[q].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float c0 = bf16lo(aw[i]), c1 = bf16hi(aw[i]);
+            const float r0 = bf16lo(bw[i]), r1 = bf16hi(bw[i]);
+            num[q] += fabsf(c0 - r0) + fabsf(c1 - r1);
+            den[q] += fabsf(r0) + fabsf(r1);
+          }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kG; ++q) {
+#pragma unroll
+      for (int o = L / 2; o > 0; o >>= 1) {
+        num[q] += __shfl_xor_sync(0xffffffffu, num[q], o);
+        den[q] += __shfl_xor_sync(0xffffffffu, den[q], o);
+      }
+      if (valid[q] && sub == 0) {
+        float s;
+        if (!ref[q]) s = INFINITY;                  // frame 0 without a predecessor
+        else if (den[q] > 0.f) s = num[q] / den[q];
+        else s = num[q] > 0.f ? INFINITY : 0.f;
+        s_sc[jj[q]] = s;
+        if (a.score_out) a.score_out[t0 + jj[q]] = s;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <int kMode, int kItems, int kV>
 __global__ void __launch_bounds__(kThreads) select_coop(CoopArgs a, int64_t N, unsigned int* ws,
                                                         int32_t* __restrict__ idx, int32_t* __restrict__ count,
                                                         unsigned int* status) {
-  __shared__ unsigned int sh[256];
-  __shared__ unsigned int s_pref, s_krem;
+  constexpr int kTileC = kThreads * kItems;
+  constexpr int kCuts = kMode == kCoopGroup ? kMaxBound : 1;
+  __shared__ unsigned int sh[kCuts][256];
+  __shared__ float s_sc[kV > 0 ? kTileC : 1];
+  __shared__ unsigned int s_pref[kCuts], s_krem[kCuts];
   __shared__ volatile int s_fail;
   __shared__ unsigned int s_sel[kWarps], s_tie[kWarps];
+  __shared__ unsigned int s_eq[kCuts][kWarps];
   const unsigned int G = gridDim.x, b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nbound = kMode == kCoopGroup ? a.nbound : 1;
   unsigned int* bar = ws;
-  unsigned int* hist = ws + kCoopHdrWords;                       // [4][256], top-k only
-  unsigned int* cnt = ws + kCoopZeroWords;                       // [G][2]
+  unsigned int* hist = ws + kCoopHdrWords;                       // [4][cuts][256]
+  unsigned int* cnt = ws + coop_zero_words(kMode, nbound);       // [G][cols]
   if (tid == 0) s_fail = 0;
-  const int64_t base = static_cast<int64_t>(b) * kCoopTile + w * (32 * kCoopItems);
-  uint32_t key[kCoopItems];
-  int cls[kCoopItems];
+  if constexpr (kV > 0) score_tile<kItems, kV>(a, N, s_sc);
+  const int64_t base = static_cast<int64_t>(b) * kTileC + w * (32 * kItems);
+  uint32_t key[kItems];
+  int cls[kItems];
 #pragma unroll
-  for (int it = 0; it < kCoopItems; ++it) {
+  for (int it = 0; it < kItems; ++it) {
     const int64_t n = base + it * 32 + lane;
     key[it] = 0u;
     cls[it] = 0;
     if (n < N) {
-      if (kMode == kCoopTopk) key[it] = score_key(a.s[n]);
-      else if (kMode == kCoopThresh) cls[it] = a.s[n] >= a.tau ? 1 : 0;
-      else {
+      if (kMode == kCoopSched) {
         const int v = a.g[n];
         cls[it] = (v >= 0 && v < a.K && ((a.act >> v) & 1u)) ? 1 : 0;
+      } else {
+        const float sv = kV > 0 ? s_sc[w * (32 * kItems) + it * 32 + lane] : a.s[n];
+        if (kMode == kCoopThresh) cls[it] = sv >= a.tau ? 1 : 0;
+        else key[it] = score_key(sv);
       }
     }
   }
   unsigned int nbar = 0;
   unsigned int krem = 0;
-  if (kMode == kCoopTopk) {
-    unsigned int prefix = 0;
-    krem = a.k;
+  if (kMode == kCoopTopk || kMode == kCoopGroup) {
+    // MSB-first radix select of every cut at once: four 8-bit digits
+    if (tid < nbound) {
+      s_pref[tid] = 0u;
+      s_krem[tid] = kMode == kCoopTopk ? a.k : a.cuts[tid];
+    }
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       const unsigned int himask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
-      sh[tid] = 0u;
+      for (int c = 0; c < nbound; ++c) sh[c][tid] = 0u;
       __syncthreads();
 #pragma unroll
-      for (int it = 0; it < kCoopItems; ++it) {
+      for (int it = 0; it < kItems; ++it) {
         const int64_t n = base + it * 32 + lane;
-        if (n < N && (key[it] & himask) == prefix) atomicAdd(&sh[(key[it] >> shift) & 255u], 1u);
+        if (n < N)
+          for (int c = 0; c < nbound; ++c)
+            if ((key[it] & himask) == s_pref[c]) atomicAdd(&sh[c][(key[it] >> shift) & 255u], 1u);
       }
       __syncthreads();
-      if (sh[tid]) atomicAdd(&hist[pass * 256u + tid], sh[tid]);   // one global histogram per pass
+      for (int c = 0; c < nbound; ++c)
+        if (sh[c][tid]) atomicAdd(&hist[(pass * nbound + c) * 256u + tid], sh[c][tid]);   // one global histogram per pass and cut
       if (!grid_sync(bar, ++nbar * G, status, &s_fail)) return;
-      const int bin = 255 - tid;                                  // descending buckets
-      const unsigned int c = __ldcg(&hist[pass * 256u + bin]);
-      unsigned int tot;
-      const unsigned int incl = block_incl_scan(c, &tot);
-      const unsigned int excl = incl - c;
-      if (excl < krem && incl >= krem) {
-        s_pref = prefix | (static_cast<unsigned int>(bin) << shift);
-        s_krem = krem - excl;
+      for (int c = 0; c < nbound; ++c) {
+        const unsigned int need = s_krem[c], pre = s_pref[c];
+        const int bin = 255 - tid;                                // descending buckets
+        const unsigned int v = __ldcg(&hist[(pass * nbound + c) * 256u + bin]);
+        unsigned int tot;
+        const unsigned int incl = block_incl_scan(v, &tot);
+        const unsigned int excl = incl - v;
+        if (excl < need && incl >= need) {
+          s_pref[c] = pre | (static_cast<unsigned int>(bin) << shift);
+          s_krem[c] = need - excl;
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      prefix = s_pref;
-      krem = s_krem;
-      __syncthreads();
     }
+    if (kMode == kCoopTopk) {
+      const unsigned int prefix = s_pref[0];
+      krem = s_krem[0];
 #pragma unroll
-    for (int it = 0; it < kCoopItems; ++it) {
-      const int64_t n = base + it * 32 + lane;
-      cls[it] = n >= N ? 0 : (key[it] > prefix ? 1 : (key[it] == prefix ? 2 : 0));
+      for (int it = 0; it < kItems; ++it) {
+        const int64_t n = base + it * 32 + lane;
+        cls[it] = n >= N ? 0 : (key[it] > prefix ? 1 : (key[it] == prefix ? 2 : 0));
+      }
     }
   }
+  const unsigned int lt = (1u << lane) - 1u;
+  if constexpr (kMode == kCoopGroup) {
+    // ---- group: rank of each token among the ties at every cut, in index order
+    for (int c = 0; c < nbound; ++c) {
+      const unsigned int ks = s_pref[c];
+      unsigned int weq = 0;
+#pragma unroll
+      for (int it = 0; it < kItems; ++it) {
+        const int64_t n = base + it * 32 + lane;
+        weq += __popc(__ballot_sync(0xffffffffu, n < N && key[it] == ks));
+      }
+      if (lane == 0) s_eq[c][w] = weq;
+    }
+    __syncthreads();
+    if (tid < nbound) {
+      unsigned int t = 0;
+      for (int i = 0; i < kWarps; ++i) t += s_eq[tid][i];
+      cnt[b * nbound + tid] = t;
+    }
+    if (!grid_sync(bar, ++nbar * G, status, &s_fail)) return;
+    int grp[kItems];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) grp[it] = 0;
+    for (int c = 0; c < nbound; ++c) {
+      unsigned int ps = 0;
+      for (unsigned int g = tid; g < b; g += kThreads) ps += __ldcg(&cnt[g * nbound + c]);
+      unsigned int eb = block_sum(ps);
+      for (int i = 0; i < w; ++i) eb += s_eq[c][i];
+      const unsigned int ks = s_pref[c], kr = s_krem[c];
+#pragma unroll
+      for (int it = 0; it < kItems; ++it) {
+        const int64_t n = base + it * 32 + lane;
+        const unsigned int m = __ballot_sync(0xffffffffu, n < N && key[it] == ks);
+        const unsigned int r = eb + __popc(m & lt);
+        const bool above = key[it] > ks || (key[it] == ks && r < kr);
+        grp[it] += above ? 0 : 1;
+        eb += __popc(m);
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int64_t n = base + it * 32 + lane;
+      if (n < N) a.group[n] = static_cast<int8_t>(grp[it]);
+    }
+    return;
+  }
   // ---- compaction ------------------------------------------------------------------
-  unsigned int msel[kCoopItems], mtie[kCoopItems];
+  unsigned int msel[kItems], mtie[kItems];
   unsigned int wsel = 0, wtie = 0;
 #pragma unroll
-  for (int it = 0; it < kCoopItems; ++it) {
+  for (int it = 0; it < kItems; ++it) {
     msel[it] = __ballot_sync(0xffffffffu, cls[it] == 1);
     mtie[it] = __ballot_sync(0xffffffffu, cls[it] == 2);
     wsel += __popc(msel[it]);
@@ -534,9 +693,8 @@ __global__ void __launch_bounds__(kThreads) select_coop(CoopArgs a, int64_t N, u
     sb += s_sel[i];
     tb += s_tie[i];
   }
-  const unsigned int lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int it = 0; it < kCoopItems; ++it) {
+  for (int it = 0; it < kItems; ++it) {
     const int64_t n = base + it * 32 + lane;
     const unsigned int sr = sb + __popc(msel[it] & lt);
     const unsigned int tr = tb + __popc(mtie[it] & lt);
@@ -548,7 +706,7 @@ __global__ void __launch_bounds__(kThreads) select_coop(CoopArgs a, int64_t N, u
 }
 
 // Max co-resident blocks of a cooperative kernel on the current device (cached).
-template <int kMode>
+template <int kMode, int kItems, int kV>
 int coop_capacity() {
   static std::atomic<int> cap[64];   // per device; two threads may both compute it, to the same value
   int dev = 0;
@@ -557,7 +715,8 @@ int coop_capacity() {
   if (!c) {
     int per_sm = 0, coop = 0;
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_coop<kMode>, kThreads, 0) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_coop<kMode, kItems, kV>, kThreads, 0) !=
+        cudaSuccess)
       return 0;
     c = per_sm * sm_count();
     cap[dev].store(c, std::memory_order_relaxed);
@@ -566,20 +725,24 @@ int coop_capacity() {
 }
 
 // Runs the cooperative path when it applies; returns -1 when it does not.
-template <int kMode>
+template <int kMode, int kItems = kCoopItems, int kV = 0>
 int try_coop(const CoopArgs& ca, int64_t N, void* ws, size_t ws_bytes, int32_t* idx, int32_t* count,
              cudaStream_t st) {
-  const int64_t G = coop_blocks(N);
-  if (G > kCoopMaxBlocks || G > coop_capacity<kMode>() || ws_bytes < coop_bytes(N, kMode)) return -1;
+  const int64_t G = coop_blocks(N, kItems);
+  const int nbound = kMode == kCoopGroup ? ca.nbound : 1;
+  if (G > kCoopMaxBlocks || G > coop_capacity<kMode, kItems, kV>() || ws_bytes < coop_bytes(G, kMode, nbound))
+    return -1;
   int err;
   unsigned int* status = device_status(&err);
   if (!status) return err;
-  if (int e = cuda_status(cudaMemsetAsync(ws, 0, kCoopZeroWords * 4, st), "selection: clear barrier")) return e;
+  if (int e = cuda_status(cudaMemsetAsync(ws, 0, static_cast<size_t>(coop_zero_words(kMode, nbound)) * 4, st),
+                          "selection: clear barrier"))
+    return e;
   CoopArgs a = ca;
   int64_t n = N;
   unsigned int* w = static_cast<unsigned int*>(ws);
   void* args[] = {&a, &n, &w, &idx, &count, &status};
-  cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_coop<kMode>),
+  cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_coop<kMode, kItems, kV>),
                                               dim3(static_cast<unsigned int>(G)), dim3(kThreads), args, 0, st);
   return cuda_status(e, "selection: cooperative launch");
 }
@@ -607,8 +770,10 @@ size_t ws_min_bytes(int op, int64_t N, int K) {
 size_t ws_bytes_for(int op, int64_t N, int K) {
   const size_t classic = ws_min_bytes(op, N, K);
   size_t coop = 0;
-  if (op != TPS_OP_GROUP && coop_blocks(N > 0 ? N : 1) <= kCoopMaxBlocks)
-    coop = coop_bytes(N > 0 ? N : 1, op == TPS_OP_SELECT ? kCoopTopk : kCoopSched);
+  const int64_t G = coop_blocks(N > 0 ? N : 1);
+  if (G <= kCoopMaxBlocks)
+    coop = op == TPS_OP_GROUP ? coop_bytes(G, kCoopGroup, K > 1 ? K - 1 : 1)
+                              : coop_bytes(G, op == TPS_OP_SELECT ? kCoopTopk : kCoopSched, 1);
   return classic > coop ? classic : coop;
 }
 
@@ -653,15 +818,39 @@ int run_compact(const Cls& cls, int64_t N, const WsView& v, int ncol, int32_t* i
 }  // namespace
 }  // namespace tps
 
+namespace tps {
+namespace {
+// lipar_front: a score scratch (used only when the fused launch does not apply
+// and the caller passes no score array), then the selection / group workspace.
+size_t front_score_bytes(int64_t N) { return (static_cast<size_t>(N > 0 ? N : 1) * 4 + 255) / 256 * 256; }
+size_t front_min_bytes(int64_t N, int K) {
+  const size_t a = ws_min_bytes(TPS_OP_SELECT, N, 0), b = ws_min_bytes(TPS_OP_GROUP, N, K);
+  return front_score_bytes(N) + (a > b ? a : b);
+}
+size_t front_bytes(int64_t N, int K) {
+  size_t m = ws_bytes_for(TPS_OP_SELECT, N, 0);
+  const size_t g = ws_bytes_for(TPS_OP_GROUP, N, K);
+  m = m > g ? m : g;
+  const size_t f1 = coop_bytes(kCoopMaxBlocks, kCoopTopk, 1);
+  const size_t f2 = coop_bytes(kCoopMaxBlocks, kCoopGroup, K > 1 ? (K - 1 < kMaxBound ? K - 1 : kMaxBound) : 1);
+  m = m > f1 ? m : f1;
+  m = m > f2 ? m : f2;
+  return front_score_bytes(N) + m;
+}
+}  // namespace
+}  // namespace tps
+
 extern "C" size_t tps_workspace_size(int op, int64_t N, int K) {
-  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
   if (N < 0) return 0;
+  if (op == TPS_OP_FRONT) return tps::front_bytes(N, K);
+  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
   return tps::ws_bytes_for(op, N, K);
 }
 
 extern "C" size_t tps_workspace_min_size(int op, int64_t N, int K) {
-  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
   if (N < 0) return 0;
+  if (op == TPS_OP_FRONT) return tps::front_min_bytes(N, K);
+  if (op != TPS_OP_SELECT && op != TPS_OP_GROUP && op != TPS_OP_SCHEDULE) return 0;
   return tps::ws_min_bytes(op, N, K);
 }
 
@@ -686,7 +875,10 @@ extern "C" int lipar_select(const float* score, int64_t N, int mode, float tau, 
   if (int e = check_ws(ws, ws_bytes, TPS_OP_SELECT, N, 0, &v, "lipar_select")) return e;
   int e;
   {
-    CoopArgs ca{score, tau, nullptr, 0u, 0, static_cast<unsigned int>(k)};
+    CoopArgs ca{};
+    ca.s = score;
+    ca.tau = tau;
+    ca.k = static_cast<unsigned int>(k);
     e = mode == TPS_SELECT_THRESHOLD ? try_coop<kCoopThresh>(ca, N, ws, ws_bytes, idx, count, st)
                                      : try_coop<kCoopTopk>(ca, N, ws, ws_bytes, idx, count, st);
     if (e >= 0) return e ? e : ok();
@@ -721,12 +913,97 @@ extern "C" int lipar_group(const float* score, int64_t N, int K, int8_t* group, 
   Cuts c{};
   const int64_t size = N / K;
   for (int b = 0; b < nbound; ++b) c.k[b] = static_cast<unsigned int>((b + 1) * size);
+  {
+    CoopArgs ca{};
+    ca.s = score;
+    ca.nbound = nbound;
+    for (int b = 0; b < nbound; ++b) ca.cuts[b] = c.k[b];
+    ca.group = group;
+    const int e = try_coop<kCoopGroup>(ca, N, ws, ws_bytes, nullptr, nullptr, st);
+    if (e >= 0) return e ? e : ok();
+  }
   if (int e = run_radix(score, N, v.hdr, nbound, c, st)) return e;
   const unsigned int nb = static_cast<unsigned int>(n_blocks(N));
   group_count<<<nb, kThreads, 0, st>>>(score, N, v.hdr, nbound, v.cnt, v.off);
   group_write<<<nb, kThreads, 0, st>>>(score, N, v.hdr, nbound, v.off, group);
   if (int e = launch_status("lipar_group")) return e;
   return ok();
+}
+
+// ---- fused front end: score + selection (or group split) in one launch -------------
+namespace tps {
+namespace {
+template <int kMode, int kV>
+int front_coop(const CoopArgs& ca, int64_t N, void* ws, size_t ws_bytes, int32_t* idx, int32_t* count,
+               cudaStream_t st) {
+  if (coop_blocks(N, 2) <= kCoopMaxBlocks) return try_coop<kMode, 2, kV>(ca, N, ws, ws_bytes, idx, count, st);
+  return try_coop<kMode, kCoopItems, kV>(ca, N, ws, ws_bytes, idx, count, st);
+}
+template <int kV>
+int front_dispatch(int mode, const CoopArgs& ca, int64_t N, void* ws, size_t ws_bytes, int32_t* idx,
+                   int32_t* count, cudaStream_t st) {
+  if (mode == TPS_FRONT_THRESHOLD) return front_coop<kCoopThresh, kV>(ca, N, ws, ws_bytes, idx, count, st);
+  if (mode == TPS_FRONT_TOPK) return front_coop<kCoopTopk, kV>(ca, N, ws, ws_bytes, idx, count, st);
+  return front_coop<kCoopGroup, kV>(ca, N, ws, ws_bytes, idx, count, st);
+}
+}  // namespace
+}  // namespace tps
+
+extern "C" int lipar_front(const tps_bf16* x, const tps_bf16* x_ref, const tps_bf16* x_prev_frame, int64_t F,
+                           int64_t HW, int64_t C, int mode, float tau, int64_t k, int K, float* score,
+                           int32_t* idx, int32_t* count, int8_t* group, void* ws, size_t ws_bytes,
+                           tps_stream stream) {
+  TPS_TRACE("lipar_front");
+  using namespace tps;
+  if (!x) return fail(TPS_ERR_INVALID_ARG, "lipar_front: x must be non-null");
+  if (F < 1 || HW < 1 || F > (INT64_C(1) << 31) / HW)
+    return fail(TPS_ERR_SHAPE, "lipar_front: need F, HW >= 1 and F*HW < 2^31");
+  if (C < 8 || C > 4096 || C % 8) return fail(TPS_ERR_SHAPE, "lipar_front: C=%lld must be a multiple of 8 in [8, 4096]", (long long)C);
+  if (x_ref && x_prev_frame) return fail(TPS_ERR_INVALID_ARG, "lipar_front: x_prev_frame is for inter-frame mode only");
+  const int64_t N = F * HW;
+  if (mode == TPS_FRONT_THRESHOLD || mode == TPS_FRONT_TOPK) {
+    if (!idx || !count) return fail(TPS_ERR_INVALID_ARG, "lipar_front: idx and count must be non-null");
+    if (mode == TPS_FRONT_TOPK && (k < 0 || k > N))
+      return fail(TPS_ERR_INVALID_ARG, "lipar_front: k=%lld not in [0, N=%lld]", (long long)k, (long long)N);
+  } else if (mode == TPS_FRONT_GROUP) {
+    if (!group) return fail(TPS_ERR_INVALID_ARG, "lipar_front: group must be non-null");
+    if (K < 1 || K > kMaxBound + 1 || K > N)
+      return fail(TPS_ERR_INVALID_ARG, "lipar_front: K=%d must be in [1, 8] and <= N", K);
+  } else {
+    return fail(TPS_ERR_INVALID_ARG, "lipar_front: mode %d is not 0 (threshold), 1 (top-k) or 2 (group)", mode);
+  }
+  if (!aligned16(x) || (x_ref && !aligned16(x_ref)) || (x_prev_frame && !aligned16(x_prev_frame)))
+    return fail(TPS_ERR_ALIGN, "lipar_front: bf16 inputs must be 16-byte aligned");
+  if (!ws) return fail(TPS_ERR_WORKSPACE, "lipar_front: workspace is null");
+  if (!aligned16(ws)) return fail(TPS_ERR_ALIGN, "lipar_front: workspace must be 16-byte aligned");
+  if (ws_bytes < front_min_bytes(N, K))
+    return fail(TPS_ERR_WORKSPACE, "lipar_front: workspace %zu bytes < required %zu", ws_bytes, front_min_bytes(N, K));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool trivial = (mode == TPS_FRONT_TOPK && k == 0) || (mode == TPS_FRONT_GROUP && K == 1);
+  if ((C == 128 || C == 64) && !trivial) {
+    CoopArgs ca{};
+    ca.tau = tau;
+    ca.k = static_cast<unsigned int>(k);
+    ca.nbound = mode == TPS_FRONT_GROUP ? K - 1 : 1;
+    for (int b = 0; b + 1 < K && b < kMaxBound; ++b) ca.cuts[b] = static_cast<unsigned int>((b + 1) * (N / K));
+    ca.group = group;
+    ca.x = x;
+    ca.xref = x_ref;
+    ca.xprev = x_prev_frame;
+    ca.HW = HW;
+    ca.score_out = score;
+    const int e = C == 128 ? front_dispatch<16>(mode, ca, N, ws, ws_bytes, idx, count, st)
+                           : front_dispatch<8>(mode, ca, N, ws, ws_bytes, idx, count, st);
+    if (e >= 0) return e ? e : ok();
+  }
+  // the separate kernels, with the scores in the caller's array or the workspace
+  float* sbuf = score ? score : static_cast<float*>(ws);
+  void* ws2 = static_cast<char*>(ws) + front_score_bytes(N);
+  const size_t ws2_bytes = ws_bytes - front_score_bytes(N);
+  if (int e = lipar_score(x, x_ref, x_prev_frame, F, HW, C, sbuf, stream)) return e;
+  if (mode == TPS_FRONT_GROUP) return lipar_group(sbuf, N, K, group, ws2, ws2_bytes, stream);
+  return lipar_select(sbuf, N, mode == TPS_FRONT_TOPK ? TPS_SELECT_TOPK : TPS_SELECT_THRESHOLD, tau, k, idx, count,
+                      ws2, ws2_bytes, stream);
 }
 
 extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32_t* budgets, int T,
@@ -756,7 +1033,10 @@ extern "C" int lipar_schedule(const int8_t* group, int64_t N, int K, const int32
   WsView v;
   if (int e = check_ws(ws, ws_bytes, TPS_OP_SCHEDULE, N, K, &v, "lipar_schedule")) return e;
   {
-    CoopArgs ca{nullptr, 0.f, group, act, K, 0u};
+    CoopArgs ca{};
+    ca.g = group;
+    ca.act = act;
+    ca.K = K;
     const int e = try_coop<kCoopSched>(ca, N, ws, ws_bytes, idx, count, st);
     if (e >= 0) return e ? e : ok();
   }

@@ -18,7 +18,8 @@ _lib = None
 
 OK, INVALID_ARG, SHAPE, ALIGN, CUDA, TIMEOUT, BOUNDS, WORKSPACE = range(8)
 SELECT_THRESHOLD, SELECT_TOPK = 0, 1
-OP_SELECT, OP_GROUP, OP_SCHEDULE = 0, 1, 2
+OP_SELECT, OP_GROUP, OP_SCHEDULE, OP_FRONT = 0, 1, 2, 3
+FRONT_THRESHOLD, FRONT_TOPK, FRONT_GROUP = 0, 1, 2
 
 _P = C.c_void_p
 _I64 = C.c_int64
@@ -29,6 +30,8 @@ SIGNATURES = {
     "lipar_score": (_INT, [_P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "lipar_select": (_INT, [_P, _I64, _INT, C.c_float, _I64, _P, _P, _P, C.c_size_t, _P]),
     "lipar_select_static": (_INT, [_P, _I64, _INT, C.c_float, _I64, _P, _P, _P]),
+    "lipar_front": (_INT, [_P, _P, _P, _I64, _I64, _I64, _INT, C.c_float, _I64, _INT, _P, _P, _P, _P, _P,
+                           C.c_size_t, _P]),
     "lipar_group": (_INT, [_P, _I64, _INT, _P, _P, C.c_size_t, _P]),
     "lipar_schedule": (_INT, [_P, _I64, _INT, _P, _INT, _INT, _INT, _P, _P, _P, C.c_size_t, _P]),
     "tps_gather_rows": (_INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -151,6 +154,30 @@ def lipar_select_static(score, mode, tau=0.0, k=0, idx=None, count=None, stream=
     _chk(lib().lipar_select_static(_ptr(score), N, mode, float(tau), int(k), _ptr(idx), _ptr(count),
                                    _stream(stream)))
     return idx, count
+
+
+def lipar_front(x, mode, x_ref=None, x_prev_frame=None, tau=0.0, k=0, K=1, score=None, idx=None, count=None,
+                group=None, ws=None, stream=None):
+    """Score + selection (mode FRONT_THRESHOLD / FRONT_TOPK -> (idx, count)) or
+    score + group split (FRONT_GROUP -> group), in one launch where it applies.
+    x [F, HW, C] bf16. Pass a tensor as `score` to also receive the scores."""
+    F, HW, Cc = x.shape
+    N = F * HW
+    dev = x.device
+    if mode == FRONT_GROUP:
+        if group is None:
+            group = torch.empty(N, dtype=torch.int8, device=dev)
+    else:
+        if idx is None:
+            idx = torch.empty(max(N if mode == FRONT_THRESHOLD else k, 1), dtype=torch.int32, device=dev)
+        if count is None:
+            count = torch.empty(1, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(OP_FRONT, N, K, dev)
+    _chk(lib().lipar_front(_ptr(x), _ptr(x_ref), _ptr(x_prev_frame), F, HW, Cc, int(mode), float(tau), int(k),
+                           int(K), _ptr(score), _ptr(idx), _ptr(count), _ptr(group), _ptr(ws), ws.numel(),
+                           _stream(stream)))
+    return group if mode == FRONT_GROUP else (idx, count)
 
 
 def lipar_group(score, K, group=None, ws=None, stream=None):
