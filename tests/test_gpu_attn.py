@@ -32,13 +32,24 @@ def _run(impl, q, k, v, idx, scale, bm=None, with_lse=True, count=None, cap=None
     return o.cpu(), (lse.cpu().numpy() if with_lse else None)
 
 
-def _check(o_gpu, lse_gpu, o_ref, lse_ref, rows=None):
+def _check(o_gpu, lse_gpu, o_ref, lse_ref, rows=None, v_absmax=None):
+    """v_absmax (stress cases with score spikes): the largest |v| per head.
+    Such spikes make single keys dominate, |o| reaches the size of |v| (4 and
+    more), and the bound that the kernel's arithmetic fixes -- probabilities in
+    bf16 (relative error <= 2^-8 each, so <= 2^-8 max|v| in o) plus the bf16
+    output (<= 2^-9 |o|) -- exceeds the absolute 2e-2; those rows are held
+    to that bound (mean-abs stays <= 2e-3)."""
     g = o_gpu.double().numpy()
     if rows is not None:
         g = g[rows]
         lse_gpu = None if lse_gpu is None else lse_gpu[rows]
-    ok, info = attn_tolerance_ok(g, o_ref)
-    assert ok, info
+    if v_absmax is None:
+        ok, info = attn_tolerance_ok(g, o_ref)
+        assert ok, info
+    else:
+        err = np.abs(g - o_ref)
+        bound = np.maximum(2e-2, 2.0 ** -8 * np.asarray(v_absmax)[None, :, None] + 2.0 ** -9 * np.abs(o_ref) + 1e-4)
+        assert np.all(err <= bound) and err.mean() <= 2e-3, dict(max_abs=float(err.max()), mean_abs=float(err.mean()))
     if lse_gpu is not None:
         fin = np.isfinite(lse_ref)
         assert np.array_equal(np.isneginf(lse_gpu), np.isneginf(lse_ref))
@@ -86,7 +97,7 @@ def test_attn_running_max_moves(impl, growth):
     scale = 1.0 / math.sqrt(d)
     o, lse = _run(impl, q, k, v, idx, scale)
     o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
-    _check(o, lse, o_ref, lse_ref)
+    _check(o, lse, o_ref, lse_ref, v_absmax=v.double().abs().amax(dim=(0, 2)).numpy())
 
 
 @pytest.mark.parametrize("impl", IMPLS)
@@ -144,13 +155,14 @@ def test_attn_blockmask_query_block_edges(impl, d):
     bm[1, 15] = 1                                           # block 1 keeps only the ragged last one
     bm[3] = 0                                               # block 3 keeps nothing
     bm[:, 7] = 1
+    vmax = v.double().abs().amax(dim=(0, 2)).numpy()
     o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm)
     o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm)
-    _check(o, lse, o_ref, lse_ref)
+    _check(o, lse, o_ref, lse_ref, v_absmax=vmax)
     c = A - 77
     o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm, count=c)
     o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm, rows=np.arange(c))
-    _check(o[:c], lse[:c], o_ref, lse_ref)
+    _check(o[:c], lse[:c], o_ref, lse_ref, v_absmax=vmax)
     assert torch.all(o[c:].float() == 7.0) and np.all(lse[c:] == 7.0)
 
 
@@ -421,13 +433,14 @@ def test_attn_cluster_split_matches_oracle(N, S, d):
     k = k.to(torch.bfloat16)
     v = synth.gaussian_bf16((N, H, d), N + S + 2)
     idx = np.sort(np.random.default_rng(S).choice(N, A, replace=False))
+    vmax = v.double().abs().amax(dim=(0, 2)).numpy()
     for scale in (1 / math.sqrt(d), 0.35):
         o, lse = _run("pruned_attn", q, k, v, idx, scale)
         o_ref, lse_ref = O.pruned_attn(q, k, v, idx, scale)
-        _check(o, lse, o_ref, lse_ref)
+        _check(o, lse, o_ref, lse_ref, v_absmax=vmax)
     o, lse = _run("pruned_attn", q, k, v, idx, 0.2, count=150)
     o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 0.2, rows=np.arange(150))
-    _check(o[:150], lse[:150], o_ref, lse_ref)
+    _check(o[:150], lse[:150], o_ref, lse_ref, v_absmax=vmax)
     assert torch.all(o[150:].float() == 7.0) and np.all(lse[150:] == 7.0)
 
 
