@@ -783,6 +783,14 @@ def kernel_case(name, dev):
         ke, ve = torch.empty_like(kc), torch.empty_like(vc)
         for _ in range(2):
             tps.kv_sync(kc, vc, kf, vf, idx, cnt, renoise=(0.025, 0.975, 4, 1), k_eff=ke, v_eff=ve)
+    elif name == "front_hsa":
+        # fused score + top-k N/3 on the HSA step's velocity tensors (61 MB read)
+        cfg = synth.CONFIGS["hsa"]
+        v = cfg.video
+        cur, prev = rnd(v.F, v.HW, v.C), rnd(v.F, v.HW, v.C)
+        ws = tps.workspace(tps.OP_FRONT, v.N, cfg.extra["K"], dev)
+        for _ in range(2):
+            tps.lipar_front(cur, tps.FRONT_TOPK, x_ref=prev, k=v.N // 3, ws=ws)
     elif name in ("attn_mid", "attn_hsa_h4"):
         if name == "attn_mid":
             cfg = synth.CONFIGS["mid"]
@@ -1064,7 +1072,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h4"], default=None,
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h4", "front_hsa"],
+                    default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
                     help="run each HSA-size stage kernel once, print its table and exit (for counter captures)")

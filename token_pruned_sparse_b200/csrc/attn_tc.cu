@@ -84,8 +84,7 @@ struct Bars {  // mbarrier indices inside the barrier block (8 bytes each)
   static constexpr int p_full = s_full + kQT;          // + tile
   static constexpr int pv_done = p_full + kQT;         // + tile
   static constexpr int drain = pv_done + kQT;          // last commit of the MMA thread
-  static constexpr int merge = drain + 1;              // cluster leader: every partner's partials staged
-  static constexpr int count = merge + 1;
+  static constexpr int count = drain + 1;
 };
 static_assert(Bars::count * 8 <= 256, "barrier block");
 
@@ -199,7 +198,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(bar(Bars::v_empty + s), 1);
     }
     mbar_init(bar(Bars::drain), 1);
-    if (prm.cluster > 1) mbar_init(bar(Bars::merge), kSoftmaxThreads * (prm.cluster - 1));
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc<kTmemCols>(smem_u32(&s_tmem));
@@ -243,9 +241,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // cluster merge: every CTA of the cluster runs and has its barriers initialised
-  // before any CTA arrives on a peer's barrier
-  if (prm.cluster > 1) cluster_sync_all();
   const uint32_t tmem = s_tmem;
   auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
@@ -482,85 +477,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     if (ok && prm.cluster > 1) {
-      // Split-key partials merged inside the cluster over distributed shared
-      // memory: a partner stages its unnormalised O rows and (m, l) in its own
-      // K/V ring region (free once its last P V has completed: the K ring holds
-      // tile 0's rows, the V ring tile 1's) and arrives on the leader's merge
-      // barrier; the leader reads every partner's rows and writes the output.
-      constexpr int kChunks = D / 4;                                   // float4 chunks per row
+      // Split-key partials: every CTA of the cluster stages its unnormalised O
+      // rows and (m, l) in its own K/V ring region (free once its last P V has
+      // completed: the K ring holds tile 0's rows, the V ring tile 1's), chunks
+      // rotated by row so the 16-byte stores of a warp hit distinct banks. The
+      // merge runs after the cluster barrier below.
+      constexpr int kChunks = D / 4;
       const int srow = t * kBM + r;
-      float4* stage = reinterpret_cast<float4*>(gbase + L::kK);       // [256][kChunks], chunk rotated by row
-      float2* ml = reinterpret_cast<float2*>(gbase + L::kList);       // [256] (m_run, l_run)
-      const uint32_t crank = cluster_ctarank();
-      if (crank != 0) {
+      float4* stage = reinterpret_cast<float4*>(gbase + L::kK);
+      float2* ml = reinterpret_cast<float2*>(gbase + L::kList);
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float o[32];
-          tmem_ld32(tO(t) + lane_off + c, o);
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        tmem_ld32(tO(t) + lane_off + c, o);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            stage[srow * kChunks + (c / 4 + q + r) % kChunks] =
-                make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-        }
-        ml[srow] = make_float2(m_run, l_run);
-        mbar_arrive_remote(map_to_rank(bar(Bars::merge), 0));
-      } else if (__all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::merge), 0, &s_abort, prm.status))) {
-        const int np = prm.cluster - 1;
-        float mk[kMaxCluster - 1], ak[kMaxCluster - 1];
-        uint32_t rbase[kMaxCluster - 1];
-        float M = m_run;
-#pragma unroll
-        for (int k = 0; k < kMaxCluster - 1; ++k) {
-          mk[k] = -INFINITY;
-          ak[k] = 0.f;
-          rbase[k] = 0u;
-          if (k < np) {
-            const float2 v = ld_cluster_f2(map_to_rank(smem_u32(&ml[srow]), k + 1));
-            mk[k] = v.x;
-            ak[k] = v.y;                                                // l of partner k, for now
-            rbase[k] = map_to_rank(smem_u32(stage), k + 1);
-            M = fmaxf(M, v.x);
-          }
-        }
-        const float a0 = m_run == -INFINITY ? 0.f : fast_exp2(m_run - M);
-        float l = a0 * l_run;
-#pragma unroll
-        for (int k = 0; k < kMaxCluster - 1; ++k) {
-          const float lk = ak[k];
-          ak[k] = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - M);
-          l += ak[k] * lk;
-        }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float o[32];
-          tmem_ld32(tO(t) + lane_off + c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= a0;
-#pragma unroll
-          for (int k = 0; k < kMaxCluster - 1; ++k) {
-            if (k >= np) break;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 x = ld_cluster_f4(rbase[k] + static_cast<uint32_t>(srow * kChunks + (c / 4 + q + r) % kChunks) * 16u);
-              o[4 * q] = fmaf(ak[k], x.x, o[4 * q]);
-              o[4 * q + 1] = fmaf(ak[k], x.y, o[4 * q + 1]);
-              o[4 * q + 2] = fmaf(ak[k], x.z, o[4 * q + 2]);
-              o[4 * q + 3] = fmaf(ak[k], x.w, o[4 * q + 3]);
-            }
-          }
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
-                                           pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                           pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                           pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
-          }
-        }
-        if (valid && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
+        for (int q = 0; q < 8; ++q)
+          stage[srow * kChunks + (c / 4 + q + r) % kChunks] =
+              make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
       }
+      ml[srow] = make_float2(m_run, l_run);
     } else if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       if (prm.nsplit > 1) {
@@ -604,13 +539,85 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
   }
 
+  // ---- split-key merge inside the cluster ------------------------------------------------
+  // After every CTA has staged its partials (cluster barrier, release/acquire at
+  // cluster scope), CTA rank k merges rows [k*R, (k+1)*R) of the 256, R =
+  // ceil(256/S), reading every rank's staged rows over distributed shared
+  // memory: two threads per row, each half a row. The second barrier keeps
+  // every CTA's shared memory valid until its peers have read it.
+  if constexpr (!kBlk) {
+    if (prm.cluster > 1) {
+      __syncthreads();                                   // warps converged for the aligned barrier
+      cluster_sync_all();
+      constexpr int kChunks = D / 4;
+      const int S = prm.cluster;
+      const int R = (kQT * kBM + S - 1) / S;
+      const uint32_t crank = cluster_ctarank();
+      const int srow = static_cast<int>(crank) * R + (tid >> 1);
+      const int half = tid & 1;
+      if (tid < 2 * R && srow < kQT * kBM && !s_abort) {
+        const int t = srow / kBM, r = srow % kBM;
+        const bool valid = r < s_nrows[t];
+        const int64_t row = static_cast<int64_t>(s_row0[t]) + r;
+        float mk[kMaxCluster], ak[kMaxCluster];
+        uint32_t sbase_k[kMaxCluster];
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kMaxCluster; ++k) {
+          mk[k] = -INFINITY;
+          ak[k] = 0.f;
+          sbase_k[k] = 0u;
+          if (k < S) {
+            const float2 v = ld_cluster_f2(map_to_rank(smem_u32(gbase + L::kList) + 8u * srow, k));
+            mk[k] = v.x;
+            ak[k] = v.y;                                                // l of rank k, for now
+            sbase_k[k] = map_to_rank(smem_u32(gbase + L::kK), k);
+            M = fmaxf(M, v.x);
+          }
+        }
+        float l = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxCluster; ++k) {
+          const float lk = ak[k];
+          ak[k] = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - M);
+          l += ak[k] * lk;
+        }
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D) + half * (D / 16);
+#pragma unroll
+        for (int c8 = 0; c8 < D / 16; ++c8) {            // 8 columns per 16-byte output vector
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = 0.f;
+#pragma unroll
+          for (int k = 0; k < kMaxCluster; ++k) {
+            if (k >= S) break;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int chunk = half * (kChunks / 2) + c8 * 2 + q;
+              const float4 x = ld_cluster_f4(sbase_k[k] + static_cast<uint32_t>(srow * kChunks + (chunk + r) % kChunks) * 16u);
+              o[4 * q] = fmaf(ak[k], x.x, o[4 * q]);
+              o[4 * q + 1] = fmaf(ak[k], x.y, o[4 * q + 1]);
+              o[4 * q + 2] = fmaf(ak[k], x.z, o[4 * q + 2]);
+              o[4 * q + 3] = fmaf(ak[k], x.w, o[4 * q + 3]);
+            }
+          }
+          if (valid)
+            orow[c8] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                                  pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+        }
+        if (valid && half == 0 && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
+      }
+      __syncthreads();
+      cluster_sync_all();
+    }
+  }
+
   // ---- teardown ------------------------------------------------------------------------
   if (warp == kMmaWarp && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // a partner's shared memory stays valid until the leader has read it
-  if (prm.cluster > 1) cluster_sync_all();
   if (warp == kMmaWarp) {
     __syncwarp();
     tmem_dealloc<kTmemCols>(tmem);

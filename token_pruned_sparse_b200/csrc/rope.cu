@@ -31,6 +31,7 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRun = 8;
+constexpr int kUnroll = 4;      // 16-byte vectors per lane in flight
 constexpr int kMaxPairs = 64;   // d <= 128
 
 struct RopeTable {
@@ -62,21 +63,30 @@ __global__ void __launch_bounds__(kThreads) rerotate_kernel(const uint4* k_cache
     for (int64_t n = r0; n < r0 + kRun && n < N; ++n) {
       const bool active = p < cnt && idx[p] == n;
       const int64_t row = n * vpr;
-      if (active) {
-        for (int v = lane; v < vpr; v += 32) k_eff[row + v] = k_cache[row + v];
-        ++p;
-      } else {
-        for (int v = lane; v < vpr; v += 32) {
-          const uint4 x = k_cache[row + v];
-          const int p0 = (v % vph) * 4;                    // first channel pair of this vector
-          const float4 c01 = *reinterpret_cast<const float4*>(&s_cs[p0]);
-          const float4 c23 = *reinterpret_cast<const float4*>(&s_cs[p0 + 2]);
-          k_eff[row + v] = make_uint4(rotate_pair(x.x, make_float2(c01.x, c01.y)),
-                                      rotate_pair(x.y, make_float2(c01.z, c01.w)),
-                                      rotate_pair(x.z, make_float2(c23.x, c23.y)),
-                                      rotate_pair(x.w, make_float2(c23.z, c23.w)));
+      // kUnroll vectors per lane in flight before any is used
+      for (int v0 = lane; v0 < vpr; v0 += 32 * kUnroll) {
+        uint4 x[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < vpr) x[u] = k_cache[row + v0 + 32 * u];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v >= vpr) continue;
+          if (active) {
+            k_eff[row + v] = x[u];
+          } else {
+            const int p0 = (v % vph) * 4;                  // first channel pair of this vector
+            const float4 c01 = *reinterpret_cast<const float4*>(&s_cs[p0]);
+            const float4 c23 = *reinterpret_cast<const float4*>(&s_cs[p0 + 2]);
+            k_eff[row + v] = make_uint4(rotate_pair(x[u].x, make_float2(c01.x, c01.y)),
+                                        rotate_pair(x[u].y, make_float2(c01.z, c01.w)),
+                                        rotate_pair(x[u].z, make_float2(c23.x, c23.y)),
+                                        rotate_pair(x[u].w, make_float2(c23.z, c23.w)));
+          }
         }
       }
+      if (active) ++p;
     }
     if (lane == 0) {
       const int64_t end = r0 + kRun < N ? r0 + kRun : N;
