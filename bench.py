@@ -255,12 +255,15 @@ class HsaStep(PathStep):
                 "ws_s": t.workspace(t.OP_SCHEDULE, self.N, self.K, dev),
                 "q": z(), "k": z(), "v": z(), "o": z()}
 
-    def front(self, X, vp, vc, q, kf, vf):
-        """score -> group -> schedule -> gathers into buffer set X."""
+    def select(self, X, vp, vc):
+        """score + group split (one launch) -> schedule, into buffer set X."""
         t = self.tps
         t.lipar_front(vc, t.FRONT_GROUP, x_ref=vp, K=self.K, group=X["group"], ws=X["ws_g"])
         t.lipar_schedule(X["group"], self.K, self.budgets, self.T, self.i, self.m, idx=X["idx"], count=X["cnt"],
                          ws=X["ws_s"])
+
+    def gather(self, X, q, kf, vf):
+        t = self.tps
         t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
         t.tps_gather_rows(X["k"], kf, X["idx"], X["cnt"])
         t.tps_gather_rows(X["v"], vf, X["idx"], X["cnt"])
@@ -274,7 +277,8 @@ class HsaStep(PathStep):
 
     def _pre(self):
         X = self.bufs
-        self.front(X, self.v_prev, self.v_cur, self.q, self.kf, self.vf)
+        self.select(X, self.v_prev, self.v_cur)
+        self.gather(X, self.q, self.kf, self.vf)
         self.sync(X)
 
     def _attn(self):
@@ -299,10 +303,12 @@ class HsaStep(PathStep):
         h2d = sum(host[k].numel() * host[k].element_size() for k in ("vp", "vc")) + 3 * self.A * R
         return h2d, self.A * R
 
-    def e2e_front(self, X, host):
+    def e2e_copy(self, X, host):
         X["vp"].copy_(host["vp"], non_blocking=True)
         X["vc"].copy_(host["vc"], non_blocking=True)
-        self.front(X, X["vp"], X["vc"], host["q"], host["k"], host["v"])     # gathers read rows over PCIe
+
+    def e2e_select(self, X):
+        self.select(X, X["vp"], X["vc"])
 
 
 class MidStep(PathStep):
@@ -353,9 +359,12 @@ class MidStep(PathStep):
                 "cnt": torch.empty(1, dtype=torch.int32, device=dev),
                 "ws": t.workspace(t.OP_FRONT, self.N, 0, dev), "q": z(), "k": z(), "v": z(), "o": z()}
 
-    def front(self, X, x, q, kf, vf):
+    def select(self, X, x):
         t = self.tps
         t.lipar_front(x, t.FRONT_TOPK, k=self.k, idx=X["idx"], count=X["cnt"], ws=X["ws"])
+
+    def gather(self, X, q, kf, vf):
+        t = self.tps
         t.tps_gather_rows(X["q"], q, X["idx"], X["cnt"])
         t.tps_gather_rows(X["k"], kf, X["idx"], X["cnt"])
         t.tps_gather_rows(X["v"], vf, X["idx"], X["cnt"])
@@ -368,7 +377,8 @@ class MidStep(PathStep):
 
     def _pre(self):
         X = self.bufs
-        self.front(X, self.x, self.q, self.kf, self.vf)
+        self.select(X, self.x)
+        self.gather(X, self.q, self.kf, self.vf)
         self.sync(X)
 
     def _attn(self):
@@ -388,9 +398,11 @@ class MidStep(PathStep):
         R = self.H * self.d * 2
         return host["x"].numel() * host["x"].element_size() + 3 * self.k * R, self.k * R
 
-    def e2e_front(self, X, host):
+    def e2e_copy(self, X, host):
         X["x"].copy_(host["x"], non_blocking=True)
-        self.front(X, X["x"], host["q"], host["k"], host["v"])
+
+    def e2e_select(self, X):
+        self.select(X, X["x"])
 
 
 # ---------------------------------------------------------------- timing ------
@@ -496,51 +508,72 @@ def e2e_leg(st, dev, steps, world):
     step copies whole (velocity or latent tensors) are copied to the device,
     the gathers read only the active rows of Q/K/V from host memory, and
     scatter_out writes only the active rows of the caller's host-side output.
-    Step i+1's copy, score, selection and gathers run on a second stream
-    beside step i's kv_sync and attention; step i's scatter_out runs on a
-    third stream beside step i+1's attention."""
+    Three buffer sets rotate so that, while step i's attention runs on the
+    compute stream, step i+1's gathers read over PCIe on a second stream, step
+    i+2's whole-tensor copy follows them, and step i-1's scatter_out writes
+    over PCIe on a third. Step i+1's selection (one cooperative launch that
+    wants every SM) runs on the compute stream between step i's kv_sync and
+    its attention, so it never waits behind a long attention kernel."""
     tps = st.tps
     host = st.host_inputs()
     o_host = torch.zeros((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory()
     if not all(tps.pointer_is_device_accessible(t) for t in list(host.values()) + [o_host]):
         return {"unavailable": "pinned host memory is not device-accessible here"}
     h2d, d2h = st.e2e_bytes(host)
-    sets = [st.new_buffers(dev), st.new_buffers(dev)]
+    sets = [st.new_buffers(dev) for _ in range(3)]
     comp = torch.cuda.current_stream()
     s_pre, s_post = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()           # noqa: E731
-    pre_done, attn_done, free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    copied, selected, gathered, attended, free = ([ev() for _ in range(3)] for _ in range(5))
     for e in free:
         e.record(comp)
 
-    def pre(i):
-        b = i & 1
+    def copy_in(i):                            # s_pre: whole-tensor copy of step i's inputs
+        b = i % 3
         with torch.cuda.stream(s_pre):
             s_pre.wait_event(free[b])
-            st.e2e_front(sets[b], host)
-            pre_done[b].record(s_pre)
+            st.e2e_copy(sets[b], host)
+            copied[b].record(s_pre)
 
-    def main(i):
-        b = i & 1
-        X = sets[b]
-        comp.wait_event(pre_done[b])
-        st.sync(X)
-        st.attend(X)
-        attn_done[b].record(comp)
-        with torch.cuda.stream(s_post):
-            s_post.wait_event(attn_done[b])
-            tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])          # rows written over PCIe
-            free[b].record(s_post)
+    def select(i):                             # compute stream: selection of step i
+        b = i % 3
+        comp.wait_event(copied[b])
+        st.e2e_select(sets[b])
+        selected[b].record(comp)
+
+    def gather(i):                             # s_pre: active rows of step i over PCIe
+        b = i % 3
+        with torch.cuda.stream(s_pre):
+            s_pre.wait_event(selected[b])
+            st.gather(sets[b], host["q"], host["k"], host["v"])
+            gathered[b].record(s_pre)
 
     def run(n):
-        pre(0)
+        copy_in(0)
+        select(0)
+        gather(0)
+        if n > 1:
+            copy_in(1)
         for i in range(n):
+            b = i % 3
+            X = sets[b]
+            comp.wait_event(gathered[b])
+            st.sync(X)
             if i + 1 < n:
-                pre(i + 1)
-            main(i)
+                select(i + 1)
+            st.attend(X)
+            attended[b].record(comp)
+            with torch.cuda.stream(s_post):
+                s_post.wait_event(attended[b])
+                tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])      # rows written over PCIe
+                free[b].record(s_post)
+            if i + 1 < n:
+                gather(i + 1)
+            if i + 2 < n:
+                copy_in(i + 2)
         comp.wait_stream(s_post)
 
-    run(2)
+    run(3)
     torch.cuda.synchronize()
     tps.tps_check()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -560,8 +593,8 @@ def e2e_leg(st, dev, steps, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 4),
             "mode": "pinned host data; whole velocity/latent tensors copied in, gathers read and scatter_out "
-                    "writes only the active rows over PCIe; step i+1's front end and step i-1's scatter overlap "
-                    "step i's attention"}
+                    "writes only the active rows over PCIe; three rotating buffer sets: step i+1's gathers and "
+                    "step i-1's scatter overlap step i's attention"}
 
 
 # ------------------------------------------------------- kernel sweeps --------
