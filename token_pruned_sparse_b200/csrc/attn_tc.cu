@@ -61,7 +61,9 @@ constexpr int kTmemCols = 512;
 constexpr int kSubBytes = 128 * 128;   // one [128 rows x 64 bf16] swizzled sub-tile
 constexpr float kSumLimit = 1099511627776.f;   // 2^40: largest tile row sum kept without a new max
 
-template <int D>
+// kLists: key-block lists (block mode: one per tile); the dense kernel's list
+// region holds the (m, l) pairs of a cluster merge instead.
+template <int D, int kLists>
 struct Layout {
   static constexpr int kSub = D / 64;                    // 64-wide sub-tiles per row of Q/K/V
   static constexpr int kQ = 0;                           // [tile][sub]
@@ -69,7 +71,7 @@ struct Layout {
   static constexpr int kV = kK + kStages * kSub * kSubBytes;
   static constexpr int kList = kV + kStages * kSub * kSubBytes;   // uint16 kept key blocks, per tile
   static constexpr int kListMax = 4096;
-  static constexpr int kBar = kList + kQT * kListMax * 2;   // mbarriers (Bars)
+  static constexpr int kBar = kList + kLists * kListMax * 2;   // mbarriers (Bars)
   static constexpr int kBytes = kBar + 256;
   static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
 };
@@ -120,11 +122,418 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return r;
 }
 
-template <int D, bool kBlk>
+template <int D, bool kClu>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams prm) {
-  using L = Layout<D>;
+  using L = Layout<D, 1>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_ntiles;
+  __shared__ volatile int s_abort;
+
+  const AttnArgs& p = prm.a;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y;
+  const int64_t rows = active_count(p.count, p.cap);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
+  if (row0 >= rows) return;   // whole CTA exits before touching TMEM or barriers
+
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t bar0 = sbase + L::kBar;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  const int nkt_all = static_cast<int>((p.N + kBN - 1) / kBN);   // key tiles = key blocks
+  // split z of nsplit (dense mode only) covers key tiles [kt0, kt0 + nkt)
+  const int kt0 = static_cast<int>((static_cast<int64_t>(nkt_all) * blockIdx.z) / prm.nsplit);
+  const int nkt = static_cast<int>((static_cast<int64_t>(nkt_all) * (blockIdx.z + 1)) / prm.nsplit) - kt0;
+
+  // ---- setup: barriers, TMEM, key-tile list ---------------------------------------------
+  if (tid == 0) {
+    s_abort = 0;
+    for (int t = 0; t < kQT; ++t) {
+      mbar_init(bar(Bars::q_full + t), 1);
+      mbar_init(bar(Bars::s_full + t), 1);
+      mbar_init(bar(Bars::p_full + t), kBM);
+      mbar_init(bar(Bars::pv_done + t), 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(Bars::k_full + s), 1);
+      mbar_init(bar(Bars::v_full + s), 1);
+      mbar_init(bar(Bars::k_empty + s), 1);
+      mbar_init(bar(Bars::v_empty + s), 1);
+    }
+    mbar_init(bar(Bars::drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tmem_alloc<kTmemCols>(smem_u32(&s_tmem));
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (tid == 0) s_ntiles = nkt;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int ntiles = s_ntiles;
+  const uint32_t tmem = s_tmem;
+  auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
+  auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
+  auto tile_kb = [&](int j) -> int { return kt0 + j; };
+
+  if (warp == kTmaWarp) {
+    // ================================ TMA producer =====================================
+    if (lane == 0) {
+      int issued_k = 0, issued_v = 0;
+      for (int t = 0; t < kQT; ++t) {
+        mbar_expect_tx(bar(Bars::q_full + t), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kQ + (t * L::kSub + s) * kSubBytes, &tmQ, 64 * s, h,
+                      static_cast<int>(row0 + t * kBM), bar(Bars::q_full + t));
+      }
+      // K and V stages are freed separately: a K stage as soon as the last S MMA
+      // reading it completes (about one period before its PV stage), so the next
+      // K tile streams in while the current P.V products still run.
+      for (int j = 0; j < ntiles; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = ((j / kStages) - 1) & 1;
+        const int key0 = tile_kb(j) * kBN;
+        if (j >= kStages && !mbar_wait(bar(Bars::k_empty + st), ph, &s_abort, prm.status)) break;
+        mbar_expect_tx(bar(Bars::k_full + st), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kK + (st * L::kSub + s) * kSubBytes, &tmK, 64 * s, h, key0, bar(Bars::k_full + st));
+        issued_k = j + 1;
+        if (j >= kStages && !mbar_wait(bar(Bars::v_empty + st), ph, &s_abort, prm.status)) break;
+        mbar_expect_tx(bar(Bars::v_full + st), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kV + (st * L::kSub + s) * kSubBytes, &tmV, 64 * s, h, key0, bar(Bars::v_full + st));
+        issued_v = j + 1;
+      }
+      // drain: every load issued above must land before the CTA may exit
+      for (int t = 0; t < kQT; ++t) drain_wait(bar(Bars::q_full + t), 0);
+      for (int j = issued_k > kStages ? issued_k - kStages : 0; j < issued_k; ++j)
+        drain_wait(bar(Bars::k_full + j % kStages), (j / kStages) & 1);
+      for (int j = issued_v > kStages ? issued_v - kStages : 0; j < issued_v; ++j)
+        drain_wait(bar(Bars::v_full + j % kStages), (j / kStages) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================ MMA issuer =======================================
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, false, false);  // Q K^T: both K-major
+      constexpr uint32_t kIdescO = idesc_bf16(kBM, D, false, true);     // P V: V is MN-major
+      auto issue_s = [&](int t, int j) {
+        const int st = j % kStages;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSubBytes + (kk & 3) * 32;   // 16 bf16 along d
+          const uint64_t da = sdesc_sw128(sbase + L::kQ + t * L::kSub * kSubBytes + off, 16, 1024);
+          const uint64_t db = sdesc_sw128(sbase + L::kK + st * L::kSub * kSubBytes + off, 16, 1024);
+          mma_f16_ss(tS(t), da, db, kIdescS, kk > 0);
+        }
+        mma_commit(bar(Bars::s_full + t));
+        if (t == kQT - 1) mma_commit(bar(Bars::k_empty + st));   // last reader of this K stage
+      };
+      bool ok = ntiles > 0;
+      if (ok) ok = mbar_wait(bar(Bars::k_full), 0, &s_abort, prm.status);
+      for (int t = 0; ok && t < kQT; ++t) {
+        ok = mbar_wait(bar(Bars::q_full + t), 0, &s_abort, prm.status);
+        tc_fence_after();
+        if (ok) issue_s(t, 0);
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int st = j % kStages;
+        for (int t = 0; ok && t < kQT; ++t) {
+          ok = mbar_wait(bar(Bars::p_full + t), j & 1, &s_abort, prm.status);
+          if (ok && t == 0) ok = mbar_wait(bar(Bars::v_full + st), (j / kStages) & 1, &s_abort, prm.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // B = V [128 keys x D], MN-major: 16 keys = 2 swizzle atoms of 8 rows;
+            // LBO = next 64-wide d sub-tile, SBO = next 8 keys. A = P_t from TMEM,
+            // 16 keys = 8 columns of bf16 pairs.
+            const uint64_t db = sdesc_sw128(sbase + L::kV + st * L::kSub * kSubBytes + kk * 16 * 128, kSubBytes, 1024);
+            mma_f16_ts(tO(t), tS(t) + 8 * kk, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(Bars::pv_done + t));
+          if (t == kQT - 1) mma_commit(bar(Bars::v_empty + st));   // last reader of this V stage
+          if (j + 1 < ntiles) {
+            // S_t(j+1) overwrites the columns P_t(j) was read from: tcgen05.mma
+            // operations of one thread execute in issue order.
+            if (t == 0) {
+              ok = mbar_wait(bar(Bars::k_full + (j + 1) % kStages), ((j + 1) / kStages) & 1, &s_abort, prm.status);
+              tc_fence_after();
+            }
+            if (ok) issue_s(t, j + 1);
+          }
+        }
+      }
+      mma_commit(bar(Bars::drain));   // fires once every MMA issued above has completed
+    }
+  } else {
+    // ================================ softmax warps ====================================
+    const int t = warp >> 2;                      // query tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
+    const int64_t row = row0 + t * kBM + r;
+    const bool valid = row < rows;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float sl2 = prm.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      // every wait result is made warp-uniform: tcgen05.ld/st are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + t), j & 1, &s_abort, prm.status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int64_t key0 = static_cast<int64_t>(tile_kb(j)) * kBN;
+      const int nvalid = static_cast<int>(p.N - key0 < kBN ? p.N - key0 : kBN);
+      uint32_t sr[kBN];
+      auto load_s = [&]() {
+        tmem_ld128(tS(t) + lane_off, sr);
+        if (nvalid < kBN) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c >= nvalid) sr[c] = __float_as_uint(-INFINITY);
+        }
+      };
+      uint32_t pk[kBN / 2];
+      // P = exp2(S * scale_log2 - base) as bf16 pairs into pk; returns the row sum of this tile
+      auto exp_pass = [&](float base) -> float {
+        const uint64_t nbase = f2_pack(-base, -base);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+        for (int c = 0; c < kBN; c += 4) {
+          float a0, a1, a2, a3;
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+          acc0 = fadd2(acc0, f2_pack(p0, p1));
+          acc1 = fadd2(acc1, f2_pack(p2, p3));
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
+        }
+        float s0, s1, s2, s3;
+        f2_unpack(acc0, s0, s1);
+        f2_unpack(acc1, s2, s3);
+        return (s0 + s1) + (s2 + s3);
+      };
+      load_s();
+      // Fast path: keep the running reference max and skip the row max. Softmax is
+      // exact for any reference; the tile's sum bounds every P, so P stays finite
+      // and well inside bf16/fp32 range while the sum is at most kSumLimit.
+      bool slow = j == 0;
+      float lt = 0.f;
+      if (!slow) {
+        const float base = m_run == -INFINITY ? 0.f : m_run;
+        lt = exp_pass(base);
+        slow = __any_sync(0xffffffffu, !(lt <= kSumLimit));
+        if (slow) load_s();                         // S is intact: P has not been stored yet
+        else m_run = base;                          // a row with only masked keys so far now uses 0
+      }
+      if (slow) {
+        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+        float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+        for (int c = 4; c < kBN; c += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+        }
+        const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+        if (j == 0) {
+          m_run = m_new;
+        } else if (__any_sync(0xffffffffu, m_new > m_run)) {
+          // the warp moves its reference maxima; O (complete up to tile j-1) is rescaled
+          const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(Bars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {         // 32 columns at a time: S stays in registers
+            float o[32];
+            tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO(t) + lane_off + c, o);
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        lt = exp_pass(m_run == -INFINITY ? 0.f : m_run);
+      }
+      l_run += lt;
+      tmem_st64(tS(t) + lane_off, pk);            // P_t(j) over the first 64 columns of S_t
+      tc_fence_before();
+      mbar_arrive(bar(Bars::p_full + t));
+    }
+    // ---- epilogue ------------------------------------------------------------------------
+    if (ok && ntiles > 0) ok = mbar_wait(bar(Bars::pv_done + t), (ntiles - 1) & 1, &s_abort, prm.status);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (kClu && ok) {
+      // Split-key partials: every CTA of the cluster stages its unnormalised O
+      // rows and (m, l) in its own K/V ring region (free once its last P V has
+      // completed: the K ring holds tile 0's rows, the V ring tile 1's), chunks
+      // rotated by row so the 16-byte stores of a warp hit distinct banks. The
+      // merge runs after the cluster barrier below.
+      constexpr int kChunks = D / 4;
+      const int srow = t * kBM + r;
+      float4* stage = reinterpret_cast<float4*>(gbase + L::kK);
+      float2* ml = reinterpret_cast<float2*>(gbase + L::kList);
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          stage[srow * kChunks + (c / 4 + q + r) % kChunks] =
+              make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+      ml[srow] = make_float2(m_run, l_run);
+    } else if (ok) {
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      if (prm.nsplit > 1) {
+        // partial result of this key range: normalised fp32 row + its log-sum-exp
+        const int64_t prow = (static_cast<int64_t>(blockIdx.z) * p.cap + row) * p.H + h;
+        float4* frow = reinterpret_cast<float4*>(prm.o_part + prow * D);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
+          else
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          if (valid) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              frow[c / 4 + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
+          }
+        }
+        if (valid) prm.lse_part[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      } else {
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
+  #pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float o[32];
+          if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
+          else
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          if (valid) {
+  #pragma unroll
+            for (int q = 0; q < 4; ++q)
+              orow[c / 8 + q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv),
+                                           pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                           pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                           pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+          }
+        }
+        if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+
+  // ---- split-key merge inside the cluster ------------------------------------------------
+  // After every CTA has staged its partials (cluster barrier, release/acquire at
+  // cluster scope), CTA rank k merges rows [k*R, (k+1)*R) of the 256, R =
+  // ceil(256/S), reading every rank's staged rows over distributed shared
+  // memory: two threads per row, each half a row. The second barrier keeps
+  // every CTA's shared memory valid until its peers have read it.
+  if constexpr (kClu) {
+    __syncthreads();                                   // warps converged for the aligned barrier
+    cluster_sync_all();
+    constexpr int kChunks = D / 4;
+    const int S = prm.cluster;
+    const int R = (kQT * kBM + S - 1) / S;
+    const uint32_t crank = cluster_ctarank();
+    const int srow = static_cast<int>(crank) * R + (tid >> 1);
+    const int half = tid & 1;
+    if (tid < 2 * R && srow < kQT * kBM && !s_abort) {
+      const int r = srow % kBM;
+      const int64_t row = row0 + srow;
+      const bool valid = row < rows;
+      float mk[kMaxCluster], ak[kMaxCluster];
+      uint32_t sbase_k[kMaxCluster];
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kMaxCluster; ++k) {
+        mk[k] = -INFINITY;
+        ak[k] = 0.f;
+        sbase_k[k] = 0u;
+        if (k < S) {
+          const float2 v = ld_cluster_f2(map_to_rank(smem_u32(gbase + L::kList) + 8u * srow, k));
+          mk[k] = v.x;
+          ak[k] = v.y;                                                  // l of rank k, for now
+          sbase_k[k] = map_to_rank(smem_u32(gbase + L::kK), k);
+          M = fmaxf(M, v.x);
+        }
+      }
+      float l = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxCluster; ++k) {
+        const float lk = ak[k];
+        ak[k] = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - M);
+        l += ak[k] * lk;
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D) + half * (D / 16);
+#pragma unroll
+      for (int c8 = 0; c8 < D / 16; ++c8) {              // 8 columns per 16-byte output vector
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxCluster; ++k) {
+          if (k >= S) break;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int chunk = half * (kChunks / 2) + c8 * 2 + q;
+            const float4 x = ld_cluster_f4(sbase_k[k] + static_cast<uint32_t>(srow * kChunks + (chunk + r) % kChunks) * 16u);
+            o[4 * q] = fmaf(ak[k], x.x, o[4 * q]);
+            o[4 * q + 1] = fmaf(ak[k], x.y, o[4 * q + 1]);
+            o[4 * q + 2] = fmaf(ak[k], x.z, o[4 * q + 2]);
+            o[4 * q + 3] = fmaf(ak[k], x.w, o[4 * q + 3]);
+          }
+        }
+        if (valid)
+          orow[c8] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                                pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+      }
+      if (valid && half == 0 && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
+    cluster_sync_all();
+  }
+
+  // ---- teardown ------------------------------------------------------------------------
+  if (warp == kMmaWarp && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tmem_dealloc<kTmemCols>(tmem);
+  }
+}
+
+// Block mode (a key-block mask is given): tile t of CTA x holds the active rows
+// of original query block qb = 2x + t -- the run of the ascending idx inside
+// [128 qb, 128 qb + 128) -- and streams only the key tiles that block keeps, so
+// every key tile a tile loads is work for all its rows. The two tiles' K and V
+// loads interleave in the rings: (j, 0), (j, 1), (j + 1, 0), ..., skipping a
+// tile whose list has ended; each stage has one reader, its own tile.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, TcParams prm) {
+  using L = Layout<D, kQT>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem;
   __shared__ int s_ntiles[kQT];
@@ -139,11 +548,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int64_t rows = active_count(p.count, p.cap);
 
   // ---- the query rows of each tile ------------------------------------------------------
-  // Dense: tile t = compacted rows [256 bx + 128 t, +128). Block mode: tile t =
-  // the active rows of original query block qb = 2 bx + t, i.e. the run of the
-  // ascending idx inside [128 qb, 128 qb + 128): every row of a tile then keeps
-  // the same key blocks, so every key tile a tile loads is work for all its rows.
-  if constexpr (kBlk) {
+  {
     if (warp == 0) {
       // lane 2t: first row of tile t; lane 2t + 1: one past its last row (lower bounds in idx)
       const int64_t key = (2 * static_cast<int64_t>(blockIdx.x) + (lane >> 1) + (lane & 1)) * 128;
@@ -162,14 +567,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     __syncthreads();
     if (s_nrows[0] == 0 && s_nrows[1] == 0) return;   // uniform: before TMEM or barriers
-  } else {
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
-    if (base >= rows) return;                          // whole CTA exits before touching TMEM or barriers
-    if (tid < kQT) {
-      const int64_t n = rows - (base + tid * kBM);
-      s_row0[tid] = static_cast<int>(base + tid * kBM);
-      s_nrows[tid] = static_cast<int>(n < 0 ? 0 : (n > kBM ? kBM : n));
-    }
   }
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -177,10 +574,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint16_t* sList = reinterpret_cast<uint16_t*>(gbase + L::kList);   // [tile][kListMax]
   const uint32_t bar0 = sbase + L::kBar;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const int nkt_all = static_cast<int>((p.N + kBN - 1) / kBN);   // key tiles = key blocks
-  // split z of nsplit (dense mode only) covers key tiles [kt0, kt0 + nkt)
-  const int kt0 = static_cast<int>((static_cast<int64_t>(nkt_all) * blockIdx.z) / prm.nsplit);
-  const int nkt = static_cast<int>((static_cast<int64_t>(nkt_all) * (blockIdx.z + 1)) / prm.nsplit) - kt0;
 
   // ---- setup: barriers, TMEM, key-tile lists ------------------------------------------
   if (tid == 0) {
@@ -206,9 +599,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if constexpr (kBlk) {
+  {
     // tile t's key list: the key blocks its query block keeps, ascending
-    __syncthreads();                                   // s_nrows visible to every warp
     int base[kQT] = {0, 0};
     const uint8_t* mrow[kQT];
     for (int t = 0; t < kQT; ++t)
@@ -235,8 +627,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       __syncthreads();
     }
     if (tid < kQT) s_ntiles[tid] = base[tid];
-  } else if (tid < kQT) {
-    s_ntiles[tid] = nkt;
   }
   tc_fence_before();
   __syncthreads();
@@ -244,17 +634,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = s_tmem;
   auto tS = [&](int t) { return tmem + 256u * t; };          // S_t, later P_t (bf16 pairs)
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
-  auto tile_kb = [&](int t, int j) -> int {
-    if constexpr (kBlk) return static_cast<int>(sList[t * L::kListMax + j]);
-    else return kt0 + j;
-  };
+  auto tile_kb = [&](int t, int j) -> int { return static_cast<int>(sList[t * L::kListMax + j]); };
   const int n0 = s_ntiles[0], n1 = s_ntiles[1];
-  // Position of (tile t, key step j) in the K and V load sequence. Dense: both
-  // tiles read the one tile of step j. Block mode: loads go (j,0), (j,1), (j+1,0),
-  // ... skipping a tile whose list has ended.
+  // position of (tile t, key step j) in the K and V load sequence
   auto seq_of = [&](int j, int t) -> int {
-    if constexpr (kBlk) return (j < n0 ? j : n0) + (j < n1 ? j : n1) + (t == 1 && j < n0 ? 1 : 0);
-    else return j;
+    return (j < n0 ? j : n0) + (j < n1 ? j : n1) + (t == 1 && j < n0 ? 1 : 0);
   };
 
   if (warp == kTmaWarp) {
@@ -274,10 +658,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // reading it completes (about one period before its PV stage), so the next
       // K tile streams in while the current P.V products still run.
       const int jmax = n0 > n1 ? n0 : n1;
-      const int ntl = kBlk ? kQT : 1;                   // loads per key step
       bool ok = true;
       for (int j = 0; ok && j < jmax; ++j) {
-        for (int t = 0; ok && t < ntl; ++t) {
+        for (int t = 0; ok && t < kQT; ++t) {
           if (j >= s_ntiles[t]) continue;
           const int q = seq_of(j, t);
           const int st = q % kStages;
@@ -320,11 +703,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_f16_ss(tS(t), da, db, kIdescS, kk > 0);
         }
         mma_commit(bar(Bars::s_full + t));
-        if (kBlk || t == kQT - 1) mma_commit(bar(Bars::k_empty + st));   // last reader of this K stage
+        mma_commit(bar(Bars::k_empty + st));           // the one reader of this K stage
       };
-      // K stage of (t, j) full: dense tiles share step j's stage and wait once (t = 0)
       auto wait_k = [&](int t, int j) -> bool {
-        if (!kBlk && t != 0) return true;
         const int q = seq_of(j, t);
         const bool r = mbar_wait(bar(Bars::k_full + q % kStages), (q / kStages) & 1, &s_abort, prm.status);
         tc_fence_after();
@@ -344,7 +725,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int q = seq_of(j, t);
           const int st = q % kStages;
           ok = mbar_wait(bar(Bars::p_full + t), j & 1, &s_abort, prm.status);
-          if (ok && (kBlk || t == 0)) ok = mbar_wait(bar(Bars::v_full + st), (q / kStages) & 1, &s_abort, prm.status);
+          if (ok) ok = mbar_wait(bar(Bars::v_full + st), (q / kStages) & 1, &s_abort, prm.status);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -356,7 +737,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mma_f16_ts(tO(t), tS(t) + 8 * kk, db, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(Bars::pv_done + t));
-          if (kBlk || t == kQT - 1) mma_commit(bar(Bars::v_empty + st));   // last reader of this V stage
+          mma_commit(bar(Bars::v_empty + st));         // the one reader of this V stage
           if (j + 1 < s_ntiles[t]) {
             // S_t(j+1) overwrites the columns P_t(j) was read from: tcgen05.mma
             // operations of one thread execute in issue order.
@@ -476,47 +857,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (ok && ntiles > 0) ok = mbar_wait(bar(Bars::pv_done + t), (ntiles - 1) & 1, &s_abort, prm.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    if (ok && prm.cluster > 1) {
-      // Split-key partials: every CTA of the cluster stages its unnormalised O
-      // rows and (m, l) in its own K/V ring region (free once its last P V has
-      // completed: the K ring holds tile 0's rows, the V ring tile 1's), chunks
-      // rotated by row so the 16-byte stores of a warp hit distinct banks. The
-      // merge runs after the cluster barrier below.
-      constexpr int kChunks = D / 4;
-      const int srow = t * kBM + r;
-      float4* stage = reinterpret_cast<float4*>(gbase + L::kK);
-      float2* ml = reinterpret_cast<float2*>(gbase + L::kList);
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        float o[32];
-        tmem_ld32(tO(t) + lane_off + c, o);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          stage[srow * kChunks + (c / 4 + q + r) % kChunks] =
-              make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-      }
-      ml[srow] = make_float2(m_run, l_run);
-    } else if (ok) {
+    if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      if (prm.nsplit > 1) {
-        // partial result of this key range: normalised fp32 row + its log-sum-exp
-        const int64_t prow = (static_cast<int64_t>(blockIdx.z) * p.cap + row) * p.H + h;
-        float4* frow = reinterpret_cast<float4*>(prm.o_part + prow * D);
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float o[32];
-          if (ntiles > 0) tmem_ld32(tO(t) + lane_off + c, o);
-          else
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0.f;
-          if (valid) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              frow[c / 4 + q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
-          }
-        }
-        if (valid) prm.lse_part[prow] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-      } else {
+      {
         uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D);
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -536,80 +879,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
-    }
-  }
-
-  // ---- split-key merge inside the cluster ------------------------------------------------
-  // After every CTA has staged its partials (cluster barrier, release/acquire at
-  // cluster scope), CTA rank k merges rows [k*R, (k+1)*R) of the 256, R =
-  // ceil(256/S), reading every rank's staged rows over distributed shared
-  // memory: two threads per row, each half a row. The second barrier keeps
-  // every CTA's shared memory valid until its peers have read it.
-  if constexpr (!kBlk) {
-    if (prm.cluster > 1) {
-      __syncthreads();                                   // warps converged for the aligned barrier
-      cluster_sync_all();
-      constexpr int kChunks = D / 4;
-      const int S = prm.cluster;
-      const int R = (kQT * kBM + S - 1) / S;
-      const uint32_t crank = cluster_ctarank();
-      const int srow = static_cast<int>(crank) * R + (tid >> 1);
-      const int half = tid & 1;
-      if (tid < 2 * R && srow < kQT * kBM && !s_abort) {
-        const int t = srow / kBM, r = srow % kBM;
-        const bool valid = r < s_nrows[t];
-        const int64_t row = static_cast<int64_t>(s_row0[t]) + r;
-        float mk[kMaxCluster], ak[kMaxCluster];
-        uint32_t sbase_k[kMaxCluster];
-        float M = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < kMaxCluster; ++k) {
-          mk[k] = -INFINITY;
-          ak[k] = 0.f;
-          sbase_k[k] = 0u;
-          if (k < S) {
-            const float2 v = ld_cluster_f2(map_to_rank(smem_u32(gbase + L::kList) + 8u * srow, k));
-            mk[k] = v.x;
-            ak[k] = v.y;                                                // l of rank k, for now
-            sbase_k[k] = map_to_rank(smem_u32(gbase + L::kK), k);
-            M = fmaxf(M, v.x);
-          }
-        }
-        float l = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMaxCluster; ++k) {
-          const float lk = ak[k];
-          ak[k] = mk[k] == -INFINITY ? 0.f : fast_exp2(mk[k] - M);
-          l += ak[k] * lk;
-        }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* orow = reinterpret_cast<uint4*>(p.o + (row * p.H + h) * D) + half * (D / 16);
-#pragma unroll
-        for (int c8 = 0; c8 < D / 16; ++c8) {            // 8 columns per 16-byte output vector
-          float o[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = 0.f;
-#pragma unroll
-          for (int k = 0; k < kMaxCluster; ++k) {
-            if (k >= S) break;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const int chunk = half * (kChunks / 2) + c8 * 2 + q;
-              const float4 x = ld_cluster_f4(sbase_k[k] + static_cast<uint32_t>(srow * kChunks + (chunk + r) % kChunks) * 16u);
-              o[4 * q] = fmaf(ak[k], x.x, o[4 * q]);
-              o[4 * q + 1] = fmaf(ak[k], x.y, o[4 * q + 1]);
-              o[4 * q + 2] = fmaf(ak[k], x.z, o[4 * q + 2]);
-              o[4 * q + 3] = fmaf(ak[k], x.w, o[4 * q + 3]);
-            }
-          }
-          if (valid)
-            orow[c8] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
-                                  pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-        }
-        if (valid && half == 0 && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
-      }
-      __syncthreads();
-      cluster_sync_all();
     }
   }
 
@@ -640,15 +909,14 @@ int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, 
 
 // Sets the kernel's dynamic shared-memory limit once per device (setting it
 // twice is harmless; devices numbered 64 and above set it on every launch).
-template <int D, bool kBlk>
-int smem_attribute() {
-  static std::atomic<bool> done[64];
+template <auto kKernel>
+int smem_attribute(int bytes) {
+  static std::atomic<bool> done[64];   // one set per kernel
   int dev = 0;
   cudaGetDevice(&dev);
   const bool cached = dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire);
   if (!cached) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, kBlk>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Layout<D>::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return cuda_status(e, "pruned_attn: smem attribute");
     if (dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_release);
   }
@@ -670,14 +938,15 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mq, a.q, a.cap, a.H, a.d)) return e;
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
-  constexpr int kSmem = Layout<D>::kAlloc;
   TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1};
   if (a.bm) {
-    if (int e = smem_attribute<D, true>()) return e;
+    constexpr int kSmem = Layout<D, kQT>::kAlloc;
+    if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
     dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
-    attn_tc_kernel<D, true><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+    attn_blk_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   } else {
-    if (int e = smem_attribute<D, false>()) return e;
+    constexpr int kSmem = Layout<D, 1>::kAlloc;
+    if (int e = smem_attribute<attn_tc_kernel<D, false>>(kSmem)) return e;
     dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
               static_cast<unsigned int>(nsplit));
     attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
@@ -699,11 +968,11 @@ int cluster_slots(int S) {
     const int v = cache[dev][S].load(std::memory_order_acquire);
     if (v > 0) return v - 1;
   }
-  if (smem_attribute<D, false>()) return 0;
+  if (smem_attribute<attn_tc_kernel<D, true>>(Layout<D, 1>::kAlloc)) return 0;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(1, 1, static_cast<unsigned int>(S));
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Layout<D>::kAlloc;
+  cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
@@ -712,7 +981,7 @@ int cluster_slots(int S) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<D, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<D, true>, &cfg) != cudaSuccess) {
     cudaGetLastError();                 // a failed query leaves its error in the last-error slot
     n = 0;
   }
@@ -764,13 +1033,13 @@ int launch_cluster(const AttnArgs& a, cudaStream_t st, int S) {
   if (int e = make_map(enc, &mq, a.q, a.cap, a.H, a.d)) return e;
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
-  if (int e = smem_attribute<D, false>()) return e;
+  if (int e = smem_attribute<attn_tc_kernel<D, true>>(Layout<D, 1>::kAlloc)) return e;
   TcParams prm{a, a.scale * kLog2e, status, S, nullptr, nullptr, S};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
                      static_cast<unsigned int>(S));
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Layout<D>::kAlloc;
+  cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -779,7 +1048,7 @@ int launch_cluster(const AttnArgs& a, cudaStream_t st, int S) {
   attr[0].val.clusterDim.z = static_cast<unsigned int>(S);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, false>, mq, mk, mv, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<D, true>, mq, mk, mv, prm);
   if (e != cudaSuccess) return cuda_status(e, "pruned_attn: cluster launch");
   return launch_status("pruned_attn");
 }
