@@ -204,9 +204,9 @@ class HsaStep(PathStep):
     zero (the step rewrites the active rows)."""
 
     # this library's kernels per step: score + group split 1 (one cooperative
-    # launch); schedule 1 (cooperative); gathers 3; kv_sync 2 (cache rows,
-    # re-noise); attention 1; scatter 1
-    LAUNCHES = {"score_group": 1, "schedule": 1, "gather": 3, "kv_sync": 2, "attn": 1, "scatter": 1}
+    # launch); schedule 1 (cooperative); gathers 3; kv_sync with re-noise 1
+    # (fresh rows and re-noised rows in one pass); attention 1; scatter 1
+    LAUNCHES = {"score_group": 1, "schedule": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
 
     def __init__(self, seed_offset: int, dev, attn: str):
         from token_pruned_sparse_b200 import tps
@@ -788,9 +788,10 @@ def kernel_case(name, dev):
     launch, then the launch to capture.
 
     attn_mid: one mid-size attention launch (6084 queries x 20280 keys, 12
-    heads). attn_hsa_h4: the HSA step's attention (39600 queries x 118800
-    keys) on 4 of its 24 heads; heads are independent units of the grid, so a
-    full launch moves 6x these bytes."""
+    heads). attn_hsa_h8: the HSA step's attention (39600 queries x 118800
+    keys) on 8 of its 24 heads (the grid still fills the GPU, so the launch
+    runs unsplit like the full one); heads are independent units of the grid,
+    so a full launch moves 3x these bytes."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
     g.manual_seed(4)
@@ -824,13 +825,14 @@ def kernel_case(name, dev):
         ws = tps.workspace(tps.OP_FRONT, v.N, cfg.extra["K"], dev)
         for _ in range(2):
             tps.lipar_front(cur, tps.FRONT_TOPK, x_ref=prev, k=v.N // 3, ws=ws)
-    elif name in ("attn_mid", "attn_hsa_h4"):
+    elif name in ("attn_mid", "attn_hsa_h8"):
         if name == "attn_mid":
             cfg = synth.CONFIGS["mid"]
             N, H, d, A = cfg.video.N, cfg.H, cfg.d, synth.keep_count(cfg.video.N, cfg.keep[0])
         else:
             cfg = synth.CONFIGS["hsa"]
-            N, H, d, A = cfg.video.N, 4, cfg.d, cfg.video.N // 3
+            N, H, d, A = cfg.video.N, 8, cfg.d, cfg.video.N // 3
+            assert tps.attn_split(A, N, H, d) == 1
         idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:A])[0].to(torch.int32)
         cnt = torch.tensor([A], dtype=torch.int32, device=dev)
         q, k, v = rnd(A, H, d), rnd(N, H, d), rnd(N, H, d)
@@ -1105,7 +1107,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h4", "front_hsa"],
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h8", "front_hsa"],
                     default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
