@@ -313,6 +313,16 @@ TPS_API size_t tps_attn_workspace_size(int64_t cap, int64_t N, int H, int d);
  * with on the current device (1 = unsplit). HOST query, no launch. */
 TPS_API int tps_attn_split(int64_t cap, int64_t N, int H, int d);
 
+/* Same contract as pruned_attn for dense attention with d = 128 (blockmask
+ * must be NULL, else TPS_ERR_INVALID_ARG), computed on pairs of CTAs: one
+ * tcgen05 MMA of M = 256 rows spans two SMs (cta_group::2), each SM holding
+ * half of every K and V tile, and the probabilities P pass through shared
+ * memory so that the next Q K^T overlaps the current softmax. */
+TPS_API int pruned_attn_pair(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
+                             const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
+                             float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
+                             tps_stream stream);
+
 /* Same contract as pruned_attn, computed with the legacy warp-level
  * mma.sync tensor-core path (kept as the baseline the tcgen05 kernel is
  * measured against). */

@@ -15,10 +15,17 @@ from workloads import attn_tolerance_ok, frame_case, oracle_idx, qkv, step_case
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-IMPLS = ["pruned_attn", "pruned_attn_mma"]
+IMPLS = ["pruned_attn", "pruned_attn_mma", "pruned_attn_pair"]
+
+
+def _supported(impl, d, bm):
+    """pruned_attn_pair takes dense attention with d = 128 only."""
+    if impl == "pruned_attn_pair" and (d != 128 or bm is not None):
+        pytest.skip("pruned_attn_pair: dense d = 128 only")
 
 
 def _run(impl, q, k, v, idx, scale, bm=None, with_lse=True, count=None, cap=None):
+    _supported(impl, q.shape[-1], bm)
     fn = getattr(tps, impl)
     qd = q.to(DEV)
     di = torch.from_numpy(np.asarray(idx, np.int32)).to(DEV) if len(idx) else torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -167,8 +174,9 @@ def test_attn_blockmask_query_block_edges(impl, d):
 
 
 @pytest.mark.parametrize("impl", IMPLS)
-def test_attn_count_below_cap_leaves_tail(impl):
-    N, A, H, d = 700, 300, 2, 64
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_count_below_cap_leaves_tail(impl, d):
+    N, A, H = 700, 300, 2
     q = synth.gaussian_bf16((A, H, d), 20)
     k = synth.gaussian_bf16((N, H, d), 21)
     v = synth.gaussian_bf16((N, H, d), 22)
@@ -183,6 +191,7 @@ def test_attn_count_below_cap_leaves_tail(impl):
 
 # ------------------------------------------------------ whole per-layer path ---
 def _layer(impl, k_cache, v_cache, q_full, k_full, v_full, o_cache, idx_d, cnt_d, cap, scale, bm=None, renoise=None):
+    _supported(impl, q_full.shape[-1], bm)
     """gather -> kv_sync -> attention -> scatter on the device."""
     H, d = q_full.shape[1], q_full.shape[2]
     q_act = torch.empty((cap, H, d), dtype=torch.bfloat16, device=DEV)
@@ -462,3 +471,30 @@ def test_attn_cluster_split_wan_keep10_sampled():
 def test_attn_no_cluster_split_when_grid_is_full():
     assert tps.attn_split(6084, 20280, 12, 128) == 1
     assert tps.attn_split(39600, 118800, 24, 128) == 1
+
+
+# -------------------------------------------------- CTA-pair kernel (d = 128) -----
+@pytest.mark.parametrize("N,A,H", [(128, 1, 1), (300, 513, 2), (1000, 1024, 3), (4099, 700, 2), (2049, 2000, 1)])
+def test_attn_pair_ragged_and_against_single_cta(N, A, H):
+    """pruned_attn_pair: 512-row pair tiles with ragged tails (a pair whose
+    second CTA or second tile has no rows), matched against the oracle and, to
+    the attention tolerance, against the single-CTA kernel; A > N exercises
+    repeated indices, which attention allows."""
+    d = 128
+    q = synth.gaussian_bf16((A, H, d), 500 + A)
+    k = synth.gaussian_bf16((N, H, d), 501 + N)
+    v = synth.gaussian_bf16((N, H, d), 502 + N)
+    idx = np.sort(np.random.default_rng(A + N).choice(N, A, replace=A > N))
+    o, lse = _run("pruned_attn_pair", q, k, v, idx, 1 / math.sqrt(d))
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d))
+    _check(o, lse, o_ref, lse_ref)
+    o1, _ = _run("pruned_attn", q, k, v, idx, 1 / math.sqrt(d))
+    ok, info = attn_tolerance_ok(o.double().numpy(), o1.double().numpy())
+    assert ok, info
+
+
+def test_attn_pair_rejects_unsupported():
+    F = tps.C.c_void_p(0x1000)
+    l = tps.lib()
+    assert l.pruned_attn_pair(F, F, F, F, F, 10, 100, 2, 64, 0.1, None, 128, F, None, None) == tps.INVALID_ARG
+    assert l.pruned_attn_pair(F, F, F, F, F, 10, 100, 2, 128, 0.1, F, 128, F, None, None) == tps.INVALID_ARG

@@ -102,25 +102,6 @@ struct TcParams {
 };
 constexpr int kMaxCluster = 4;
 
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi) in one packed instruction
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 
 template <int D, bool kClu>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1123,6 +1104,27 @@ extern "C" int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tp
   int e = d == 64 ? launch<64>(a, st, S, o_part, lse_part) : launch<128>(a, st, S, o_part, lse_part);
   if (e) return e;
   e = merge_split_parts(o_part, lse_part, S, count, cap, H, d, o_act, lse, st);
+  return e ? e : ok();
+}
+
+// CTA-pair kernel for dense d = 128 launches (attn_pair.cu).
+namespace tps {
+int launch_pair(const AttnArgs& a, cudaStream_t st);
+}
+
+extern "C" int pruned_attn_pair(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
+                                const int32_t* count, int64_t cap, int64_t N, int H, int d, float scale,
+                                const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse, tps_stream stream) {
+  TPS_TRACE("pruned_attn_pair");
+  using namespace tps;
+  AttnArgs a;
+  if (int e = attn_validate("pruned_attn_pair", q_act, k, v, idx, count, cap, N, H, d, scale, blockmask, block,
+                            o_act, lse, &a))
+    return e;
+  if (d != 128 || blockmask)
+    return fail(TPS_ERR_INVALID_ARG, "pruned_attn_pair: dense attention with d = 128 only (d=%d, mask %s)", d,
+                blockmask ? "given" : "none");
+  const int e = launch_pair(a, static_cast<cudaStream_t>(stream));
   return e ? e : ok();
 }
 

@@ -42,6 +42,7 @@ SIGNATURES = {
                               C.c_size_t, _P]),
     "tps_attn_workspace_size": (C.c_size_t, [_I64, _I64, _INT, _INT]),
     "tps_attn_split": (_INT, [_I64, _I64, _INT, _INT]),
+    "pruned_attn_pair": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
     "hsa_euler_update": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _I64, C.c_float, _P]),
@@ -285,6 +286,12 @@ def pruned_attn_ws(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_
                               _ptr(blockmask), int(block), _ptr(o_act), _ptr(lse), _ptr(ws), ws.numel(),
                               _stream(stream)))
     return o_act
+
+
+def pruned_attn_pair(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None,
+                     cap=None, stream=None):
+    return _attn(lib().pruned_attn_pair, q_act, k, v, idx, count, scale, blockmask, block, o_act, lse, cap,
+                 stream)
 
 
 def pruned_attn_mma(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None,
