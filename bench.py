@@ -292,23 +292,38 @@ class HsaStep(PathStep):
         return int(self.bufs["cnt"].item())
 
     # ---- end to end: the step's inputs in pinned host memory ------------------
+    # End to end, the step's inputs (2.25 GB) cross PCIe whole on the copy
+    # engines: about 40 ms, hidden under the 51 ms attention. Kernels that
+    # gathered the active rows straight from host memory beside the attention
+    # kernel were starved of SM time (14 ms alone, 62 ms beside it).
+    E2E_COPIES = True
+
     def host_inputs(self):
         """Pinned host copies of the step's inputs: the two velocity tensors and
-        the Q/K/V projections (the gathers read only the active rows of these)."""
+        the Q/K/V projections."""
         return {"vp": self.host["vp"].pin_memory(), "vc": self.host["vc"].pin_memory(),
                 "q": self.q.cpu().pin_memory(), "k": self.kf.cpu().pin_memory(), "v": self.vf.cpu().pin_memory()}
 
     def e2e_bytes(self, host):
         R = self.H * self.d * 2
-        h2d = sum(host[k].numel() * host[k].element_size() for k in ("vp", "vc")) + 3 * self.A * R
-        return h2d, self.A * R
+        return sum(t.numel() * t.element_size() for t in host.values()), self.A * R
+
+    def e2e_buffers(self, dev):
+        X = self.new_buffers(dev)
+        X.update({"qf": torch.empty_like(self.q), "kf": torch.empty_like(self.kf), "vf": torch.empty_like(self.vf)})
+        return X
 
     def e2e_copy(self, X, host):
         X["vp"].copy_(host["vp"], non_blocking=True)
         X["vc"].copy_(host["vc"], non_blocking=True)
+        for key in ("q", "k", "v"):
+            X[key + "f"].copy_(host[key], non_blocking=True)
 
     def e2e_select(self, X):
         self.select(X, X["vp"], X["vc"])
+
+    def e2e_gather(self, X, host):
+        self.gather(X, X["qf"], X["kf"], X["vf"])             # rows of the device copies
 
 
 class MidStep(PathStep):
@@ -391,6 +406,11 @@ class MidStep(PathStep):
     def active_count(self) -> int:
         return int(self.bufs["cnt"].item())
 
+    # End to end the gathers read only the active rows straight from pinned
+    # host memory (61 MB per step): whole-tensor copies (250 MB) would take
+    # longer than the 0.7 ms step.
+    E2E_COPIES = False
+
     def host_inputs(self):
         return {k: v.pin_memory() for k, v in self.host.items()}
 
@@ -398,11 +418,17 @@ class MidStep(PathStep):
         R = self.H * self.d * 2
         return host["x"].numel() * host["x"].element_size() + 3 * self.k * R, self.k * R
 
+    def e2e_buffers(self, dev):
+        return self.new_buffers(dev)
+
     def e2e_copy(self, X, host):
         X["x"].copy_(host["x"], non_blocking=True)
 
     def e2e_select(self, X):
         self.select(X, X["x"])
+
+    def e2e_gather(self, X, host):
+        self.gather(X, host["q"], host["k"], host["v"])       # active rows over PCIe
 
 
 # ---------------------------------------------------------------- timing ------
@@ -504,23 +530,25 @@ def e2e_leg(st, dev, steps, world):
     memory and the result written back into host memory.
 
     The library's kernels address pinned host memory directly (unified
-    addressing, checked with tps_pointer_is_device_accessible): the inputs the
-    step copies whole (velocity or latent tensors) are copied to the device,
-    the gathers read only the active rows of Q/K/V from host memory, and
-    scatter_out writes only the active rows of the caller's host-side output.
-    Three buffer sets rotate so that, while step i's attention runs on the
-    compute stream, step i+1's gathers read over PCIe on a second stream, step
-    i+2's whole-tensor copy follows them, and step i-1's scatter_out writes
-    over PCIe on a third. Step i+1's selection (one cooperative launch that
-    wants every SM) runs on the compute stream between step i's kv_sync and
-    its attention, so it never waits behind a long attention kernel."""
+    addressing, checked with tps_pointer_is_device_accessible): scatter_out
+    writes only the active rows of the caller's host-side output. The inputs
+    reach the device in one of two ways, per workload (E2E_COPIES): whole
+    tensors on the copy engines, gathered on the device; or the velocity /
+    latent tensors whole and the active rows of Q/K/V gathered straight from
+    host memory. Three buffer sets rotate so that, while step i's attention
+    runs on the compute stream, step i+2's copies (and, in the second way,
+    step i+1's gathers) run on a second stream and step i-1's scatter_out on a
+    third. Step i+1's selection (one cooperative launch that wants every SM)
+    runs on the compute stream between step i's kv_sync and its attention, so
+    it never waits behind a long attention kernel."""
     tps = st.tps
     host = st.host_inputs()
     o_host = torch.zeros((st.N, st.H, st.d), dtype=torch.bfloat16).pin_memory()
     if not all(tps.pointer_is_device_accessible(t) for t in list(host.values()) + [o_host]):
         return {"unavailable": "pinned host memory is not device-accessible here"}
     h2d, d2h = st.e2e_bytes(host)
-    sets = [st.new_buffers(dev) for _ in range(3)]
+    sets = [st.e2e_buffers(dev) for _ in range(3)]
+    copies = bool(getattr(st, "E2E_COPIES", False))
     comp = torch.cuda.current_stream()
     s_pre, s_post = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()           # noqa: E731
@@ -541,11 +569,15 @@ def e2e_leg(st, dev, steps, world):
         st.e2e_select(sets[b])
         selected[b].record(comp)
 
-    def gather(i):                             # s_pre: active rows of step i over PCIe
+    def gather(i):                             # active rows of step i
         b = i % 3
-        with torch.cuda.stream(s_pre):
+        if copies:                             # from the device copies, on the compute stream
+            st.e2e_gather(sets[b], host)
+            gathered[b].record(comp)
+            return
+        with torch.cuda.stream(s_pre):         # over PCIe, beside the attention
             s_pre.wait_event(selected[b])
-            st.gather(sets[b], host["q"], host["k"], host["v"])
+            st.e2e_gather(sets[b], host)
             gathered[b].record(s_pre)
 
     def run(n):
@@ -561,13 +593,15 @@ def e2e_leg(st, dev, steps, world):
             st.sync(X)
             if i + 1 < n:
                 select(i + 1)
+                if copies:
+                    gather(i + 1)
             st.attend(X)
             attended[b].record(comp)
             with torch.cuda.stream(s_post):
                 s_post.wait_event(attended[b])
                 tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])      # rows written over PCIe
                 free[b].record(s_post)
-            if i + 1 < n:
+            if i + 1 < n and not copies:
                 gather(i + 1)
             if i + 2 < n:
                 copy_in(i + 2)
@@ -592,9 +626,12 @@ def e2e_leg(st, dev, steps, world):
     return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 4),
-            "mode": "pinned host data; whole velocity/latent tensors copied in, gathers read and scatter_out "
-                    "writes only the active rows over PCIe; three rotating buffer sets: step i+1's gathers and "
-                    "step i-1's scatter overlap step i's attention"}
+            "mode": ("pinned host data; all inputs copied whole on the copy engines and gathered on the device, "
+                     "scatter_out writes only the active rows over PCIe; three rotating buffer sets: step i+2's "
+                     "copies and step i-1's scatter overlap step i's attention") if copies else
+                    ("pinned host data; whole latent tensors copied in, gathers read and scatter_out writes only "
+                     "the active rows over PCIe; three rotating buffer sets: step i+1's gathers and step i-1's "
+                     "scatter overlap step i's attention")}
 
 
 # ------------------------------------------------------- kernel sweeps --------
