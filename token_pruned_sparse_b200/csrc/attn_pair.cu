@@ -22,10 +22,12 @@
 // Warp roles in each CTA: warps 0-3 / 4-7 softmax of tile 0 / 1 (thread r owns
 // row r of the CTA's half of the tile = TMEM lane r), warp 8 TMA producer
 // (its own Q rows, its halves of K and V), warp 9 MMA issuer (rank 0 only;
-// both ranks allocate the pair's TMEM). The softmax is the one of
-// attn_tc_kernel: log2-domain exponentials against the running reference
-// maximum, whose row maximum is taken only on the first tile or when a tile's
-// row sum exceeds 2^40, with the O accumulator rescaled in TMEM then.
+// both ranks allocate the pair's TMEM). The softmax takes each tile's row
+// maximum while S is in registers and then releases S, so the next Q K^T
+// overlaps its exponentials (log2 domain, packed f32x2 arithmetic); the
+// running reference maximum moves only when a tile's maximum exceeds it by
+// more than 2^8, with the O accumulator rescaled in TMEM then. The MMA
+// issuer runs both tiles' next Q K^T before their P V products.
 //
 // Synchronisation. Barriers that rank 1 also signals live in rank 0 and are
 // waited on with acquire at cluster scope: TMA completions of both CTAs'
@@ -59,7 +61,7 @@ constexpr int kTmemCols = 512;
 constexpr int kRowsPerPair = 2 * kQT * kBM;      // 512 query rows per cluster
 constexpr int kSub = 128 * 128;                  // [128 rows x 64 bf16], 128-byte swizzle
 constexpr int kHalfSub = 64 * 128;               // [64 keys x 64 bf16] (a K half)
-constexpr float kSumLimit = 1099511627776.f;     // 2^40
+constexpr float kRefSlack = 8.f;                 // P < 2^8 between reference moves
 
 struct PairLayout {
   static constexpr int kQ = 0;                                  // [tile][d half]  Q rows of this CTA
@@ -224,17 +226,19 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (ok) issue_s(t, 0);
       }
       for (int j = 0; ok && j < ntiles; ++j) {
+        // S of the next key tile for both tiles first: each is released as soon as
+        // the softmax has S in registers, long before its P is ready
+        for (int t = 0; ok && t < kQT && j + 1 < ntiles; ++t) {
+          // the softmax of both CTAs has read S_t(j): S_t(j+1) may overwrite it
+          ok = mbar_wait_cluster(bar(PairBars::s_read + t), j & 1, &s_abort, prm.status);
+          if (ok && t == 0)
+            ok = mbar_wait_cluster(bar(PairBars::k_full + (j + 1) % kStages), ((j + 1) / kStages) & 1, &s_abort,
+                                   prm.status);
+          tc_fence_after();
+          if (ok) issue_s(t, j + 1);
+        }
         for (int t = 0; ok && t < kQT; ++t) {
-          if (j + 1 < ntiles) {
-            // the softmax of both CTAs has read S_t(j): S_t(j+1) may overwrite it
-            ok = mbar_wait_cluster(bar(PairBars::s_read + t), j & 1, &s_abort, prm.status);
-            if (ok && t == 0)
-              ok = mbar_wait_cluster(bar(PairBars::k_full + (j + 1) % kStages), ((j + 1) / kStages) & 1, &s_abort,
-                                     prm.status);
-            tc_fence_after();
-            if (ok) issue_s(t, j + 1);
-          }
-          if (ok) ok = mbar_wait_cluster(bar(PairBars::p_full + t), j & 1, &s_abort, prm.status);
+          ok = mbar_wait_cluster(bar(PairBars::p_full + t), j & 1, &s_abort, prm.status);
           if (ok && t == 0)
             ok = mbar_wait_cluster(bar(PairBars::v_full + j % kStages), (j / kStages) & 1, &s_abort, prm.status);
           tc_fence_after();
@@ -297,53 +301,46 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         return (s0 + s1) + (s2 + s3);
       };
       load_s();
-      bool slow = j == 0;
-      float lt = 0.f;
-      if (!slow) {
-        const float base_m = m_run == -INFINITY ? 0.f : m_run;
-        lt = exp_pass(base_m);
-        slow = __any_sync(0xffffffffu, !(lt <= kSumLimit));
-        if (slow) load_s();                      // S is intact: this thread has not released it yet
-        else m_run = base_m;
+      // The row maximum of every tile is taken while S is in registers, so S
+      // can be released at once: the next Q K^T then overlaps this tile's
+      // exponentials. The reference maximum moves only when the tile's
+      // maximum exceeds it by more than kRefSlack (log2 units), which keeps
+      // every P below 2^kRefSlack and makes O rescales rare.
+      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+      float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+      for (int c = 4; c < kBN; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
       }
-      if (slow) {
-        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-        float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
-#pragma unroll
-        for (int c = 4; c < kBN; c += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
-        }
-        const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
-        if (j == 0) {
-          m_run = m_new;
-        } else if (__any_sync(0xffffffffu, m_new > m_run)) {
-          const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_new);
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(PairBars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < kD; c += 32) {
-            float o[32];
-            tmem_ld32(tO(t) + lane_off + c, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO(t) + lane_off + c, o);
-          }
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        lt = exp_pass(m_run == -INFINITY ? 0.f : m_run);
-      }
-      l_run += lt;
       // S_t(j) is in registers: the next Q K^T may overwrite it
       tc_fence_before();
       if (lead) mbar_arrive(s_read_bar);
       else mbar_arrive_remote(s_read_bar);
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_target = m_run == -INFINITY || m_tile > m_run + kRefSlack ? fmaxf(m_run, m_tile) : m_run;
+      if (j > 0 && __any_sync(0xffffffffu, m_target > m_run)) {
+        // O (complete up to tile j-1) moves to the new reference
+        const float alpha = m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_target);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(PairBars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kD; c += 32) {
+          float o[32];
+          tmem_ld32(tO(t) + lane_off + c, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(tO(t) + lane_off + c, o);
+        }
+        l_run *= alpha;
+      }
+      m_run = m_target;
+      l_run += exp_pass(m_run == -INFINITY ? 0.f : m_run);
       // P_t(j-1) must have been consumed before its buffer is overwritten
       if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(PairBars::pv_done + t), (j - 1) & 1, &s_abort, prm.status))) {
         ok = false;
