@@ -828,7 +828,8 @@ def kernel_case(name, dev):
     heads). attn_hsa_h8: the HSA step's attention (39600 queries x 118800
     keys) on 8 of its 24 heads (the grid still fills the GPU, so the launch
     runs unsplit like the full one); heads are independent units of the grid,
-    so a full launch moves 3x these bytes."""
+    so a full launch moves 3x these bytes. overlap_hsa is not a capture case:
+    it times the HSA step's host transfers alone and beside the attention."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
     g.manual_seed(4)
@@ -862,6 +863,8 @@ def kernel_case(name, dev):
         ws = tps.workspace(tps.OP_FRONT, v.N, cfg.extra["K"], dev)
         for _ in range(2):
             tps.lipar_front(cur, tps.FRONT_TOPK, x_ref=prev, k=v.N // 3, ws=ws)
+    elif name == "overlap_hsa":
+        return overlap_probe(dev)
     elif name in ("attn_mid", "attn_hsa_h8"):
         if name == "attn_mid":
             cfg = synth.CONFIGS["mid"]
@@ -881,6 +884,72 @@ def kernel_case(name, dev):
     torch.cuda.synchronize()
     tps.tps_check()
     return {"kernel_case": name, "ok": True}
+
+
+def overlap_probe(dev):
+    """How the HSA step's host transfers share the GPU with its attention:
+    CUDA-event times of the attention launch (39600 x 118800 keys, 24 heads),
+    of the three row gathers straight from pinned host memory, of scatter_out
+    into pinned host memory, of whole-tensor copies of Q/K/V on the copy
+    engines, each alone and each beside the attention on a second stream."""
+    from token_pruned_sparse_b200 import tps
+    cfg = synth.CONFIGS["hsa"]
+    N, H, d = cfg.video.N, cfg.H, cfg.d
+    A = N // 3
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rnd = lambda *s: torch.randn(*s, generator=g, device=dev).to(torch.bfloat16)   # noqa: E731
+    q, k, v = rnd(A, H, d), rnd(N, H, d), rnd(N, H, d)
+    idx = torch.arange(A, device=dev, dtype=torch.int32) * 3
+    cnt = torch.tensor([A], dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    hq = torch.randn(N, H, d).to(torch.bfloat16).pin_memory()
+    hk, hv = hq.clone().pin_memory(), hq.clone().pin_memory()
+    ho = torch.zeros(N, H, d, dtype=torch.bfloat16).pin_memory()
+    rows = [torch.empty_like(q) for _ in range(3)]
+    whole = torch.empty(N, H, d, dtype=torch.bfloat16, device=dev)
+    side = torch.cuda.Stream()
+    comp = torch.cuda.current_stream()
+
+    def attn():
+        tps.pruned_attn(q, k, v, idx, cnt, 1 / math.sqrt(d), o_act=o)
+
+    def gathers():
+        for dst, src in zip(rows, (hq, hk, hv)):
+            tps.tps_gather_rows(dst, src, idx, cnt)
+
+    def scatter():
+        tps.scatter_out(ho, o, idx, cnt)
+
+    def copies():
+        for t in (hq, hk, hv):
+            whole.copy_(t, non_blocking=True)
+
+    def timed(main, beside=None, reps=3):
+        out = []
+        for _ in range(reps + 1):
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(comp)
+            if beside:
+                side.wait_event(ev[0])
+                with torch.cuda.stream(side):
+                    ev[2].record(side)
+                    beside()
+                    ev[3].record(side)
+            main()
+            ev[1].record(comp)
+            torch.cuda.synchronize()
+            out.append((ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]) if beside else None))
+        out = sorted(out[1:])
+        mid = out[len(out) // 2]
+        return {"ms": round(mid[0], 3), "beside_ms": None if mid[1] is None else round(mid[1], 3)}
+    res = {"attention": timed(attn), "row_gathers_from_host": timed(gathers),
+           "scatter_to_host": timed(scatter), "whole_qkv_copies": timed(copies),
+           "attention_with_row_gathers": timed(attn, gathers), "attention_with_scatter": timed(attn, scatter),
+           "attention_with_whole_copies": timed(attn, copies)}
+    tps.tps_check()
+    return {"kernel_case": "overlap_hsa", "ok": True, "times": res}
 
 
 # -------------------------------------------------------- CPU oracle leg ------
@@ -1144,7 +1213,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h8", "front_hsa"],
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h8", "front_hsa",
+                                              "overlap_hsa"],
                     default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")
     ap.add_argument("--stages-once", action="store_true",
