@@ -426,7 +426,7 @@ def test_attn_ws_no_split_when_grid_is_full():
 
 
 # ------------------------------- split-key attention merged inside a cluster -----
-@pytest.mark.parametrize("N,S", [(1100, 2), (1600, 3), (4099, 4)])
+@pytest.mark.parametrize("N,S", [(1100, 2), (1600, 3), (2100, 4), (4099, 4)])
 @pytest.mark.parametrize("d", [64, 128])
 def test_attn_cluster_split_matches_oracle(N, S, d):
     """One query tile pair x one head fills one SM: pruned_attn splits the keys

@@ -86,6 +86,32 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return r;
 }
 
+// P = 2^(S * scale_log2 - base) for one row of a kN-column S tile (fp32 bits in sr), as bf16
+// pairs into pk; returns the fp32 row sum. The exponentials run on the MUFU unit (ex2.approx).
+template <int kN>
+__device__ __forceinline__ float exp_row(const uint32_t (&sr)[kN], uint64_t sl2x2, float base,
+                                         uint32_t (&pk)[kN / 2]) {
+  const uint64_t nbase = f2_pack(-base, -base);
+  uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int c = 0; c < kN; c += 4) {
+    const uint64_t a01 = ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase);
+    const uint64_t a23 = ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase);
+    float a0, a1, a2, a3;
+    f2_unpack(a01, a0, a1);
+    f2_unpack(a23, a2, a3);
+    const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
+    acc0 = fadd2(acc0, f2_pack(p0, p1));
+    acc1 = fadd2(acc1, f2_pack(p2, p3));
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+    pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
+  }
+  float s0, s1, s2, s3;
+  f2_unpack(acc0, s0, s1);
+  f2_unpack(acc1, s2, s3);
+  return (s0 + s1) + (s2 + s3);
+}
+
 constexpr float kLog2e = 1.4426950408889634074f;
 constexpr float kLn2 = 0.69314718055994530942f;
 

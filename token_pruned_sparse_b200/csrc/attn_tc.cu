@@ -283,25 +283,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       uint32_t pk[kBN / 2];
       // P = exp2(S * scale_log2 - base) as bf16 pairs into pk; returns the row sum of this tile
-      auto exp_pass = [&](float base) -> float {
-        const uint64_t nbase = f2_pack(-base, -base);
-        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-        for (int c = 0; c < kBN; c += 4) {
-          float a0, a1, a2, a3;
-          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
-          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
-          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
-          acc0 = fadd2(acc0, f2_pack(p0, p1));
-          acc1 = fadd2(acc1, f2_pack(p2, p3));
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
-        }
-        float s0, s1, s2, s3;
-        f2_unpack(acc0, s0, s1);
-        f2_unpack(acc1, s2, s3);
-        return (s0 + s1) + (s2 + s3);
-      };
+      auto exp_pass = [&](float base) -> float { return exp_row<kBN>(sr, sl2x2, base, pk); };
       load_s();
       // Fast path: keep the running reference max and skip the row max. Softmax is
       // exact for any reference; the tile's sum bounds every P, so P stays finite
@@ -763,25 +745,7 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       };
       uint32_t pk[kBN / 2];
       // P = exp2(S * scale_log2 - base) as bf16 pairs into pk; returns the row sum of this tile
-      auto exp_pass = [&](float base) -> float {
-        const uint64_t nbase = f2_pack(-base, -base);
-        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-        for (int c = 0; c < kBN; c += 4) {
-          float a0, a1, a2, a3;
-          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nbase), a0, a1);
-          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2, nbase), a2, a3);
-          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1), p2 = fast_exp2(a2), p3 = fast_exp2(a3);
-          acc0 = fadd2(acc0, f2_pack(p0, p1));
-          acc1 = fadd2(acc1, f2_pack(p2, p3));
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          pk[(c >> 1) + 1] = pack_bf16x2(p2, p3);
-        }
-        float s0, s1, s2, s3;
-        f2_unpack(acc0, s0, s1);
-        f2_unpack(acc1, s2, s3);
-        return (s0 + s1) + (s2 + s3);
-      };
+      auto exp_pass = [&](float base) -> float { return exp_row<kBN>(sr, sl2x2, base, pk); };
       load_s();
       // Fast path: keep the running reference max and skip the row max. Softmax is
       // exact for any reference; the tile's sum bounds every P, so P stays finite

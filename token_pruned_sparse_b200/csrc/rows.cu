@@ -176,8 +176,12 @@ __device__ __forceinline__ uint4 renoise_vec(uint4 c, float a, float b, const fl
 // A warp owns a run of kRun consecutive rows; one warp-cooperative search finds the first
 // active index >= the run start, then the (ascending) list is walked in step.
 constexpr int kRun = 8;
+// Ten resident blocks per SM (at most 48 registers; a few bytes spill) against
+// eight at the compiler's 59 registers: the memory stream has more rows in
+// flight and the pass runs 2.7% faster at the HSA size (0.615 -> 0.599 ms).
+constexpr int kRenoiseBlocks = 10;
 
-__global__ void __launch_bounds__(kMoveThreads) kv_sync_renoise(
+__global__ void __launch_bounds__(kMoveThreads, kRenoiseBlocks) kv_sync_renoise(
     uint4* __restrict__ kc, uint4* __restrict__ vc, const uint4* __restrict__ kf,
     const uint4* __restrict__ vf, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
     int64_t cap, int64_t N, int vpr, float a, float b, const __grid_constant__ PhiloxKeys keys, uint32_t step,
