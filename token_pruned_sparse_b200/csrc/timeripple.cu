@@ -90,26 +90,30 @@ __device__ __forceinline__ void unpack(const uint4& w, float2 (&f)[4]) {
   f[3] = make_float2(bf16lo(w.w), bf16hi(w.w));
 }
 
-// s += sum over the chunk's channels in mask m (bit e = channel e) of
-// (c_e - n_e)^2, two channels per packed fp32 operation and two independent
-// accumulators; c - n is formed as fma(n, -1, c), one rounding of the exact
-// difference.
-__device__ __forceinline__ void sq_acc(float2 (&s)[2], const float2 (&c)[4], const float2 (&n)[4], uint32_t m) {
-  const float2 neg1 = make_float2(-1.f, -1.f);
-  if (m == 0xffu) {
+// (n - c) for the two bf16 channels packed in w against their fp32 centre values:
+// the mixed-precision subtraction takes the bf16 operand directly (widening is
+// exact), one rounding, the same value as -(c - n).
+__device__ __forceinline__ float2 sub_bf16x2_f32(uint32_t w, float2 c) {
+  float2 r;
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n sub.rn.f32.bf16 %0, lo, %3;\n sub.rn.f32.bf16 %1, hi, %4;\n}"
+      : "=f"(r.x), "=f"(r.y)
+      : "r"(w), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+// s += sum over the chunk's channels in mask m (bit e = channel e) of (n_e - c_e)^2,
+// two channels per packed square-and-add and two independent accumulators. The
+// neighbour n stays packed as bf16 pairs (nw); only the centre c is widened.
+__device__ __forceinline__ void sq_acc(float2 (&s)[2], const float2 (&c)[4], const uint4& nw, uint32_t m) {
+  const uint32_t w[4] = {nw.x, nw.y, nw.z, nw.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 d = __ffma2_rn(n[q], neg1, c[q]);
-      s[q & 1] = __ffma2_rn(d, d, s[q & 1]);
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float2 d = __ffma2_rn(n[q], neg1, c[q]);
+  for (int q = 0; q < 4; ++q) {
+    float2 d = sub_bf16x2_f32(w[q], c[q]);
+    if (m != 0xffu) {
       d.x = (m >> (2 * q)) & 1u ? d.x : 0.f;
       d.y = (m >> (2 * q + 1)) & 1u ? d.y : 0.f;
-      s[q & 1] = __ffma2_rn(d, d, s[q & 1]);
     }
+    s[q & 1] = __ffma2_rn(d, d, s[q & 1]);
   }
 }
 
@@ -167,7 +171,7 @@ __device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, ui
       nlw = lds128(swz(box, rc - 1, j + 1));
       nuw = lds128(swz(box, rc - kBoxCols, j + 1));
     }
-    float2 c[4], nb[4];
+    float2 c[4];
     unpack(cw, c);
     uint32_t mt, mx, my;
     if constexpr (kFixed) {
@@ -187,18 +191,9 @@ __device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, ui
       mx = j < 4 ? (wlo[1] >> (8 * j)) & 0xffu : (whi[1] >> (8 * (j - 4))) & 0xffu;
       my = j < 4 ? (wlo[2] >> (8 * j)) & 0xffu : (whi[2] >> (8 * (j - 4))) & 0xffu;
     }
-    if (has_t && mt) {
-      unpack(make_uint4(prev[4 * j], prev[4 * j + 1], prev[4 * j + 2], prev[4 * j + 3]), nb);
-      sq_acc(at, c, nb, mt);
-    }
-    if (mx) {
-      unpack(lw, nb);
-      sq_acc(ax, c, nb, mx);
-    }
-    if (my) {
-      unpack(uw, nb);
-      sq_acc(ay, c, nb, my);
-    }
+    if (has_t && mt) sq_acc(at, c, make_uint4(prev[4 * j], prev[4 * j + 1], prev[4 * j + 2], prev[4 * j + 3]), mt);
+    if (mx) sq_acc(ax, c, lw, mx);
+    if (my) sq_acc(ay, c, uw, my);
     prev[4 * j] = cw.x, prev[4 * j + 1] = cw.y, prev[4 * j + 2] = cw.z, prev[4 * j + 3] = cw.w;
   }
 }
