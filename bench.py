@@ -305,8 +305,8 @@ class HsaStep(PathStep):
                 "q": self.q.cpu().pin_memory(), "k": self.kf.cpu().pin_memory(), "v": self.vf.cpu().pin_memory()}
 
     def e2e_bytes(self, host):
-        R = self.H * self.d * 2
-        return sum(t.numel() * t.element_size() for t in host.values()), self.A * R
+        # in: every input tensor whole; out: the whole output tensor, read on the copy engine
+        return sum(t.numel() * t.element_size() for t in host.values()), self.N * self.H * self.d * 2
 
     def e2e_buffers(self, dev):
         X = self.new_buffers(dev)
@@ -530,15 +530,17 @@ def e2e_leg(st, dev, steps, world):
     memory and the result written back into host memory.
 
     The library's kernels address pinned host memory directly (unified
-    addressing, checked with tps_pointer_is_device_accessible): scatter_out
-    writes only the active rows of the caller's host-side output. The inputs
-    reach the device in one of two ways, per workload (E2E_COPIES): whole
-    tensors on the copy engines, gathered on the device; or the velocity /
-    latent tensors whole and the active rows of Q/K/V gathered straight from
-    host memory. Three buffer sets rotate so that, while step i's attention
-    runs on the compute stream, step i+2's copies (and, in the second way,
-    step i+1's gathers) run on a second stream and step i-1's scatter_out on a
-    third. Step i+1's selection (one cooperative launch that wants every SM)
+    addressing, checked with tps_pointer_is_device_accessible). The data
+    moves in one of two ways, per workload (E2E_COPIES): every input tensor
+    whole on the copy engines, gathered on the device, and the output scattered
+    into a device-side full output that one copy-engine transfer reads back
+    whole (no kernel touches PCIe, so nothing competes with the attention for
+    SMs); or the velocity / latent tensors whole, the active rows of Q/K/V
+    gathered straight from host memory and scatter_out writing only the active
+    rows of the caller's host-side output. Three buffer sets rotate so that,
+    while step i's attention runs on the compute stream, step i+2's copies (and,
+    in the second way, step i+1's gathers) run on a second stream and step i-1's
+    read-back (or scatter_out) on a third. Step i+1's selection (one cooperative launch that wants every SM)
     runs on the compute stream between step i's kv_sync and its attention, so
     it never waits behind a long attention kernel."""
     tps = st.tps
@@ -555,6 +557,10 @@ def e2e_leg(st, dev, steps, world):
     copied, selected, gathered, attended, free = ([ev() for _ in range(3)] for _ in range(5))
     for e in free:
         e.record(comp)
+    # copies: the full output lives on the device (scattered into in place) and is read back whole
+    o_dev = torch.zeros_like(o_host, device=dev) if copies else None
+    read_done = ev()
+    read_done.record(comp)
 
     def copy_in(i):                            # s_pre: whole-tensor copy of step i's inputs
         b = i % 3
@@ -596,11 +602,21 @@ def e2e_leg(st, dev, steps, world):
                 if copies:
                     gather(i + 1)
             st.attend(X)
-            attended[b].record(comp)
-            with torch.cuda.stream(s_post):
-                s_post.wait_event(attended[b])
-                tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])      # rows written over PCIe
-                free[b].record(s_post)
+            if copies:
+                comp.wait_event(read_done)                                # step i-1's read-back is done
+                tps.scatter_out(o_dev, X["o"], X["idx"], X["cnt"])
+                attended[b].record(comp)
+                free[b].record(comp)
+                with torch.cuda.stream(s_post):
+                    s_post.wait_event(attended[b])
+                    o_host.copy_(o_dev, non_blocking=True)               # whole output, copy engine
+                    read_done.record(s_post)
+            else:
+                attended[b].record(comp)
+                with torch.cuda.stream(s_post):
+                    s_post.wait_event(attended[b])
+                    tps.scatter_out(o_host, X["o"], X["idx"], X["cnt"])  # rows written over PCIe
+                    free[b].record(s_post)
             if i + 1 < n and not copies:
                 gather(i + 1)
             if i + 2 < n:
@@ -626,9 +642,10 @@ def e2e_leg(st, dev, steps, world):
     return {"value": round(job_throughput(st.flops, world, steps, ms) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "ms_per_step": round(ms / steps, 4),
-            "mode": ("pinned host data; all inputs copied whole on the copy engines and gathered on the device, "
-                     "scatter_out writes only the active rows over PCIe; three rotating buffer sets: step i+2's "
-                     "copies and step i-1's scatter overlap step i's attention") if copies else
+            "mode": ("pinned host data; all inputs copied whole on the copy engines and gathered on the device; "
+                     "scatter_out into the device-side full output, read back whole on the copy engine; three "
+                     "rotating buffer sets: step i+2's copies and step i-1's read-back overlap step i's "
+                     "attention") if copies else
                     ("pinned host data; whole latent tensors copied in, gathers read and scatter_out writes only "
                      "the active rows over PCIe; three rotating buffer sets: step i+1's gathers and step i-1's "
                      "scatter overlap step i's attention")}
