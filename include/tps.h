@@ -317,9 +317,9 @@ TPS_API int tps_attn_split(int64_t cap, int64_t N, int H, int d);
  * must be NULL, else TPS_ERR_INVALID_ARG), computed on pairs of CTAs: one
  * tcgen05 MMA of M = 256 rows spans two SMs (cta_group::2), each SM holding
  * half of every K and V tile, and the probabilities P pass through shared
- * memory so that the next Q K^T overlaps the current softmax. Results equal
- * pruned_attn's unsplit kernel; on B200 it runs at about 0.6-0.7 of
- * pruned_attn's throughput, which does not route to it. */
+ * memory so that the next Q K^T overlaps the current softmax. Results agree
+ * with pruned_attn within the attention tolerance; on B200 it runs at about
+ * 0.6-0.7 of pruned_attn's throughput, and pruned_attn does not route to it. */
 TPS_API int pruned_attn_pair(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
                              const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
                              float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
