@@ -78,9 +78,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
   return v;
 }
 
-// 16-byte chunk j of box row r under the 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz(uint32_t box, int r, int j) {
-  return box + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(j ^ (r & 7)) << 4);
+// Box row r under the 128-byte swizzle, with the row's swizzle key folded into
+// its address: the row starts on a 128-byte boundary (box is 1 KB aligned), so
+// its 16-byte chunk j sits at row_key(box, r) ^ (j << 4).
+__device__ __forceinline__ uint32_t row_key(uint32_t box, int r) {
+  return (box + static_cast<uint32_t>(r) * 128u) | (static_cast<uint32_t>(r & 7) << 4);
 }
 
 __device__ __forceinline__ void unpack(const uint4& w, float2 (&f)[4]) {
@@ -159,17 +161,19 @@ __device__ __forceinline__ constexpr uint32_t fixed_bits() {
 // The checks of one frame for this thread's token and 64 channels: chunk j+1's
 // three rows are loaded while chunk j is checked. kFixed: compile-time windows.
 template <int D, int HALF, bool kFixed>
-__device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, uint32_t (&prev)[32], float2 (&at)[2],
+__device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, const uint32_t (&pin)[32],
+                                            uint32_t (&pout)[32], float2 (&at)[2],
                                             float2 (&ax)[2], float2 (&ay)[2], const uint32_t (&wlo)[3],
                                             const uint32_t (&whi)[3]) {
-  uint4 ncw = lds128(swz(box, rc, 0)), nlw = lds128(swz(box, rc - 1, 0)), nuw = lds128(swz(box, rc - kBoxCols, 0));
+  const uint32_t kc = row_key(box, rc), kl = row_key(box, rc - 1), ku = row_key(box, rc - kBoxCols);
+  uint4 ncw = lds128(kc), nlw = lds128(kl), nuw = lds128(ku);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint4 cw = ncw, lw = nlw, uw = nuw;
     if (j < 7) {
-      ncw = lds128(swz(box, rc, j + 1));
-      nlw = lds128(swz(box, rc - 1, j + 1));
-      nuw = lds128(swz(box, rc - kBoxCols, j + 1));
+      ncw = lds128(kc ^ static_cast<uint32_t>((j + 1) << 4));
+      nlw = lds128(kl ^ static_cast<uint32_t>((j + 1) << 4));
+      nuw = lds128(ku ^ static_cast<uint32_t>((j + 1) << 4));
     }
     float2 c[4];
     unpack(cw, c);
@@ -191,10 +195,10 @@ __device__ __forceinline__ void check_frame(uint32_t box, int rc, bool has_t, ui
       mx = j < 4 ? (wlo[1] >> (8 * j)) & 0xffu : (whi[1] >> (8 * (j - 4))) & 0xffu;
       my = j < 4 ? (wlo[2] >> (8 * j)) & 0xffu : (whi[2] >> (8 * (j - 4))) & 0xffu;
     }
-    if (has_t && mt) sq_acc(at, c, make_uint4(prev[4 * j], prev[4 * j + 1], prev[4 * j + 2], prev[4 * j + 3]), mt);
+    if (has_t && mt) sq_acc(at, c, make_uint4(pin[4 * j], pin[4 * j + 1], pin[4 * j + 2], pin[4 * j + 3]), mt);
     if (mx) sq_acc(ax, c, lw, mx);
     if (my) sq_acc(ay, c, uw, my);
-    prev[4 * j] = cw.x, prev[4 * j + 1] = cw.y, prev[4 * j + 2] = cw.z, prev[4 * j + 3] = cw.w;
+    pout[4 * j] = cw.x, pout[4 * j + 1] = cw.y, pout[4 * j + 2] = cw.z, pout[4 * j + 3] = cw.w;
   }
 }
 
@@ -259,8 +263,9 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 2) tr_kernel(const __grid_co
 #pragma unroll
   for (int i = 0; i < 32; ++i) prev[i] = 0;
 
-  int k = 0;
-  for (; k < nload; ++k) {
+  // one frame: checks against pin (the previous frame), this frame's centres into pout;
+  // false when a wait gave up (the CTA leaves together)
+  auto step = [&](int k, const uint32_t (&pin)[32], uint32_t (&pout)[32]) -> bool {
     const uint32_t bar = (k & 1) ? bar1 : bar0;
     // a wait that gives up sets the abort flag; the CTA leaves together after the barrier below
     mbar_wait(bar, static_cast<uint32_t>((k >> 1) & 1), abort_flag, p.status);
@@ -272,16 +277,16 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 2) tr_kernel(const __grid_co
     if (prime) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint4 c = lds128(swz(box, rc, j));
-        prev[4 * j] = c.x, prev[4 * j + 1] = c.y, prev[4 * j + 2] = c.z, prev[4 * j + 3] = c.w;
+        const uint4 c = lds128(row_key(box, rc) ^ static_cast<uint32_t>(j << 4));
+        pout[4 * j] = c.x, pout[4 * j + 1] = c.y, pout[4 * j + 2] = c.z, pout[4 * j + 3] = c.w;
       }
     } else {
       const bool has_t = f > 0;
       if (p.fixed_windows) {
-        if (half == 0) check_frame<D, 0, true>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
-        else check_frame<D, (L::kHalves > 1 ? 1 : 0), true>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
+        if (half == 0) check_frame<D, 0, true>(box, rc, has_t, pin, pout, at, ax, ay, wlo, whi);
+        else check_frame<D, (L::kHalves > 1 ? 1 : 0), true>(box, rc, has_t, pin, pout, at, ax, ay, wlo, whi);
       } else {
-        check_frame<D, 0, false>(box, rc, has_t, prev, at, ax, ay, wlo, whi);
+        check_frame<D, 0, false>(box, rc, has_t, pin, pout, at, ax, ay, wlo, whi);
       }
     }
     float s[3] = {(at[0].x + at[1].x) + (at[0].y + at[1].y), (ax[0].x + ax[1].x) + (ax[0].y + ax[1].y),
@@ -289,12 +294,12 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 2) tr_kernel(const __grid_co
     float* r = red + (k & 1) * 3 * kTile;
     if (L::kHalves == 2 && half == 1 && !prime) r[t] = s[0], r[kTile + t] = s[1], r[2 * kTile + t] = s[2];
     __syncthreads();                                 // slot consumed, partial sums visible
-    if (*abort_flag) break;                          // same value in every thread: set before the barrier
+    if (*abort_flag) return false;                   // same value in every thread: set before the barrier
     if (tid == 0 && issued < nload) {
       fence_proxy_async_smem();
       issue(issued++);
     }
-    if (prime || half != 0 || !inb) continue;
+    if (prime || half != 0 || !inb) return true;
     if (L::kHalves == 2) s[0] += r[t], s[1] += r[kTile + t], s[2] += r[2 * kTile + t];
     const bool has[3] = {f > 0, gx > 0, gy > 0};
     const int64_t n = (static_cast<int64_t>(f) * p.Hs + gy) * p.Ws + gx;
@@ -306,6 +311,17 @@ __global__ void __launch_bounds__(Lay<D>::kThreads, 2) tr_kernel(const __grid_co
       if (p.delta) p.delta[(static_cast<int64_t>(a) * p.N + n) * p.H + h] = dl;
     }
     p.reuse[n * p.H + h] = static_cast<uint8_t>(bits);
+    return true;
+  };
+  // two frames per iteration with the previous-frame arrays swapping roles, so a frame's
+  // centres land in their registers for the next frame without a copy
+  uint32_t prev2[32];
+  int k = 0;
+  while (k < nload) {
+    if (!step(k, prev, prev2)) break;
+    if (++k >= nload) break;
+    if (!step(k, prev2, prev)) break;
+    ++k;
   }
   if (k < nload && tid == 0) {                       // gave up: let this CTA's copies land first
     for (int kk = k; kk < issued; ++kk) drain_wait((kk & 1) ? bar1 : bar0, static_cast<uint32_t>((kk >> 1) & 1));
