@@ -196,6 +196,14 @@ class PathStep:
             self._post()
 
 
+def attn_launches(tps, attn, cap, N, H, d) -> int:
+    """Kernel launches of one dense attention call: one, or two when the
+    launch plan runs the grid's last query tiles split in a second launch."""
+    if attn != "tc":
+        return 1
+    return 2 if tps.attn_plan(cap, N, H, d)[2] > 1 else 1
+
+
 class HsaStep(PathStep):
     """HSA step at |A| = N/3 (step i = 1 of T = 40) on the 118800-token video.
 
@@ -205,7 +213,8 @@ class HsaStep(PathStep):
 
     # this library's kernels per step: score + group split 1 (one cooperative
     # launch); schedule 1 (cooperative); gathers 3; kv_sync with re-noise 1
-    # (fresh rows and re-noised rows in one pass); attention 1; scatter 1
+    # (fresh rows and re-noised rows in one pass); attention 1 (2 when its launch
+    # plan adds a split tail launch, counted in __init__); scatter 1
     LAUNCHES = {"score_group": 1, "schedule": 1, "gather": 3, "kv_sync": 1, "attn": 1, "scatter": 1}
 
     def __init__(self, seed_offset: int, dev, attn: str):
@@ -240,7 +249,7 @@ class HsaStep(PathStep):
         self.attn_fn = tps.pruned_attn if attn == "tc" else tps.pruned_attn_mma
         self.flops = 4.0 * self.d * self.H * self.A * self.N
         self.units = self.A
-        self.launches = sum(self.LAUNCHES.values())
+        self.launches = sum(self.LAUNCHES.values()) - 1 + attn_launches(tps, attn, self.A, self.N, self.H, self.d)
 
     def new_buffers(self, dev):
         t = self.tps
@@ -363,7 +372,7 @@ class MidStep(PathStep):
         self.attn_fn = tps.pruned_attn if attn == "tc" else tps.pruned_attn_mma
         self.flops = 4.0 * self.d * self.H * self.k * self.N
         self.units = self.k
-        self.launches = sum(self.LAUNCHES.values())
+        self.launches = sum(self.LAUNCHES.values()) - 1 + attn_launches(tps, attn, self.k, self.N, self.H, self.d)
 
     def new_buffers(self, dev):
         t = self.tps
@@ -1330,7 +1339,7 @@ def main():
         "config": hsa_config(world),
         "impl_details": {"attn_kernel": kernel, "cuda_graphs": graphs},
         "active_tokens_per_s": round(tok_s, 1),
-        "gpu_launches": sum(HsaStep.LAUNCHES.values()) * a.steps,
+        "gpu_launches": st.launches * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
         "mid": mid, "keep_sweep_wan": sweep, "configs": configs, "cpu_baseline_configs": cpu_configs,
     }

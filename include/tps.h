@@ -285,11 +285,13 @@ TPS_API int kv_rerotate(const tps_bf16* k_cache, const int32_t* idx, const int32
  * scale must be finite and > 0 (typically 1/sqrt(d)).
  * bf16 inputs, fp32 accumulation and softmax, tcgen05 tensor cores.
  * d in {64, 128}; 1 <= H <= 256; N < 2^31; pointers 16-byte aligned.
- * Dense launches that would fill the GPU poorly (few 256-row query tiles x
- * heads, e.g. a low keep ratio) split the key range S <= 4 ways over a
+ * Dense launches whose last wave of 256-row query tiles x heads would be
+ * mostly empty (e.g. a low keep ratio) split the key range S <= 4 ways over a
  * thread-block cluster whose CTAs merge their partial results over
- * distributed shared memory (S from tps_attn_split; no workspace). Results
- * agree with the unsplit kernel within the attention tolerance. */
+ * distributed shared memory (no workspace): either the whole grid, or only
+ * the query tiles left after the grid's full waves, in a second launch on the
+ * same stream (tps_attn_plan reports which). Results agree with the unsplit
+ * kernel within the attention tolerance. */
 TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
                 const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
                 float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,
@@ -309,9 +311,18 @@ TPS_API int pruned_attn_ws(const tps_bf16* q_act, const tps_bf16* k, const tps_b
                            void* ws, size_t ws_bytes, tps_stream stream);
 TPS_API size_t tps_attn_workspace_size(int64_t cap, int64_t N, int H, int d);
 
-/* The key-range split S (1..4) a dense pruned_attn call of this shape runs
- * with on the current device (1 = unsplit). HOST query, no launch. */
+/* The key-range split S (1..4) of the whole grid of a dense pruned_attn call
+ * of this shape on the current device (1 = the grid is not split as a whole).
+ * HOST query, no launch. */
 TPS_API int tps_attn_split(int64_t cap, int64_t N, int H, int d);
+
+/* The launch plan of a dense pruned_attn call of this shape on the current
+ * device (HOST query, no launch): *split = whole-grid key split (1 = none);
+ * *main_rows = rows [0, main_rows) of the unsplit launch (cap when there is no
+ * tail launch); *tail_split = key split of the second launch that takes rows
+ * [main_rows, cap) (1 = no second launch). Pointers are HOST, non-NULL.
+ * Returns TPS_ERR_INVALID_ARG for a bad shape or a NULL pointer. */
+TPS_API int tps_attn_plan(int64_t cap, int64_t N, int H, int d, int* split, int64_t* main_rows, int* tail_split);
 
 /* Same contract as pruned_attn for dense attention with d = 128 (blockmask
  * must be NULL, else TPS_ERR_INVALID_ARG), computed on pairs of CTAs: one

@@ -159,6 +159,19 @@ def test_rerotate_validation():
     assert l.kv_rerotate(F, F, F, 10, 0, 2, 64, P(good), F, NULL) == tps.SHAPE
 
 
+def test_attn_plan_validation():
+    l = tps.lib()
+    s, t = C.c_int(0), C.c_int(0)
+    m = C.c_int64(0)
+    args = lambda cap, N, H, d: (cap, N, H, d, C.byref(s), C.byref(m), C.byref(t))   # noqa: E731
+    assert l.tps_attn_plan(*args(100, 0, 2, 128)) == tps.INVALID_ARG
+    assert l.tps_attn_plan(*args(100, 10, 2, 96)) == tps.INVALID_ARG
+    assert l.tps_attn_plan(*args(-1, 10, 2, 64)) == tps.INVALID_ARG
+    assert l.tps_attn_plan(100, 10, 2, 64, NULL, C.byref(m), C.byref(t)) == tps.INVALID_ARG
+    assert l.tps_attn_plan(*args(0, 10, 2, 64)) == tps.OK
+    assert (s.value, m.value, t.value) == (1, 0, 1)
+
+
 def test_front_validation():
     l = tps.lib()
     need = tps.workspace_min_size(tps.OP_FRONT, 100, 3)

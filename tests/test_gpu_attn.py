@@ -455,13 +455,15 @@ def test_attn_cluster_split_matches_oracle(N, S, d):
 
 def test_attn_cluster_split_wan_keep10_sampled():
     """The Wan-like layer at keep 10% (3276 queries x 32760 keys, 12 heads:
-    156 CTAs on 148 SMs) through pruned_attn: the cluster split is chosen and
-    matches the oracle on sampled rows."""
+    156 CTAs on 148 SMs) through pruned_attn: a cluster split is chosen (of the
+    whole grid or of the tiles past its full wave) and matches the oracle on
+    sampled rows."""
     Q, K, V = qkv("wan")
     N, H, d = Q.shape
     idx = oracle_idx("wan", 0)
     A = len(idx)
-    assert tps.attn_split(A, N, H, d) > 1
+    split, _, tail = tps.attn_plan(A, N, H, d)
+    assert split > 1 or tail > 1                            # the whole grid or its last tiles split
     o, lse = _run("pruned_attn", Q[idx], K, V, idx, 1 / math.sqrt(d))
     rows = _sample(A, 192, 6)
     o_ref, lse_ref = O.pruned_attn(Q[idx], K, V, idx, 1 / math.sqrt(d), rows=rows)
@@ -471,6 +473,54 @@ def test_attn_cluster_split_wan_keep10_sampled():
 def test_attn_no_cluster_split_when_grid_is_full():
     assert tps.attn_split(6084, 20280, 12, 128) == 1
     assert tps.attn_split(39600, 118800, 24, 128) == 1
+    assert tps.attn_plan(6084, 20280, 12, 128) == (1, 6084, 1)
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def test_attn_plan_hsa_tail():
+    """The HSA step's attention (155 tile pairs x 24 heads = 3720 units on 148
+    SMs, 25.1 waves): the full waves run unsplit and the last tile pair of
+    every head runs split 4 ways in a second launch."""
+    if _sms() != 148:
+        pytest.skip("plan figures are for 148 SMs")
+    split, main_rows, tail = tps.attn_plan(39600, 118800, 24, 128)
+    assert (split, main_rows, tail) == (1, 154 * 256, 4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_attn_tail_split_matches_oracle(d):
+    """A grid one wave and two tile pairs long (H = 1): the first launch takes
+    the full wave unsplit, the second the remaining tile pairs split over a
+    cluster. Sampled rows on both sides of the boundary and the ragged last
+    tile match the oracle; counts below cap (inside the first launch and
+    inside the tail) leave the rows past the count untouched."""
+    P = _sms()
+    H = 1
+    A = (P + 2) * 256 - 50
+    N = A + 1000
+    split, main_rows, tail = tps.attn_plan(A, N, H, d)
+    assert split == 1 and main_rows == P * 256 and tail > 1
+    q = synth.gaussian_bf16((A, H, d), 71)
+    k = synth.gaussian_bf16((N, H, d), 72).double()
+    k[N - 300:N - 200] *= 25.0                              # a spike inside the last key split
+    k = k.to(torch.bfloat16)
+    v = synth.gaussian_bf16((N, H, d), 73)
+    idx = np.sort(np.random.default_rng(d).choice(N, A, replace=False))
+    vmax = v.double().abs().amax(dim=(0, 2)).numpy()
+    b = main_rows
+    rows = np.unique(np.concatenate([_sample(A, 96, 5), np.arange(b - 3, b + 3), np.arange(A - 4, A)]))
+    o, lse = _run("pruned_attn", q, k, v, idx, 1 / math.sqrt(d))
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), rows=rows)
+    _check(o, lse, o_ref, lse_ref, rows=rows, v_absmax=vmax)
+    for count in (b - 100, b + 100):
+        o, lse = _run("pruned_attn", q, k, v, idx, 0.2, count=count)
+        sub = rows[rows < count]
+        o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 0.2, rows=sub)
+        _check(o, lse, o_ref, lse_ref, rows=sub, v_absmax=vmax)
+        assert torch.all(o[count:].float() == 7.0) and np.all(lse[count:] == 7.0)
 
 
 # -------------------------------------------------- CTA-pair kernel (d = 128) -----

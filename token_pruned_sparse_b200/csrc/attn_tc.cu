@@ -99,6 +99,7 @@ struct TcParams {
   float* lse_part;     // nsplit > 1, workspace merge: partial log-sum-exp, fp32 [nsplit][cap][H]
   int cluster;         // > 1: the nsplit CTAs of a cluster merge their partials over distributed
                        // shared memory (no workspace); 1 otherwise
+  int tile0;           // dense mode: first 256-row query tile of this launch (blockIdx.x + tile0)
 };
 constexpr int kMaxCluster = 4;
 
@@ -117,7 +118,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int64_t rows = active_count(p.count, p.cap);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kQT * kBM);
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) + prm.tile0) * (kQT * kBM);
   if (row0 >= rows) return;   // whole CTA exits before touching TMEM or barriers
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -872,7 +873,8 @@ int smem_attribute(int bytes) {
 // Masked (block mode): ceil(nb/2) x H CTAs, CTA x holding the active rows of
 // query blocks 2x and 2x+1, each tile with its own key list.
 template <int D>
-int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr) {
+int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr,
+           int64_t tile0 = 0, int64_t ntiles = -1) {
   if (a.cap == 0) return TPS_OK;
   EncodeTiledFn enc;
   if (int e = tensor_map_encoder(&enc, "pruned_attn")) return e;
@@ -883,7 +885,7 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mq, a.q, a.cap, a.H, a.d)) return e;
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
-  TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1};
+  TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1, static_cast<int>(tile0)};
   if (a.bm) {
     constexpr int kSmem = Layout<D, kQT>::kAlloc;
     if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
@@ -892,8 +894,8 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   } else {
     constexpr int kSmem = Layout<D, 1>::kAlloc;
     if (int e = smem_attribute<attn_tc_kernel<D, false>>(kSmem)) return e;
-    dim3 grid(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
-              static_cast<unsigned int>(nsplit));
+    if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
+    dim3 grid(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(nsplit));
     attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   }
   return launch_status("pruned_attn");
@@ -935,40 +937,70 @@ int cluster_slots(int S) {
   return slots;
 }
 
-// Key-range splits merged inside a thread-block cluster, for a dense launch
-// that would fill the GPU poorly: ceil(cap/256) x H CTAs that leave most of
-// their last wave empty run as S <= 4 key-range splits, the S CTAs of one
-// (query tile pair, head) forming a cluster along z that merges its partials
-// over distributed shared memory. S is chosen by wave efficiency against the
-// CTAs the GPU keeps resident in clusters of S; >= 4 key tiles per split.
+// How a dense launch runs. The unit of work is one 256-row query tile pair of
+// one head; an unsplit grid of U units on P SMs (one CTA each) takes
+// ceil(U / P) unit times. Two ways out of a mostly empty last wave:
+//  - the whole grid split S <= 4 ways along the keys, the S CTAs of a unit
+//    forming a cluster along z that merges its partials over distributed shared
+//    memory: ceil(U S / slots_S) / S unit times, slots_S = CTAs the GPU keeps
+//    resident in clusters of S;
+//  - the grid's full waves unsplit, then its remaining query tiles in a second
+//    launch split S_t ways: those waves plus the split tail.
+// A split pays its merge and cluster barriers (kSplitTax, measured on mid: 5%
+// at equal wave counts) and a second launch its gap (kLaunchGap, in unit
+// times); each split keeps >= 4 key tiles; a plan must gain 2% to be taken.
+struct DensePlan {
+  int split = 1;            // whole-grid key split (1: none)
+  int64_t main_tiles = 0;   // tiles of the unsplit launch (all of them without a tail)
+  int tail_split = 1;       // key split of the tail launch (1: no tail launch)
+};
+constexpr double kSplitTax = 1.06;
+constexpr double kLaunchGap = 0.02;
+
 template <int D>
-int choose_cluster_split(int64_t cap, int H, int64_t N) {
-  const int64_t units = ((cap + kQT * kBM - 1) / (kQT * kBM)) * H;
+DensePlan plan_dense(int64_t cap, int H, int64_t N) {
+  DensePlan plan;
+  const int64_t tiles = (cap + kQT * kBM - 1) / (kQT * kBM);
+  plan.main_tiles = tiles;
+  const int64_t units = tiles * H;
   const int64_t nkt = (N + kBN - 1) / kBN;
-  if (units <= 0) return 1;
-  const int64_t sms = sm_count();
-  if (static_cast<double>(units) / static_cast<double>(((units + sms - 1) / sms) * sms) >= 0.9) return 1;
-  // time in units of one unsplit CTA: waves of S-split CTAs, each doing 1/S of the keys
-  auto cost = [&](int S) -> double {
-    const int64_t slots = cluster_slots<D>(S);
+  const int64_t P = sm_count();
+  if (units <= 0 || P <= 0) return plan;
+  auto waves = [&](int64_t u, int S) -> double {   // unit times of u units split S ways
+    const int64_t slots = S == 1 ? P : cluster_slots<D>(S);
     if (slots <= 0) return 1e30;
-    return static_cast<double>((units * S + slots - 1) / slots) / S;
+    return static_cast<double>((u * S + slots - 1) / slots) / S * (S > 1 ? kSplitTax : 1.0);
   };
-  int best = 1;
-  double bc = cost(1);
-  for (int S = 2; S <= kMaxCluster; ++S) {
-    if (nkt < 4 * S) break;
-    const double c = cost(S);
-    if (c < 0.98 * bc) {
-      best = S;
-      bc = c;
+  const double base = waves(units, 1);
+  double best = base;
+  for (int S = 2; S <= kMaxCluster && nkt >= 4 * S; ++S) {
+    const double c = waves(units, S);
+    if (c < best) {
+      best = c;
+      plan.split = S;
     }
   }
-  return best;
+  const int64_t full = units / P;
+  const int64_t t1 = full * P / H;                 // tiles that fit the full waves
+  if (full >= 1 && t1 >= 1 && t1 < tiles) {
+    const double main_cost = waves(t1 * H, 1) + kLaunchGap;
+    const int64_t ut = (tiles - t1) * H;
+    for (int S = 2; S <= kMaxCluster && nkt >= 4 * S; ++S) {
+      const double c = main_cost + waves(ut, S);
+      if (c < best) {
+        best = c;
+        plan.split = 1;
+        plan.main_tiles = t1;
+        plan.tail_split = S;
+      }
+    }
+  }
+  if (best > 0.98 * base) plan = DensePlan{1, tiles, 1};
+  return plan;
 }
 
 template <int D>
-int launch_cluster(const AttnArgs& a, cudaStream_t st, int S) {
+int launch_cluster(const AttnArgs& a, cudaStream_t st, int S, int64_t tile0 = 0, int64_t ntiles = -1) {
   EncodeTiledFn enc;
   if (int e = tensor_map_encoder(&enc, "pruned_attn")) return e;
   int err;
@@ -979,10 +1011,10 @@ int launch_cluster(const AttnArgs& a, cudaStream_t st, int S) {
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   if (int e = smem_attribute<attn_tc_kernel<D, true>>(Layout<D, 1>::kAlloc)) return e;
-  TcParams prm{a, a.scale * kLog2e, status, S, nullptr, nullptr, S};
+  TcParams prm{a, a.scale * kLog2e, status, S, nullptr, nullptr, S, static_cast<int>(tile0)};
+  if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned int>((a.cap + kQT * kBM - 1) / (kQT * kBM)), static_cast<unsigned int>(a.H),
-                     static_cast<unsigned int>(S));
+  cfg.gridDim = dim3(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(S));
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cfg.stream = st;
@@ -1095,7 +1127,20 @@ extern "C" int pruned_attn_pair(const tps_bf16* q_act, const tps_bf16* k, const 
 extern "C" int tps_attn_split(int64_t cap, int64_t N, int H, int d) {
   using namespace tps;
   if (cap <= 0 || N <= 0 || H <= 0 || (d != 64 && d != 128)) return 1;
-  return d == 64 ? choose_cluster_split<64>(cap, H, N) : choose_cluster_split<128>(cap, H, N);
+  return (d == 64 ? plan_dense<64>(cap, H, N) : plan_dense<128>(cap, H, N)).split;
+}
+
+extern "C" int tps_attn_plan(int64_t cap, int64_t N, int H, int d, int* split, int64_t* main_rows, int* tail_split) {
+  using namespace tps;
+  if (!split || !main_rows || !tail_split) return fail(TPS_ERR_INVALID_ARG, "tps_attn_plan: null pointer");
+  if (cap < 0 || N <= 0 || H <= 0 || (d != 64 && d != 128))
+    return fail(TPS_ERR_INVALID_ARG, "tps_attn_plan: need cap >= 0, N > 0, H > 0, d in {64, 128}");
+  DensePlan plan;
+  if (cap > 0) plan = d == 64 ? plan_dense<64>(cap, H, N) : plan_dense<128>(cap, H, N);
+  *split = plan.split;
+  *main_rows = plan.tail_split > 1 ? plan.main_tiles * (kQT * kBM) : cap;
+  *tail_split = plan.tail_split;
+  return ok();
 }
 
 extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v, const int32_t* idx,
@@ -1108,10 +1153,21 @@ extern "C" int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_b
                             lse, &a))
     return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (blockmask || cap == 0) {
+    const int e = d == 64 ? launch<64>(a, st) : launch<128>(a, st);
+    return e ? e : ok();
+  }
+  const DensePlan plan = d == 64 ? plan_dense<64>(cap, H, N) : plan_dense<128>(cap, H, N);
   int e;
-  const int S = blockmask || cap == 0 ? 1 : (d == 64 ? choose_cluster_split<64>(cap, H, N)
-                                                     : choose_cluster_split<128>(cap, H, N));
-  if (S > 1) e = d == 64 ? launch_cluster<64>(a, st, S) : launch_cluster<128>(a, st, S);
-  else e = d == 64 ? launch<64>(a, st) : launch<128>(a, st);
+  if (plan.split > 1) {
+    e = d == 64 ? launch_cluster<64>(a, st, plan.split) : launch_cluster<128>(a, st, plan.split);
+  } else {
+    e = d == 64 ? launch<64>(a, st, 1, nullptr, nullptr, 0, plan.main_tiles)
+                : launch<128>(a, st, 1, nullptr, nullptr, 0, plan.main_tiles);
+    const int64_t tiles = (cap + kQT * kBM - 1) / (kQT * kBM);
+    if (!e && plan.tail_split > 1)
+      e = d == 64 ? launch_cluster<64>(a, st, plan.tail_split, plan.main_tiles, tiles - plan.main_tiles)
+                  : launch_cluster<128>(a, st, plan.tail_split, plan.main_tiles, tiles - plan.main_tiles);
+  }
   return e ? e : ok();
 }

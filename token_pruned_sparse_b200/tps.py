@@ -42,6 +42,7 @@ SIGNATURES = {
                               C.c_size_t, _P]),
     "tps_attn_workspace_size": (C.c_size_t, [_I64, _I64, _INT, _INT]),
     "tps_attn_split": (_INT, [_I64, _I64, _INT, _INT]),
+    "tps_attn_plan": (_INT, [_I64, _I64, _INT, _INT, _P, _P, _P]),
     "pruned_attn_pair": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "pruned_attn_mma": (_INT, [_P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, C.c_float, _P, _INT, _P, _P, _P]),
     "scatter_out": (_INT, [_P, _P, _P, _P, _I64, _I64, _INT, _INT, _P]),
@@ -270,8 +271,16 @@ def attn_workspace(cap, N, H, d, device=None):
 
 
 def attn_split(cap, N, H, d) -> int:
-    """Key-range split a dense pruned_attn call of this shape uses (1 = none)."""
+    """Whole-grid key-range split a dense pruned_attn call of this shape uses (1 = none)."""
     return int(lib().tps_attn_split(int(cap), int(N), int(H), int(d)))
+
+
+def attn_plan(cap, N, H, d):
+    """(split, main_rows, tail_split) of a dense pruned_attn call of this shape."""
+    split, tail = C.c_int(0), C.c_int(0)
+    main = C.c_int64(0)
+    _chk(lib().tps_attn_plan(int(cap), int(N), int(H), int(d), C.byref(split), C.byref(main), C.byref(tail)))
+    return split.value, main.value, tail.value
 
 
 def pruned_attn_ws(q_act, k, v, idx, count, scale, blockmask=None, block=128, o_act=None, lse=None, cap=None,
