@@ -852,9 +852,11 @@ def kernel_case(name, dev):
 
     attn_mid: one mid-size attention launch (6084 queries x 20280 keys, 12
     heads). attn_hsa_h8: the HSA step's attention (39600 queries x 118800
-    keys) on 8 of its 24 heads (the grid still fills the GPU, so the launch
-    runs unsplit like the full one); heads are independent units of the grid,
-    so a full launch moves 3x these bytes. overlap_hsa is not a capture case:
+    keys) on 8 of its 24 heads: the grid still fills the GPU, so the call runs
+    like the full one, its full waves unsplit and its remaining query tiles
+    split in a second launch (capture both launches of the second call);
+    heads are independent units of the grid, so a full call moves about 3x
+    these bytes. overlap_hsa is not a capture case:
     it times the HSA step's host transfers alone and beside the attention."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
@@ -1294,6 +1296,7 @@ def main():
     roofline["frac_of_burst"] = round(roofline["achieved"] / float(pk["bf16_tflops"]), 4)
     e2e = None if a.no_e2e else e2e_leg(st, dev, max(3, min(a.steps, 20)), world)
     graphs = bool(getattr(st, "graphs", False))
+    launches = st.launches
     del st
     torch.cuda.empty_cache()
 
@@ -1339,7 +1342,7 @@ def main():
         "config": hsa_config(world),
         "impl_details": {"attn_kernel": kernel, "cuda_graphs": graphs},
         "active_tokens_per_s": round(tok_s, 1),
-        "gpu_launches": st.launches * a.steps,
+        "gpu_launches": launches * a.steps,
         "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
         "mid": mid, "keep_sweep_wan": sweep, "configs": configs, "cpu_baseline_configs": cpu_configs,
     }
