@@ -32,6 +32,9 @@
 //   warp 9     MMA issuer and TMEM owner. Per key tile j and tile t:
 //              O_t += P_t(j) V_j (A operand read from TMEM), then
 //              S_t(j+1) = Q_t K_{j+1}^T; completion via tcgen05.commit.
+//   warps 10-11 (dense kernel only) idle: with warps 8-9 they form a producer
+//              warpgroup that gives up registers (setmaxnreg) so that each softmax
+//              thread holds S and P of a whole tile (232 registers) without spilling.
 // While softmax t works on S_t(j+1), the tensor cores run the other tile's
 // P V and Q K^T, so MMA and softmax overlap.
 // TMEM: tile t owns columns [256t, 256t+128) for S/P and [256t+128, +D) for O.
@@ -54,6 +57,15 @@ constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
 constexpr int kSoftmaxThreads = kQT * kBM;
 constexpr int kThreads = kSoftmaxThreads + 64;   // + TMA warp + MMA warp
+// The dense kernel runs a fourth warpgroup (TMA warp, MMA warp, two idle warps) that
+// hands registers to the two softmax warpgroups (setmaxnreg). 12 warps put 3 on each
+// SM sub-partition, so the launch allots 16384 / (3 * 32) -> 168 registers per thread;
+// the softmax warps then hold S and P of a whole tile without spilling.
+constexpr int kDenseThreads = kSoftmaxThreads + 128;
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 40;
+constexpr int kSoftmaxRegs = 232;
+static_assert(8 * kSoftmaxRegs + 4 * kProducerRegs <= 12 * kLaunchRegs, "register split exceeds the launch");
 constexpr int kWarps = kThreads / 32;
 constexpr int kTmaWarp = kSoftmaxThreads / 32;
 constexpr int kMmaWarp = kTmaWarp + 1;
@@ -103,9 +115,23 @@ struct TcParams {
 };
 constexpr int kMaxCluster = 4;
 
+// CTA and cluster barriers; the non-aligned forms when warps reach them from
+// different code (each warpgroup running its own copy of the kernel's tail).
+template <bool kNonAligned>
+__device__ __forceinline__ void cta_sync() {
+  if constexpr (kNonAligned) asm volatile("barrier.sync 0;" ::: "memory");
+  else __syncthreads();
+}
+template <bool kNonAligned>
+__device__ __forceinline__ void cluster_sync() {
+  if constexpr (kNonAligned)
+    asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;" ::: "memory");
+  else cluster_sync_all();
+}
+
 
 template <int D, bool kClu>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDenseThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams prm) {
   using L = Layout<D, 1>;
@@ -164,7 +190,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   auto tO = [&](int t) { return tmem + 256u * t + 128u; };   // O_t accumulator
   auto tile_kb = [&](int j) -> int { return kt0 + j; };
 
-  if (warp == kTmaWarp) {
+  auto tma_role = [&]() {
     // ================================ TMA producer =====================================
     if (lane == 0) {
       int issued_k = 0, issued_v = 0;
@@ -199,7 +225,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int j = issued_v > kStages ? issued_v - kStages : 0; j < issued_v; ++j)
         drain_wait(bar(Bars::v_full + j % kStages), (j / kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
+  };
+  auto mma_role = [&]() {
     // ================================ MMA issuer =======================================
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, false, false);  // Q K^T: both K-major
@@ -253,7 +280,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       mma_commit(bar(Bars::drain));   // fires once every MMA issued above has completed
     }
-  } else {
+  };
+  auto softmax_role = [&]() {
     // ================================ softmax warps ====================================
     const int t = warp >> 2;                      // query tile of this warpgroup
     const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
@@ -402,8 +430,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
-  }
-
+  };
+  // the common tail; each warpgroup runs its own copy, so its CTA and cluster barriers
+  // are the non-aligned forms
+  auto tail = [&]() {
   // ---- split-key merge inside the cluster ------------------------------------------------
   // After every CTA has staged its partials (cluster barrier, release/acquire at
   // cluster scope), CTA rank k merges rows [k*R, (k+1)*R) of the 256, R =
@@ -411,8 +441,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // memory: two threads per row, each half a row. The second barrier keeps
   // every CTA's shared memory valid until its peers have read it.
   if constexpr (kClu) {
-    __syncthreads();                                   // warps converged for the aligned barrier
-    cluster_sync_all();
+    cta_sync<true>();                                   // warps converged for the aligned barrier
+    cluster_sync<true>();
     constexpr int kChunks = D / 4;
     const int S = prm.cluster;
     const int R = (kQT * kBM + S - 1) / S;
@@ -472,18 +502,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (valid && half == 0 && p.lse) p.lse[row * p.H + h] = l > 0.f ? (M + __log2f(l)) * kLn2 : -INFINITY;
     }
-    __syncthreads();
-    cluster_sync_all();
+    cta_sync<true>();
+    cluster_sync<true>();
   }
 
   // ---- teardown ------------------------------------------------------------------------
   if (warp == kMmaWarp && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
   tc_fence_before();
-  __syncthreads();
+  cta_sync<true>();
   tc_fence_after();
   if (warp == kMmaWarp) {
     __syncwarp();
     tmem_dealloc<kTmemCols>(tmem);
+  }
+  };
+  // the producer warpgroup (TMA, MMA and two idle warps) hands registers to the two
+  // softmax warpgroups; each side then runs to the end on its own (ptxas allots a
+  // region the registers of its setmaxnreg only if the region does not rejoin the
+  // other warps' code)
+  if (warp >= kTmaWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kTmaWarp) tma_role();
+    else if (warp == kMmaWarp) mma_role();
+    tail();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    softmax_role();
+    tail();
   }
 }
 
@@ -896,7 +941,7 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
     if (int e = smem_attribute<attn_tc_kernel<D, false>>(kSmem)) return e;
     if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
     dim3 grid(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(nsplit));
-    attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+    attn_tc_kernel<D, false><<<grid, kDenseThreads, kSmem, st>>>(mq, mk, mv, prm);
   }
   return launch_status("pruned_attn");
 }
@@ -918,7 +963,7 @@ int cluster_slots(int S) {
   if (smem_attribute<attn_tc_kernel<D, true>>(Layout<D, 1>::kAlloc)) return 0;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(1, 1, static_cast<unsigned int>(S));
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kDenseThreads, 1, 1);
   cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1015,7 +1060,7 @@ int launch_cluster(const AttnArgs& a, cudaStream_t st, int S, int64_t tile0 = 0,
   if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(S));
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kDenseThreads, 1, 1);
   cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
