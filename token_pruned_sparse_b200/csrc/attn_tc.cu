@@ -32,9 +32,9 @@
 //   warp 9     MMA issuer and TMEM owner. Per key tile j and tile t:
 //              O_t += P_t(j) V_j (A operand read from TMEM), then
 //              S_t(j+1) = Q_t K_{j+1}^T; completion via tcgen05.commit.
-//   warps 10-11 (dense kernel only) idle: with warps 8-9 they form a producer
-//              warpgroup that gives up registers (setmaxnreg) so that each softmax
-//              thread holds S and P of a whole tile (232 registers) without spilling.
+//   warps 10-11 idle: with warps 8-9 they form a producer warpgroup that gives
+//              up registers (setmaxnreg) so that each softmax thread holds S and P
+//              of a whole tile (232 registers) without spilling.
 // While softmax t works on S_t(j+1), the tensor cores run the other tile's
 // P V and Q K^T, so MMA and softmax overlap.
 // TMEM: tile t owns columns [256t, 256t+128) for S/P and [256t+128, +D) for O.
@@ -56,17 +56,15 @@ constexpr int kQT = 2;          // query tiles per CTA
 constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
 constexpr int kSoftmaxThreads = kQT * kBM;
-constexpr int kThreads = kSoftmaxThreads + 64;   // + TMA warp + MMA warp
-// The dense kernel runs a fourth warpgroup (TMA warp, MMA warp, two idle warps) that
-// hands registers to the two softmax warpgroups (setmaxnreg). 12 warps put 3 on each
-// SM sub-partition, so the launch allots 16384 / (3 * 32) -> 168 registers per thread;
-// the softmax warps then hold S and P of a whole tile without spilling.
-constexpr int kDenseThreads = kSoftmaxThreads + 128;
+// + a fourth warpgroup (TMA warp, MMA warp, two idle warps) that hands registers to
+// the two softmax warpgroups (setmaxnreg). 12 warps put 3 on each SM sub-partition,
+// so the launch allots 16384 / (3 * 32) -> 168 registers per thread; the softmax
+// warps then hold S and P of a whole tile without spilling.
+constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kLaunchRegs = 168;
 constexpr int kProducerRegs = 40;
 constexpr int kSoftmaxRegs = 232;
 static_assert(8 * kSoftmaxRegs + 4 * kProducerRegs <= 12 * kLaunchRegs, "register split exceeds the launch");
-constexpr int kWarps = kThreads / 32;
 constexpr int kTmaWarp = kSoftmaxThreads / 32;
 constexpr int kMmaWarp = kTmaWarp + 1;
 constexpr int kTmemCols = 512;
@@ -131,7 +129,7 @@ __device__ __forceinline__ void cluster_sync() {
 
 
 template <int D, bool kClu>
-__global__ void __launch_bounds__(kDenseThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams prm) {
   using L = Layout<D, 1>;
@@ -549,7 +547,7 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __shared__ int s_nrows[kQT];
   __shared__ int s_row0[kQT];
   __shared__ volatile int s_abort;
-  __shared__ unsigned int s_wcnt[kQT][kWarps];
+  __shared__ unsigned int s_wcnt[kQT][kThreads / 32];
 
   const AttnArgs& p = prm.a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -625,7 +623,7 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncthreads();
       for (int t = 0; t < kQT; ++t) {
         int off = base[t], tot = 0;
-        for (int i = 0; i < kWarps; ++i) {
+        for (int i = 0; i < kThreads / 32; ++i) {
           off += i < warp ? s_wcnt[t][i] : 0;
           tot += s_wcnt[t][i];
         }
@@ -650,7 +648,7 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     return (j < n0 ? j : n0) + (j < n1 ? j : n1) + (t == 1 && j < n0 ? 1 : 0);
   };
 
-  if (warp == kTmaWarp) {
+  auto tma_role = [&]() {
     // ================================ TMA producer =====================================
     if (lane == 0) {
       int issued_k = 0, issued_v = 0;
@@ -697,7 +695,8 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int q = issued_v > kStages ? issued_v - kStages : 0; q < issued_v; ++q)
         drain_wait(bar(Bars::v_full + q % kStages), (q / kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
+  };
+  auto mma_role = [&]() {
     // ================================ MMA issuer =======================================
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kBM, kBN, false, false);  // Q K^T: both K-major
@@ -757,7 +756,8 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       mma_commit(bar(Bars::drain));   // fires once every MMA issued above has completed
     }
-  } else {
+  };
+  auto softmax_role = [&]() {
     // ================================ softmax warps ====================================
     const int t = warp >> 2;                      // query tile of this warpgroup
     const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
@@ -871,16 +871,29 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (valid && p.lse) p.lse[row * p.H + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
-  }
-
+  };
+  // the common tail; each warpgroup runs its own copy (non-aligned barrier)
+  auto tail = [&]() {
   // ---- teardown ------------------------------------------------------------------------
   if (warp == kMmaWarp && lane == 0) drain_wait(bar(Bars::drain), 0);   // no MMA may still write TMEM
   tc_fence_before();
-  __syncthreads();
+  cta_sync<true>();
   tc_fence_after();
   if (warp == kMmaWarp) {
     __syncwarp();
     tmem_dealloc<kTmemCols>(tmem);
+  }
+  };
+  // registers from the producer warpgroup to the softmax warpgroups (as in attn_tc_kernel)
+  if (warp >= kTmaWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kTmaWarp) tma_role();
+    else if (warp == kMmaWarp) mma_role();
+    tail();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    softmax_role();
+    tail();
   }
 }
 
@@ -941,7 +954,7 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
     if (int e = smem_attribute<attn_tc_kernel<D, false>>(kSmem)) return e;
     if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
     dim3 grid(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(nsplit));
-    attn_tc_kernel<D, false><<<grid, kDenseThreads, kSmem, st>>>(mq, mk, mv, prm);
+    attn_tc_kernel<D, false><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
   }
   return launch_status("pruned_attn");
 }
@@ -963,7 +976,7 @@ int cluster_slots(int S) {
   if (smem_attribute<attn_tc_kernel<D, true>>(Layout<D, 1>::kAlloc)) return 0;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(1, 1, static_cast<unsigned int>(S));
-  cfg.blockDim = dim3(kDenseThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1060,7 +1073,7 @@ int launch_cluster(const AttnArgs& a, cudaStream_t st, int S, int64_t tile0 = 0,
   if (ntiles < 0) ntiles = (a.cap + kQT * kBM - 1) / (kQT * kBM);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned int>(ntiles), static_cast<unsigned int>(a.H), static_cast<unsigned int>(S));
-  cfg.blockDim = dim3(kDenseThreads, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = Layout<D, 1>::kAlloc;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
