@@ -1305,7 +1305,11 @@ def main():
     if not a.no_mid:
         ms = MidStep(rank_seed_offset(rank), dev, a.attn)
         msteps = max(a.steps, 100)
+        msampler = ClockSampler(local)
+        msampler.start()
+        time.sleep(0.3)
         m_total, m_attn = run_path(ms, msteps, a.warmup, world, not a.no_graph, flush, dev)
+        mclocks = msampler.stop()
         mid = {"workload": "mid: 13x30x52 = 20280 tokens, 12 heads, d=128, inter-frame rel-L1 score, top-k 30% = "
                            "6084 active queries x 20280 keys; step = score+select+gather+kv_sync+pruned_attn+"
                            "scatter_out",
@@ -1314,7 +1318,10 @@ def main():
                "active_tokens_per_s": round(job_throughput(ms.units, world, msteps, m_total), 1),
                "roofline": roofline_block(ms.flops, m_attn, float(pk["bf16_tflops"]), f"bf16 dense burst ({pk_kind})",
                                           recorded_traffic("pruned_attn_mid.json") if a.attn == "tc" else None,
-                                          kernel)}
+                                          kernel),
+               "clocks": mclocks}
+        # the 0.6 ms launches run back to back for the whole timed region: the sustained figure, beside
+        mid["roofline"]["frac_of_sustained"] = round(mid["roofline"]["achieved"] / float(pk["bf16_tflops_sustained"]), 4)
         if not a.no_e2e:
             mid["e2e"] = e2e_leg(ms, dev, max(3, min(msteps, 50)), world)
         del ms
