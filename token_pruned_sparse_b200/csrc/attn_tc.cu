@@ -897,12 +897,532 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
+// ---- block mode, transposed products (d = 128) ------------------------------------------------
+// A query block keeps few of its 128 tokens active (about 51 at 40% kept), so an M = 128 tile of
+// query rows is mostly padding. Here the 128 keys of a key tile are the MMA's M and a unit of at
+// most 64 active rows of one query block is its N:
+//   S^T  = K Q^T     [128 keys x 64 rows]:     A = K tile (K-major), B = Q rows (K-major)
+//   O^T += V^T P^T   [128 channels x 64 rows]: A = V tile read MN-major, B = P^T (MN-major)
+// CTA (x, h, z) takes rows [64z, 64z + 64) of the active runs of query blocks 2x and 2x + 1 as
+// units 0 and 1, one after the other: one stream of key tiles g = 0, 1, ... (unit 0's list, then
+// unit 1's) through two-stage K and V rings. S^T and P^T are double-buffered (TMEM and shared
+// memory), so the MMAs of tiles g + 2 and g overlap the softmax of tile g + 1.
+// The eight softmax warps split a tile's 64 columns: warpgroup w takes columns [32w, 32w + 32);
+// thread r of it owns key r of S^T (TMEM lane r) and channel r of O^T. The reference maximum is
+// one per column (query row), shared by the 128 key threads of its warpgroup: after a unit's
+// first key tile it changes only when an exponent argument exceeds kXLimit somewhere in the
+// warpgroup's half of the tile, which one barrier reduction over the warpgroup decides. The two
+// warpgroups share no barrier. The per-column sums stay in the key threads' registers and are
+// reduced across threads once per unit.
+// The single MMA-issuing thread is the pipeline's serial stage (each tcgen05.mma of N = 64 and
+// each tcgen05.commit costs it tens of cycles), so it commits twice per tile: S^T(g)'s commit
+// also frees K stage g % 2, and P V(g)'s commit frees V stage g % 2 and tells the softmax that
+// O^T holds tile g.
+namespace blkt {
+constexpr int kUR = 64;                 // query rows per unit (MMA N)
+constexpr int kHalf = kUR / 2;          // columns per softmax warpgroup
+constexpr int kQSub = kUR * 128;        // one [64 rows x 64 bf16] swizzled Q sub-tile
+constexpr int kPTBytes = 128 * 128;     // P^T of one tile: 128 keys x 64 rows bf16 (one 128-byte row per key)
+constexpr float kXLimit = 64.f;         // largest exponent argument (log2) kept without a new reference
+constexpr int kTmemColsT = 256;         // S^T buffers at [0, 64) and [64, 128); O^T of unit u at [128 + 64u, +64)
+
+struct LayoutT {
+  static constexpr int kSub = 2;                                // d = 128: two 64-wide sub-tiles
+  static constexpr int kQ = 0;                                  // [unit][sub] x kQSub
+  static constexpr int kK = kQ + kQT * kSub * kQSub;            // [stage][sub] x kSubBytes
+  static constexpr int kV = kK + kStages * kSub * kSubBytes;
+  static constexpr int kPT = kV + kStages * kSub * kSubBytes;   // [buffer] x kPTBytes
+  static constexpr int kRed = kPT + 2 * kPTBytes;               // float [warpgroup][warp][kHalf]: column folds
+  static constexpr int kRef = kRed + 2 * 4 * kHalf * 4;         // float [kUR]: minus the reference (log2)
+  static constexpr int kAux = kRef + kUR * 4;                   // float [kUR]: rescale factors, then 1/l
+  static constexpr int kList = kAux + kUR * 4;                  // uint16 [unit][kListMax]: kept key blocks
+  static constexpr int kListMax = 4096;
+  static constexpr int kBar = kList + kQT * kListMax * 2;
+  static constexpr int kBytes = kBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+static_assert(LayoutT::kK % 1024 == 0 && LayoutT::kV % 1024 == 0 && LayoutT::kPT % 1024 == 0, "swizzle atoms");
+static_assert(LayoutT::kAlloc <= 227 * 1024, "shared memory");
+
+static_assert(kStages == 2, "S^T buffer g % 2 and K stage g % 2 share their barrier");
+struct BarsT {  // mbarrier indices (8 bytes each)
+  static constexpr int q_full = 0;                     // + unit
+  static constexpr int k_full = q_full + kQT;          // + stage
+  static constexpr int v_full = k_full + kStages;      // + stage
+  static constexpr int s_full = v_full + kStages;      // + g % 2: S^T(g) complete, K stage g % 2 free
+  static constexpr int pv_done = s_full + 2;           // + g % 2: P V(g) complete, V stage g % 2 free
+  static constexpr int p_full = pv_done + 2;           // + g % 2: P^T(g) written (256 arrivals)
+  static constexpr int drain = p_full + 2;             // last commit of the MMA thread
+  static constexpr int count = drain + 1;
+};
+static_assert(BarsT::count * 8 <= 256, "barrier block");
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Barrier of one softmax warpgroup (named barrier `id`, 128 threads).
+__device__ __forceinline__ void wg_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+// Barrier of one softmax warpgroup that also returns the OR of `pred` over its 128 threads.
+__device__ __forceinline__ bool wg_any(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, %2, 128, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id)
+      : "memory");
+  return r != 0;
+}
+// Shared-memory descriptor (128-byte swizzle, SBO 1024) as two 32-bit words: lo = start address
+// >> 4 | LBO >> 4 << 16, hi = SBO >> 4 | version | swizzle mode. Adding (offset >> 4) to lo moves
+// the start address (shared addresses stay below 2^18, so the 14-bit field cannot carry).
+__host__ __device__ constexpr uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) { return (saddr >> 4) | ((lbo >> 4) << 16); }
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ void mma_ss_words(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\n.reg .b64 da, db;\nsetp.ne.b32 p, %4, 0;\nmov.b64 da, {%1, %5};\nmov.b64 db, {%2, %5};\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kDescHi)
+      : "memory");
+}
+// Folds 32 per-thread column values across the warp's 32 lanes by recursive halving (max or
+// sum); afterwards lane l holds the warp's result for column l in v[0].
+template <bool kMax>
+__device__ __forceinline__ void warp_fold32(float (&v)[kHalf], int lane) {
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int o = 16 >> s, n = kHalf >> s;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = up ? v[i] : v[i + n / 2];
+      const float keep = up ? v[i + n / 2] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+}
+}  // namespace blkt
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, TcParams prm) {
+  using namespace blkt;
+  constexpr int D = 128;
+  using L = LayoutT;
+  using B = BarsT;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_ntiles[kQT];
+  __shared__ int s_nrows[kQT];
+  __shared__ int s_row0[kQT];
+  __shared__ volatile int s_abort;
+  __shared__ unsigned int s_wcnt[kQT][kThreads / 32];
+
+  const AttnArgs& p = prm.a;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y;
+  const int64_t rows = active_count(p.count, p.cap);
+
+  // ---- the query rows of each unit --------------------------------------------------------
+  {
+    if (warp == 0) {
+      // lane 2u: first row of query block 2x + u; lane 2u + 1: one past its last (lower bounds in idx)
+      const int64_t key = (2 * static_cast<int64_t>(blockIdx.x) + (lane >> 1) + (lane & 1)) * 128;
+      int64_t lo = 0, hi = rows;
+      while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (p.idx[mid] < key) lo = mid + 1;
+        else hi = mid;
+      }
+      const int64_t end = __shfl_down_sync(0xffffffffu, lo, 1);
+      if (lane < 2 * kQT && (lane & 1) == 0) {
+        const int64_t r0 = lo + static_cast<int64_t>(kUR) * blockIdx.z;
+        const int64_t n = end - r0;
+        s_row0[lane >> 1] = static_cast<int>(r0 < rows ? r0 : rows);
+        s_nrows[lane >> 1] = static_cast<int>(n < 0 ? 0 : (n > kUR ? kUR : n));
+      }
+    }
+    __syncthreads();
+    if (s_nrows[0] == 0 && s_nrows[1] == 0) return;   // uniform: before TMEM or barriers
+  }
+
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - smem_u32(smem_raw));
+  uint16_t* sList = reinterpret_cast<uint16_t*>(gbase + L::kList);   // [unit][kListMax]
+  const uint32_t bar0 = sbase + L::kBar;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  // ---- setup: barriers, TMEM, key-tile lists ------------------------------------------------
+  if (tid == 0) {
+    s_abort = 0;
+    for (int u = 0; u < kQT; ++u) mbar_init(bar(B::q_full + u), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B::k_full + s), 1);
+      mbar_init(bar(B::v_full + s), 1);
+      mbar_init(bar(B::s_full + s), 1);
+      mbar_init(bar(B::pv_done + s), 1);
+      mbar_init(bar(B::p_full + s), kSoftmaxThreads);
+    }
+    mbar_init(bar(B::drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) tmem_alloc<kTmemColsT>(smem_u32(&s_tmem));
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  {
+    // unit u's key list: the key blocks its query block keeps, ascending
+    int base[kQT] = {0, 0};
+    const uint8_t* mrow[kQT];
+    for (int u = 0; u < kQT; ++u)
+      mrow[u] = p.bm + (2 * static_cast<int64_t>(blockIdx.x) + u) * p.nb;
+    for (int kb0 = 0; kb0 < p.nb; kb0 += kThreads) {
+      const int kb = kb0 + tid;
+      unsigned int m[kQT];
+      for (int u = 0; u < kQT; ++u) {
+        const bool keep = s_nrows[u] > 0 && kb < p.nb && mrow[u][kb] != 0;
+        m[u] = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) s_wcnt[u][warp] = __popc(m[u]);
+      }
+      __syncthreads();
+      for (int u = 0; u < kQT; ++u) {
+        int off = base[u], tot = 0;
+        for (int i = 0; i < kThreads / 32; ++i) {
+          off += i < warp ? s_wcnt[u][i] : 0;
+          tot += s_wcnt[u][i];
+        }
+        if ((m[u] >> lane) & 1u)
+          sList[u * L::kListMax + off + __popc(m[u] & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb);
+        base[u] += tot;
+      }
+      __syncthreads();
+    }
+    if (tid < kQT) s_ntiles[tid] = base[tid];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  auto tS = [&](int b) { return tmem + 64u * b; };           // S^T buffer b (fp32, 64 columns)
+  auto tO = [&](int u) { return tmem + 128u + 64u * u; };    // O^T of unit u (fp32, 64 columns)
+  const int n0 = s_ntiles[0], nt = n0 + s_ntiles[1];          // key tiles of unit 0, of both
+  auto unit_of = [&](int g) { return g < n0 ? 0 : 1; };
+  auto step_of = [&](int g) { return g < n0 ? g : g - n0; };  // position in its unit's list
+  auto tile_kb = [&](int g) -> int { return static_cast<int>(sList[unit_of(g) * L::kListMax + step_of(g)]); };
+
+  auto tma_role = [&]() {
+    // ================================ TMA producer =====================================
+    if (lane == 0) {
+      int issued_k = 0, issued_v = 0;
+      bool q_issued[kQT];
+      for (int u = 0; u < kQT; ++u) {
+        q_issued[u] = s_ntiles[u] > 0;
+        if (!q_issued[u]) continue;
+        mbar_expect_tx(bar(B::q_full + u), L::kSub * kQSub);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kQ + (u * L::kSub + s) * kQSub, &tmQ, 64 * s, h, s_row0[u], bar(B::q_full + u));
+      }
+      // K and V stages are freed separately: K stage g % 2 when S^T(g) completes (two tiles
+      // ahead of its P V), V stage g % 2 when P V(g) does
+      for (int g = 0; g < nt; ++g) {
+        const int st = g % kStages;
+        const uint32_t ph = ((g / kStages) - 1) & 1;
+        const int key0 = tile_kb(g) * kBN;
+        if (g >= kStages && !mbar_wait(bar(B::s_full + st), ph, &s_abort, prm.status)) break;
+        mbar_expect_tx(bar(B::k_full + st), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kK + (st * L::kSub + s) * kSubBytes, &tmK, 64 * s, h, key0, bar(B::k_full + st));
+        issued_k = g + 1;
+        if (g >= kStages && !mbar_wait(bar(B::pv_done + st), ph, &s_abort, prm.status)) break;
+        mbar_expect_tx(bar(B::v_full + st), L::kSub * kSubBytes);
+        for (int s = 0; s < L::kSub; ++s)
+          tma_load_3d(sbase + L::kV + (st * L::kSub + s) * kSubBytes, &tmV, 64 * s, h, key0, bar(B::v_full + st));
+        issued_v = g + 1;
+      }
+      // drain: every load issued above must land before the CTA may exit
+      for (int u = 0; u < kQT; ++u)
+        if (q_issued[u]) drain_wait(bar(B::q_full + u), 0);
+      for (int g = issued_k > kStages ? issued_k - kStages : 0; g < issued_k; ++g)
+        drain_wait(bar(B::k_full + g % kStages), (g / kStages) & 1);
+      for (int g = issued_v > kStages ? issued_v - kStages : 0; g < issued_v; ++g)
+        drain_wait(bar(B::v_full + g % kStages), (g / kStages) & 1);
+    }
+  };
+  auto mma_role = [&]() {
+    // ================================ MMA issuer =======================================
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(kBN, kUR, false, false);  // K Q^T: both K-major
+      constexpr uint32_t kIdescO = idesc_bf16(D, kUR, true, true);      // V^T P^T: both MN-major
+      // descriptor words of the operand bases (LBO: 16 bytes for K-major operands; the next
+      // 64-wide sub-tile for V^T, the next 64 rows for P^T, neither reached by N = 64 rows)
+      const uint32_t k_lo = sdesc_lo(sbase + L::kK, 16), q_lo = sdesc_lo(sbase + L::kQ, 16);
+      const uint32_t v_lo = sdesc_lo(sbase + L::kV, kSubBytes), pt_lo = sdesc_lo(sbase + L::kPT, kPTBytes);
+      // S^T(g) = K_g Q_u^T into buffer g % 2
+      auto issue_s = [&](int g) -> bool {
+        const int st = g % kStages, u = unit_of(g);
+        if (!mbar_wait(bar(B::k_full + st), (g / kStages) & 1, &s_abort, prm.status)) return false;
+        if (step_of(g) == 0 && !mbar_wait(bar(B::q_full + u), 0, &s_abort, prm.status)) return false;
+        tc_fence_after();
+        const uint32_t a0 = k_lo + ((st * L::kSub * kSubBytes) >> 4), b0 = q_lo + ((u * L::kSub * kQSub) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // 16 channels: sub-tile kk / 4, 32-byte chunk kk % 4 of each 128-byte row
+          mma_ss_words(tS(g & 1), a0 + (((kk >> 2) * kSubBytes + (kk & 3) * 32) >> 4),
+                       b0 + (((kk >> 2) * kQSub + (kk & 3) * 32) >> 4), kIdescS, kk > 0);
+        }
+        mma_commit(bar(B::s_full + st));               // S^T(g) complete; K stage g % 2 free
+        return true;
+      };
+      bool ok = true;
+      for (int g = 0; ok && g < nt && g < 2; ++g) ok = issue_s(g);
+      for (int g = 0; ok && g < nt; ++g) {
+        const int st = g % kStages, u = unit_of(g), j = step_of(g);
+        ok = mbar_wait(bar(B::p_full + st), (g >> 1) & 1, &s_abort, prm.status);
+        if (ok) ok = mbar_wait(bar(B::v_full + st), (g / kStages) & 1, &s_abort, prm.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a0 = v_lo + ((st * L::kSub * kSubBytes) >> 4), b0 = pt_lo + ((st * kPTBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // A = V^T [128 channels x 16 keys], MN-major: 16 keys = 2 swizzle atoms of 8 rows
+          // (SBO), channels 64-127 in the next sub-tile (LBO). B = P^T [64 rows x 16 keys],
+          // MN-major: one 64-row atom, 8 keys per SBO.
+          mma_ss_words(tO(u), a0 + ((kk * 16 * 128) >> 4), b0 + ((kk * 16 * 128) >> 4), kIdescO,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(B::pv_done + st));              // P V(g) complete; V stage g % 2 free
+        // S^T(g+2) reuses buffer g % 2: the softmax has read S^T(g), since P^T(g) is complete.
+        // tcgen05.mma operations of one thread execute in issue order, so S^T(g+2)'s
+        // completion also implies that P V(g) has finished reading P^T buffer g % 2.
+        if (g + 2 < nt) ok = issue_s(g + 2);
+      }
+      mma_commit(bar(B::drain));   // fires once every MMA issued above has completed
+    }
+  };
+  auto softmax_role = [&]() {
+    // ================================ softmax warps ====================================
+    const int w = warp >> 2;                       // column half of this warpgroup
+    const int r = (warp & 3) * 32 + lane;          // key of S^T, channel of O^T == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int c0 = kHalf * w;                      // first column (query row of the unit) of this half
+    const int bid = 1 + w;                         // this warpgroup's named barrier
+    float* red = reinterpret_cast<float*>(gbase + L::kRed) + w * 4 * kHalf;
+    float* nref = reinterpret_cast<float*>(gbase + L::kRef) + c0;
+    float* aux = reinterpret_cast<float*>(gbase + L::kAux) + c0;
+    const float sl2 = prm.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t zero2 = f2_pack(0.f, 0.f);
+    // a unit with rows but no kept key block: zero output, log-sum-exp -inf
+    for (int u = 0; u < kQT; ++u) {
+      if (s_ntiles[u] > 0 || s_nrows[u] == 0) continue;
+      const int64_t row0 = s_row0[u];
+      for (int i = tid; i < s_nrows[u] * (D / 8); i += kSoftmaxThreads)
+        *reinterpret_cast<uint4*>(p.o + ((row0 + i / (D / 8)) * p.H + h) * D + (i % (D / 8)) * 8) =
+            make_uint4(0u, 0u, 0u, 0u);
+      if (p.lse)
+        for (int i = tid; i < s_nrows[u]; i += kSoftmaxThreads) p.lse[(row0 + i) * p.H + h] = -INFINITY;
+    }
+    uint64_t lsum[kHalf / 2];                      // per-column partial sums over this thread's keys
+#pragma unroll
+    for (int i = 0; i < kHalf / 2; ++i) lsum[i] = zero2;
+    for (int g = 0; g < nt; ++g) {
+      const int u = unit_of(g), j = step_of(g), b = g & 1;
+      // every wait result is made warp-uniform: tcgen05.ld/st are .sync.aligned
+      const bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B::s_full + b), (g >> 1) & 1, &s_abort, prm.status));
+      const bool kvalid = static_cast<int64_t>(tile_kb(g)) * kBN + r < p.N;   // keys past N are masked
+      float sv[kHalf];
+      auto load_s = [&]() {
+        tmem_ld32(tS(b) + lane_off + c0, sv);
+        if (!kvalid) {
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c) sv[c] = -INFINITY;
+        }
+      };
+      // exponent arguments x = S * scale_log2 - reference, in place; returns their maximum
+      auto x_pass = [&]() -> float {
+        float xm0 = -INFINITY, xm1 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 4) {
+          const float4 nr = *reinterpret_cast<const float4*>(nref + c);
+          const uint64_t x01 = ffma2(f2_pack(sv[c], sv[c + 1]), sl2x2, f2_pack(nr.x, nr.y));
+          const uint64_t x23 = ffma2(f2_pack(sv[c + 2], sv[c + 3]), sl2x2, f2_pack(nr.z, nr.w));
+          f2_unpack(x01, sv[c], sv[c + 1]);
+          f2_unpack(x23, sv[c + 2], sv[c + 3]);
+          xm0 = fmax3f(xm0, sv[c], sv[c + 1]);
+          xm1 = fmax3f(xm1, sv[c + 2], sv[c + 3]);
+        }
+        return fmaxf(xm0, xm1);
+      };
+      // P = 2^x in place (fp32) and as bf16 pairs
+      uint32_t pk[kHalf / 2];
+      auto exp_pass = [&]() {
+#pragma unroll
+        for (int c = 0; c < kHalf; c += 2) {
+          sv[c] = fast_exp2(sv[c]);
+          sv[c + 1] = fast_exp2(sv[c + 1]);
+          pk[c >> 1] = pack_bf16x2(sv[c], sv[c + 1]);
+        }
+      };
+      // Fast path: keep the references. Softmax is exact for any reference (the final l uses
+      // the same one); while every argument is at most kXLimit, P and the sums stay finite.
+      // The exponentials run before the warpgroup's vote and are discarded if it fails.
+      bool slow = j == 0;
+      if (w_ok) {
+        tc_fence_after();
+        load_s();
+        if (!slow) {
+          slow = !(x_pass() <= kXLimit);
+          exp_pass();
+        }
+      }
+      if (wg_any(bid, !w_ok || slow)) {
+        if (wg_any(bid, !w_ok)) break;             // uniform over the warpgroup
+        // new references: this tile's column maxima over the 128 keys
+        if (j > 0) load_s();                       // S^T is intact: P^T(g) has not been released
+        {
+          float v[kHalf];
+#pragma unroll
+          for (int c = 0; c < kHalf; ++c) v[c] = sv[c];
+          warp_fold32<true>(v, lane);
+          red[(warp & 3) * kHalf + lane] = v[0];
+        }
+        wg_sync(bid);
+        if (r < kHalf) {
+          const float mx = fmaxf(fmaxf(red[r], red[kHalf + r]), fmaxf(red[2 * kHalf + r], red[3 * kHalf + r])) * sl2;
+          const float old = j == 0 ? -INFINITY : -nref[r];
+          float mnew = fmaxf(old, mx);
+          if (mnew == -INFINITY) mnew = 0.f;       // a column without a finite score keeps reference 0
+          aux[r] = j == 0 ? 1.f : fast_exp2(old - mnew);
+          nref[r] = -mnew;
+        }
+        wg_sync(bid);
+        load_s();
+        if (j > 0) {
+          // O^T must hold every P V of this unit up to tile j-1 before it moves to the new
+          // references (P V(g-1) was issued after S^T(g), so it may still run; P V(g-3) has
+          // completed and P V(g+1) cannot start, so the parity names P V(g-1))
+          const bool pv_ok = __all_sync(
+              0xffffffffu, mbar_wait(bar(B::pv_done + ((g - 1) & 1)), ((g - 1) >> 1) & 1, &s_abort, prm.status));
+          if (wg_any(bid, !pv_ok)) break;
+          tc_fence_after();
+          float o[kHalf];
+          tmem_ld32(tO(u) + lane_off + c0, o);
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 4) {
+            const float4 al = *reinterpret_cast<const float4*>(aux + c);
+            o[c] *= al.x;
+            o[c + 1] *= al.y;
+            o[c + 2] *= al.z;
+            o[c + 3] *= al.w;
+            lsum[c >> 1] = ffma2(lsum[c >> 1], f2_pack(al.x, al.y), zero2);
+            lsum[(c >> 1) + 1] = ffma2(lsum[(c >> 1) + 1], f2_pack(al.z, al.w), zero2);
+          }
+          tmem_st32(tO(u) + lane_off + c0, o);
+        }
+        x_pass();
+        exp_pass();
+      }
+      // per-column partial sums (this thread's one key of the tile)
+#pragma unroll
+      for (int c = 0; c < kHalf; c += 2) lsum[c >> 1] = fadd2(lsum[c >> 1], f2_pack(sv[c], sv[c + 1]));
+      // this half of key r's row of P^T: 16-byte chunks 4w..4w+3, 128-byte swizzle (chunk q at q ^ (r % 8))
+      uint8_t* ptb = gbase + L::kPT + b * kPTBytes;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(ptb + r * 128 + (((4 * w + q) ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      fence_proxy_async_smem();                    // the tensor core reads P^T through the async proxy
+      tc_fence_before();
+      mbar_arrive(bar(B::p_full + b));
+      if (j == s_ntiles[u] - 1) {
+        // ---- unit u complete: column sums, O^T / l, stores ------------------------------
+        // P V(g), the unit's last (P V(g-2) has completed and P V(g+2) cannot start)
+        const bool d_ok =
+            __all_sync(0xffffffffu, mbar_wait(bar(B::pv_done + b), (g >> 1) & 1, &s_abort, prm.status));
+        if (wg_any(bid, !d_ok)) break;
+        tc_fence_after();
+        {
+          float v[kHalf];
+#pragma unroll
+          for (int i = 0; i < kHalf / 2; ++i) f2_unpack(lsum[i], v[2 * i], v[2 * i + 1]);
+          warp_fold32<false>(v, lane);
+          red[(warp & 3) * kHalf + lane] = v[0];
+        }
+        wg_sync(bid);
+        const int nrows = s_nrows[u];
+        const int64_t row0 = s_row0[u];
+        uint8_t* qbuf = gbase + L::kQ + u * L::kSub * kQSub;
+        if (r < kHalf) {
+          const float l = (red[r] + red[kHalf + r]) + (red[2 * kHalf + r] + red[3 * kHalf + r]);
+          aux[r] = l > 0.f ? 1.f / l : 0.f;
+          if (c0 + r < nrows && p.lse)
+            p.lse[(row0 + c0 + r) * p.H + h] = l > 0.f ? (__log2f(l) - nref[r]) * kLn2 : -INFINITY;
+        }
+        wg_sync(bid);
+        {
+          // O^T / l, transposed through unit u's Q buffer (its last reader, S^T(g), has
+          // completed): row c of the unit at c * 256 bytes; each warpgroup its own 32 rows
+          float o[kHalf];
+          tmem_ld32(tO(u) + lane_off + c0, o);
+          uint16_t* ot = reinterpret_cast<uint16_t*>(qbuf);
+#pragma unroll
+          for (int c = 0; c < kHalf; c += 4) {
+            const float4 inv = *reinterpret_cast<const float4*>(aux + c);
+            const uint32_t w01 = pack_bf16x2(o[c] * inv.x, o[c + 1] * inv.y);
+            const uint32_t w23 = pack_bf16x2(o[c + 2] * inv.z, o[c + 3] * inv.w);
+            ot[(c0 + c) * D + r] = static_cast<uint16_t>(w01 & 0xffffu);
+            ot[(c0 + c + 1) * D + r] = static_cast<uint16_t>(w01 >> 16);
+            ot[(c0 + c + 2) * D + r] = static_cast<uint16_t>(w23 & 0xffffu);
+            ot[(c0 + c + 3) * D + r] = static_cast<uint16_t>(w23 >> 16);
+          }
+        }
+        wg_sync(bid);
+        for (int i = r; i < kHalf * (D / 8); i += kBM) {
+          const int c = c0 + i / (D / 8), q = i % (D / 8);
+          if (c < nrows)
+            *reinterpret_cast<uint4*>(p.o + ((row0 + c) * p.H + h) * D + q * 8) =
+                *reinterpret_cast<const uint4*>(qbuf + c * (D * 2) + q * 16);
+        }
+#pragma unroll
+        for (int i = 0; i < kHalf / 2; ++i) lsum[i] = zero2;
+      }
+    }
+  };
+  // the common tail; each warpgroup runs its own copy (non-aligned barrier)
+  auto tail = [&]() {
+    if (warp == kMmaWarp && lane == 0) drain_wait(bar(B::drain), 0);   // no MMA may still write TMEM
+    tc_fence_before();
+    cta_sync<true>();
+    tc_fence_after();
+    if (warp == kMmaWarp) {
+      __syncwarp();
+      tmem_dealloc<kTmemColsT>(tmem);
+    }
+  };
+  // registers from the producer warpgroup to the softmax warpgroups (as in attn_tc_kernel)
+  if (warp >= kTmaWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kTmaWarp) tma_role();
+    else if (warp == kMmaWarp) mma_role();
+    tail();
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    softmax_role();
+    tail();
+  }
+}
+
 // ---- host ------------------------------------------------------------------------------------
-// [rows, H, d] bf16, token-major -> 3-D map (d, H, rows), box (64, 1, 128), 128-byte swizzle.
-int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, int H, int d) {
+// [rows, H, d] bf16, token-major -> 3-D map (d, H, rows), box (64, 1, box_rows), 128-byte swizzle.
+int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, int64_t rows, int H, int d, int box_rows = 128) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -929,7 +1449,8 @@ int smem_attribute(int bytes) {
 
 // Dense: ceil(cap/256) x H x nsplit CTAs of two 128-row tiles of compacted rows.
 // Masked (block mode): ceil(nb/2) x H CTAs, CTA x holding the active rows of
-// query blocks 2x and 2x+1, each tile with its own key list.
+// query blocks 2x and 2x+1, each tile with its own key list; with d = 128 the
+// transposed kernel, ceil(nb/2) x H x 2 CTAs (z: rows 0-63 or 64-127 of each run).
 template <int D>
 int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = nullptr, float* lse_part = nullptr,
            int64_t tile0 = 0, int64_t ntiles = -1) {
@@ -944,7 +1465,15 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1, static_cast<int>(tile0)};
-  if (a.bm) {
+  if (a.bm && D == 128) {
+    // transposed products: units of at most 64 rows of one query block, z = which 64 rows
+    CUtensorMap mq64;
+    if (int e = make_map(enc, &mq64, a.q, a.cap, a.H, a.d, blkt::kUR)) return e;
+    constexpr int kSmem = blkt::LayoutT::kAlloc;
+    if (int e = smem_attribute<attn_blkt_kernel>(kSmem)) return e;
+    dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), kBM / blkt::kUR);
+    attn_blkt_kernel<<<grid, kThreads, kSmem, st>>>(mq64, mk, mv, prm);
+  } else if (a.bm) {
     constexpr int kSmem = Layout<D, kQT>::kAlloc;
     if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
     dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
