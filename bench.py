@@ -690,14 +690,19 @@ def keep_sweep(dev, attn, reps=5):
 def executed_flops(idx: np.ndarray, N: int, H: int, d: int, nb_mask=None) -> float:
     """FLOPs the attention kernel executes, padding rows and whole 128-key
     tiles included. Dense: ceil(A/256) CTAs of two 128-row tiles, every key
-    tile. Masked: one 128-row tile per original query block holding an active
-    row, the key tiles that block keeps."""
+    tile. Masked, d = 128: one 64-row unit per 64 active rows (or fewer) of an
+    original query block (the transposed products' N), the key tiles that block
+    keeps. Masked, d = 64: one 128-row tile per query block holding an active
+    row."""
     nkt = -(-N // 128)
     A = len(idx)
     if nb_mask is None:
         return 4.0 * d * H * 256 * 128 * (-(-A // 256)) * nkt
-    blocks = np.unique(np.asarray(idx) // 128)
-    return 4.0 * d * H * 128 * 128 * float(nb_mask[blocks].astype(np.int64).sum())
+    blocks, rows = np.unique(np.asarray(idx) // 128, return_counts=True)
+    kept = nb_mask[blocks].astype(np.int64).sum(axis=1)
+    if d == 128:
+        return 4.0 * d * H * 64 * 128 * float(np.sum(-(-rows // 64) * kept))
+    return 4.0 * d * H * 128 * 128 * float(kept.sum())
 
 
 def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
@@ -856,7 +861,9 @@ def kernel_case(name, dev):
     like the full one, its full waves unsplit and its remaining query tiles
     split in a second launch (capture both launches of the second call);
     heads are independent units of the grid, so a full call moves about 3x
-    these bytes. overlap_hsa is not a capture case:
+    these bytes. attn_block_h2: the block-sparse config's attention on 2 of
+    its 24 heads (one launch of the transposed block kernel). overlap_hsa is
+    not a capture case:
     it times the HSA step's host transfers alone and beside the attention."""
     from token_pruned_sparse_b200 import tps
     g = torch.Generator(device=dev)
@@ -893,6 +900,19 @@ def kernel_case(name, dev):
             tps.lipar_front(cur, tps.FRONT_TOPK, x_ref=prev, k=v.N // 3, ws=ws)
     elif name == "overlap_hsa":
         return overlap_probe(dev)
+    elif name == "attn_block_h2":
+        # the block-sparse config (118800 tokens, 40% active rows, 139 of 929 key blocks kept per
+        # query block) on 2 of its 24 heads: 465 x 2 x 2 CTAs of the transposed kernel
+        cfg = synth.CONFIGS["block"]
+        N, H, d = cfg.video.N, 2, cfg.d
+        A = synth.keep_count(N, cfg.keep[0])
+        idx = torch.sort(torch.randperm(N, device=dev, generator=g)[:A])[0].to(torch.int32)
+        cnt = torch.tensor([A], dtype=torch.int32, device=dev)
+        q, k, v = rnd(A, H, d), rnd(N, H, d), rnd(N, H, d)
+        bm = synth.block_mask_band_random(cfg.video, 128, cfg.extra["kept_per_row"], cfg.video.seed).to(dev)
+        o = torch.empty_like(q)
+        for _ in range(2):
+            tps.pruned_attn(q, k, v, idx, cnt, 1 / math.sqrt(d), blockmask=bm, o_act=o)
     elif name in ("attn_mid", "attn_hsa_h8"):
         if name == "attn_mid":
             cfg = synth.CONFIGS["mid"]
@@ -1241,7 +1261,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-config kernel sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch the step's stages eagerly (no CUDA graphs)")
-    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h8", "front_hsa",
+    ap.add_argument("--kernel-case", choices=["timeripple", "renoise", "attn_mid", "attn_hsa_h8", "attn_block_h2", "front_hsa",
                                               "overlap_hsa"],
                     default=None,
                     help="run one kernel's small capture case (warm-up + one launch) and exit")

@@ -907,7 +907,7 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 // units 0 and 1, one after the other: one stream of key tiles g = 0, 1, ... (unit 0's list, then
 // unit 1's) through two-stage K and V rings. S^T and P^T are double-buffered (TMEM and shared
 // memory), so the MMAs of tiles g + 2 and g overlap the softmax of tile g + 1.
-// The eight softmax warps split a tile's 64 columns: warpgroup w takes columns [32w, 32w + 32);
+// Four softmax warpgroups split a tile's 64 columns: warpgroup w takes columns [16w, 16w + 16);
 // thread r of it owns key r of S^T (TMEM lane r) and channel r of O^T. The reference maximum is
 // one per column (query row), shared by the 128 key threads of its warpgroup: after a unit's
 // first key tile it changes only when an exponent argument exceeds kXLimit somewhere in the
@@ -920,7 +920,14 @@ attn_blk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 // O^T holds tile g.
 namespace blkt {
 constexpr int kUR = 64;                 // query rows per unit (MMA N)
-constexpr int kHalf = kUR / 2;          // columns per softmax warpgroup
+constexpr int kWG = 4;                  // softmax warpgroups
+constexpr int kCols = kUR / kWG;        // columns per softmax warpgroup
+constexpr int kSmThreadsT = kWG * 128;  // softmax threads
+// + one producer warpgroup (TMA warp, MMA warp, two idle warps). 20 warps leave 96 registers a
+// thread, enough for a softmax thread's 16 columns, so the kernel needs no register split.
+constexpr int kThreadsT = kSmThreadsT + 128;
+constexpr int kTmaWarpT = kSmThreadsT / 32;
+constexpr int kMmaWarpT = kTmaWarpT + 1;
 constexpr int kQSub = kUR * 128;        // one [64 rows x 64 bf16] swizzled Q sub-tile
 constexpr int kPTBytes = 128 * 128;     // P^T of one tile: 128 keys x 64 rows bf16 (one 128-byte row per key)
 constexpr float kXLimit = 64.f;         // largest exponent argument (log2) kept without a new reference
@@ -932,8 +939,8 @@ struct LayoutT {
   static constexpr int kK = kQ + kQT * kSub * kQSub;            // [stage][sub] x kSubBytes
   static constexpr int kV = kK + kStages * kSub * kSubBytes;
   static constexpr int kPT = kV + kStages * kSub * kSubBytes;   // [buffer] x kPTBytes
-  static constexpr int kRed = kPT + 2 * kPTBytes;               // float [warpgroup][warp][kHalf]: column folds
-  static constexpr int kRef = kRed + 2 * 4 * kHalf * 4;         // float [kUR]: minus the reference (log2)
+  static constexpr int kRed = kPT + 2 * kPTBytes;               // float [warpgroup][warp][kCols]: column folds
+  static constexpr int kRef = kRed + kWG * 4 * kCols * 4;       // float [kUR]: minus the reference (log2)
   static constexpr int kAux = kRef + kUR * 4;                   // float [kUR]: rescale factors, then 1/l
   static constexpr int kList = kAux + kUR * 4;                  // uint16 [unit][kListMax]: kept key blocks
   static constexpr int kListMax = 4096;
@@ -951,7 +958,7 @@ struct BarsT {  // mbarrier indices (8 bytes each)
   static constexpr int v_full = k_full + kStages;      // + stage
   static constexpr int s_full = v_full + kStages;      // + g % 2: S^T(g) complete, K stage g % 2 free
   static constexpr int pv_done = s_full + 2;           // + g % 2: P V(g) complete, V stage g % 2 free
-  static constexpr int p_full = pv_done + 2;           // + g % 2: P^T(g) written (256 arrivals)
+  static constexpr int p_full = pv_done + 2;           // + g % 2: P^T(g) written (every softmax thread)
   static constexpr int drain = p_full + 2;             // last commit of the MMA thread
   static constexpr int count = drain + 1;
 };
@@ -987,26 +994,31 @@ __device__ __forceinline__ void mma_ss_words(uint32_t d_tmem, uint32_t a_lo, uin
       ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kDescHi)
       : "memory");
 }
-// Folds 32 per-thread column values across the warp's 32 lanes by recursive halving (max or
-// sum); afterwards lane l holds the warp's result for column l in v[0].
-template <bool kMax>
-__device__ __forceinline__ void warp_fold32(float (&v)[kHalf], int lane) {
+// Folds kN per-thread column values across the warp's 32 lanes by recursive halving (max or
+// sum); afterwards lane l holds the warp's result for column l / (32 / kN) in v[0].
+template <int kN, bool kMax>
+__device__ __forceinline__ void warp_fold(float (&v)[kN], int lane) {
 #pragma unroll
   for (int s = 0; s < 5; ++s) {
-    const int o = 16 >> s, n = kHalf >> s;
-    const bool up = (lane & o) != 0;
+    const int o = 16 >> s, n = kN >> s;
+    if (n >= 2) {
+      const bool up = (lane & o) != 0;
 #pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float send = up ? v[i] : v[i + n / 2];
-      const float keep = up ? v[i + n / 2] : v[i];
-      const float got = __shfl_xor_sync(0xffffffffu, send, o);
-      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+      for (int i = 0; i < n / 2; ++i) {
+        const float send = up ? v[i] : v[i + n / 2];
+        const float keep = up ? v[i + n / 2] : v[i];
+        const float got = __shfl_xor_sync(0xffffffffu, send, o);
+        v[i] = kMax ? fmaxf(keep, got) : keep + got;
+      }
+    } else {   // lanes l and l ^ o hold the same column
+      const float got = __shfl_xor_sync(0xffffffffu, v[0], o);
+      v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
     }
   }
 }
 }  // namespace blkt
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(blkt::kThreadsT, 1)
 attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, TcParams prm) {
   using namespace blkt;
@@ -1019,7 +1031,7 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __shared__ int s_nrows[kQT];
   __shared__ int s_row0[kQT];
   __shared__ volatile int s_abort;
-  __shared__ unsigned int s_wcnt[kQT][kThreads / 32];
+  __shared__ unsigned int s_wcnt[kQT][kThreadsT / 32];
 
   const AttnArgs& p = prm.a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1064,13 +1076,13 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(bar(B::v_full + s), 1);
       mbar_init(bar(B::s_full + s), 1);
       mbar_init(bar(B::pv_done + s), 1);
-      mbar_init(bar(B::p_full + s), kSoftmaxThreads);
+      mbar_init(bar(B::p_full + s), kSmThreadsT);
     }
     mbar_init(bar(B::drain), 1);
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) tmem_alloc<kTmemColsT>(smem_u32(&s_tmem));
-  if (warp == kTmaWarp && lane == 0) {
+  if (warp == kMmaWarpT) tmem_alloc<kTmemColsT>(smem_u32(&s_tmem));
+  if (warp == kTmaWarpT && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -1081,7 +1093,7 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint8_t* mrow[kQT];
     for (int u = 0; u < kQT; ++u)
       mrow[u] = p.bm + (2 * static_cast<int64_t>(blockIdx.x) + u) * p.nb;
-    for (int kb0 = 0; kb0 < p.nb; kb0 += kThreads) {
+    for (int kb0 = 0; kb0 < p.nb; kb0 += kThreadsT) {
       const int kb = kb0 + tid;
       unsigned int m[kQT];
       for (int u = 0; u < kQT; ++u) {
@@ -1092,7 +1104,7 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       __syncthreads();
       for (int u = 0; u < kQT; ++u) {
         int off = base[u], tot = 0;
-        for (int i = 0; i < kThreads / 32; ++i) {
+        for (int i = 0; i < kThreadsT / 32; ++i) {
           off += i < warp ? s_wcnt[u][i] : 0;
           tot += s_wcnt[u][i];
         }
@@ -1206,12 +1218,12 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   };
   auto softmax_role = [&]() {
     // ================================ softmax warps ====================================
-    const int w = warp >> 2;                       // column half of this warpgroup
+    const int w = warp >> 2;                       // column group of this warpgroup
     const int r = (warp & 3) * 32 + lane;          // key of S^T, channel of O^T == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int c0 = kHalf * w;                      // first column (query row of the unit) of this half
+    const int c0 = kCols * w;                      // first column (query row of the unit) of this group
     const int bid = 1 + w;                         // this warpgroup's named barrier
-    float* red = reinterpret_cast<float*>(gbase + L::kRed) + w * 4 * kHalf;
+    float* red = reinterpret_cast<float*>(gbase + L::kRed) + w * 4 * kCols;
     float* nref = reinterpret_cast<float*>(gbase + L::kRef) + c0;
     float* aux = reinterpret_cast<float*>(gbase + L::kAux) + c0;
     const float sl2 = prm.scale_log2;
@@ -1221,33 +1233,33 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int u = 0; u < kQT; ++u) {
       if (s_ntiles[u] > 0 || s_nrows[u] == 0) continue;
       const int64_t row0 = s_row0[u];
-      for (int i = tid; i < s_nrows[u] * (D / 8); i += kSoftmaxThreads)
+      for (int i = tid; i < s_nrows[u] * (D / 8); i += kSmThreadsT)
         *reinterpret_cast<uint4*>(p.o + ((row0 + i / (D / 8)) * p.H + h) * D + (i % (D / 8)) * 8) =
             make_uint4(0u, 0u, 0u, 0u);
       if (p.lse)
-        for (int i = tid; i < s_nrows[u]; i += kSoftmaxThreads) p.lse[(row0 + i) * p.H + h] = -INFINITY;
+        for (int i = tid; i < s_nrows[u]; i += kSmThreadsT) p.lse[(row0 + i) * p.H + h] = -INFINITY;
     }
-    uint64_t lsum[kHalf / 2];                      // per-column partial sums over this thread's keys
+    uint64_t lsum[kCols / 2];                      // per-column partial sums over this thread's keys
 #pragma unroll
-    for (int i = 0; i < kHalf / 2; ++i) lsum[i] = zero2;
+    for (int i = 0; i < kCols / 2; ++i) lsum[i] = zero2;
     for (int g = 0; g < nt; ++g) {
       const int u = unit_of(g), j = step_of(g), b = g & 1;
       // every wait result is made warp-uniform: tcgen05.ld/st are .sync.aligned
       const bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar(B::s_full + b), (g >> 1) & 1, &s_abort, prm.status));
       const bool kvalid = static_cast<int64_t>(tile_kb(g)) * kBN + r < p.N;   // keys past N are masked
-      float sv[kHalf];
+      float sv[kCols];
       auto load_s = [&]() {
-        tmem_ld32(tS(b) + lane_off + c0, sv);
+        tmem_ld16(tS(b) + lane_off + c0, sv);
         if (!kvalid) {
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) sv[c] = -INFINITY;
+          for (int c = 0; c < kCols; ++c) sv[c] = -INFINITY;
         }
       };
       // exponent arguments x = S * scale_log2 - reference, in place; returns their maximum
       auto x_pass = [&]() -> float {
         float xm0 = -INFINITY, xm1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kHalf; c += 4) {
+        for (int c = 0; c < kCols; c += 4) {
           const float4 nr = *reinterpret_cast<const float4*>(nref + c);
           const uint64_t x01 = ffma2(f2_pack(sv[c], sv[c + 1]), sl2x2, f2_pack(nr.x, nr.y));
           const uint64_t x23 = ffma2(f2_pack(sv[c + 2], sv[c + 3]), sl2x2, f2_pack(nr.z, nr.w));
@@ -1259,10 +1271,10 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         return fmaxf(xm0, xm1);
       };
       // P = 2^x in place (fp32) and as bf16 pairs
-      uint32_t pk[kHalf / 2];
+      uint32_t pk[kCols / 2];
       auto exp_pass = [&]() {
 #pragma unroll
-        for (int c = 0; c < kHalf; c += 2) {
+        for (int c = 0; c < kCols; c += 2) {
           sv[c] = fast_exp2(sv[c]);
           sv[c + 1] = fast_exp2(sv[c + 1]);
           pk[c >> 1] = pack_bf16x2(sv[c], sv[c + 1]);
@@ -1285,15 +1297,15 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // new references: this tile's column maxima over the 128 keys
         if (j > 0) load_s();                       // S^T is intact: P^T(g) has not been released
         {
-          float v[kHalf];
+          float v[kCols];
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) v[c] = sv[c];
-          warp_fold32<true>(v, lane);
-          red[(warp & 3) * kHalf + lane] = v[0];
+          for (int c = 0; c < kCols; ++c) v[c] = sv[c];
+          warp_fold<kCols, true>(v, lane);
+          if ((lane & (32 / kCols - 1)) == 0) red[(warp & 3) * kCols + lane / (32 / kCols)] = v[0];
         }
         wg_sync(bid);
-        if (r < kHalf) {
-          const float mx = fmaxf(fmaxf(red[r], red[kHalf + r]), fmaxf(red[2 * kHalf + r], red[3 * kHalf + r])) * sl2;
+        if (r < kCols) {
+          const float mx = fmaxf(fmaxf(red[r], red[kCols + r]), fmaxf(red[2 * kCols + r], red[3 * kCols + r])) * sl2;
           const float old = j == 0 ? -INFINITY : -nref[r];
           float mnew = fmaxf(old, mx);
           if (mnew == -INFINITY) mnew = 0.f;       // a column without a finite score keeps reference 0
@@ -1310,10 +1322,10 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               0xffffffffu, mbar_wait(bar(B::pv_done + ((g - 1) & 1)), ((g - 1) >> 1) & 1, &s_abort, prm.status));
           if (wg_any(bid, !pv_ok)) break;
           tc_fence_after();
-          float o[kHalf];
-          tmem_ld32(tO(u) + lane_off + c0, o);
+          float o[kCols];
+          tmem_ld16(tO(u) + lane_off + c0, o);
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 4) {
+          for (int c = 0; c < kCols; c += 4) {
             const float4 al = *reinterpret_cast<const float4*>(aux + c);
             o[c] *= al.x;
             o[c + 1] *= al.y;
@@ -1322,19 +1334,20 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             lsum[c >> 1] = ffma2(lsum[c >> 1], f2_pack(al.x, al.y), zero2);
             lsum[(c >> 1) + 1] = ffma2(lsum[(c >> 1) + 1], f2_pack(al.z, al.w), zero2);
           }
-          tmem_st32(tO(u) + lane_off + c0, o);
+          tmem_st16(tO(u) + lane_off + c0, o);
         }
         x_pass();
         exp_pass();
       }
       // per-column partial sums (this thread's one key of the tile)
 #pragma unroll
-      for (int c = 0; c < kHalf; c += 2) lsum[c >> 1] = fadd2(lsum[c >> 1], f2_pack(sv[c], sv[c + 1]));
-      // this half of key r's row of P^T: 16-byte chunks 4w..4w+3, 128-byte swizzle (chunk q at q ^ (r % 8))
+      for (int c = 0; c < kCols; c += 2) lsum[c >> 1] = fadd2(lsum[c >> 1], f2_pack(sv[c], sv[c + 1]));
+      // this group's part of key r's row of P^T: 16-byte chunks 2w and 2w + 1, 128-byte swizzle
+      // (chunk q at q ^ (r % 8))
       uint8_t* ptb = gbase + L::kPT + b * kPTBytes;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(ptb + r * 128 + (((4 * w + q) ^ (r & 7)) << 4)) =
+      for (int q = 0; q < kCols / 8; ++q)
+        *reinterpret_cast<uint4*>(ptb + r * 128 + ((((kCols / 8) * w + q) ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       fence_proxy_async_smem();                    // the tensor core reads P^T through the async proxy
       tc_fence_before();
@@ -1347,18 +1360,18 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (wg_any(bid, !d_ok)) break;
         tc_fence_after();
         {
-          float v[kHalf];
+          float v[kCols];
 #pragma unroll
-          for (int i = 0; i < kHalf / 2; ++i) f2_unpack(lsum[i], v[2 * i], v[2 * i + 1]);
-          warp_fold32<false>(v, lane);
-          red[(warp & 3) * kHalf + lane] = v[0];
+          for (int i = 0; i < kCols / 2; ++i) f2_unpack(lsum[i], v[2 * i], v[2 * i + 1]);
+          warp_fold<kCols, false>(v, lane);
+          if ((lane & (32 / kCols - 1)) == 0) red[(warp & 3) * kCols + lane / (32 / kCols)] = v[0];
         }
         wg_sync(bid);
         const int nrows = s_nrows[u];
         const int64_t row0 = s_row0[u];
         uint8_t* qbuf = gbase + L::kQ + u * L::kSub * kQSub;
-        if (r < kHalf) {
-          const float l = (red[r] + red[kHalf + r]) + (red[2 * kHalf + r] + red[3 * kHalf + r]);
+        if (r < kCols) {
+          const float l = (red[r] + red[kCols + r]) + (red[2 * kCols + r] + red[3 * kCols + r]);
           aux[r] = l > 0.f ? 1.f / l : 0.f;
           if (c0 + r < nrows && p.lse)
             p.lse[(row0 + c0 + r) * p.H + h] = l > 0.f ? (__log2f(l) - nref[r]) * kLn2 : -INFINITY;
@@ -1366,12 +1379,12 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         wg_sync(bid);
         {
           // O^T / l, transposed through unit u's Q buffer (its last reader, S^T(g), has
-          // completed): row c of the unit at c * 256 bytes; each warpgroup its own 32 rows
-          float o[kHalf];
-          tmem_ld32(tO(u) + lane_off + c0, o);
+          // completed): row c of the unit at c * 256 bytes; each warpgroup its own 16 rows
+          float o[kCols];
+          tmem_ld16(tO(u) + lane_off + c0, o);
           uint16_t* ot = reinterpret_cast<uint16_t*>(qbuf);
 #pragma unroll
-          for (int c = 0; c < kHalf; c += 4) {
+          for (int c = 0; c < kCols; c += 4) {
             const float4 inv = *reinterpret_cast<const float4*>(aux + c);
             const uint32_t w01 = pack_bf16x2(o[c] * inv.x, o[c + 1] * inv.y);
             const uint32_t w23 = pack_bf16x2(o[c + 2] * inv.z, o[c + 3] * inv.w);
@@ -1382,38 +1395,29 @@ attn_blkt_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
         }
         wg_sync(bid);
-        for (int i = r; i < kHalf * (D / 8); i += kBM) {
+        for (int i = r; i < kCols * (D / 8); i += kBM) {
           const int c = c0 + i / (D / 8), q = i % (D / 8);
           if (c < nrows)
             *reinterpret_cast<uint4*>(p.o + ((row0 + c) * p.H + h) * D + q * 8) =
                 *reinterpret_cast<const uint4*>(qbuf + c * (D * 2) + q * 16);
         }
 #pragma unroll
-        for (int i = 0; i < kHalf / 2; ++i) lsum[i] = zero2;
+        for (int i = 0; i < kCols / 2; ++i) lsum[i] = zero2;
       }
     }
   };
   // the common tail; each warpgroup runs its own copy (non-aligned barrier)
-  auto tail = [&]() {
-    if (warp == kMmaWarp && lane == 0) drain_wait(bar(B::drain), 0);   // no MMA may still write TMEM
-    tc_fence_before();
-    cta_sync<true>();
-    tc_fence_after();
-    if (warp == kMmaWarp) {
-      __syncwarp();
-      tmem_dealloc<kTmemColsT>(tmem);
-    }
-  };
-  // registers from the producer warpgroup to the softmax warpgroups (as in attn_tc_kernel)
-  if (warp >= kTmaWarp) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
-    if (warp == kTmaWarp) tma_role();
-    else if (warp == kMmaWarp) mma_role();
-    tail();
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-    softmax_role();
-    tail();
+  if (warp == kTmaWarpT) tma_role();
+  else if (warp == kMmaWarpT) mma_role();
+  else if (warp < kTmaWarpT) softmax_role();
+  // ---- teardown ------------------------------------------------------------------------
+  if (warp == kMmaWarpT && lane == 0) drain_wait(bar(B::drain), 0);   // no MMA may still write TMEM
+  tc_fence_before();
+  cta_sync<true>();
+  tc_fence_after();
+  if (warp == kMmaWarpT) {
+    __syncwarp();
+    tmem_dealloc<kTmemColsT>(tmem);
   }
 }
 
@@ -1472,7 +1476,7 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
     constexpr int kSmem = blkt::LayoutT::kAlloc;
     if (int e = smem_attribute<attn_blkt_kernel>(kSmem)) return e;
     dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), kBM / blkt::kUR);
-    attn_blkt_kernel<<<grid, kThreads, kSmem, st>>>(mq64, mk, mv, prm);
+    attn_blkt_kernel<<<grid, blkt::kThreadsT, kSmem, st>>>(mq64, mk, mv, prm);
   } else if (a.bm) {
     constexpr int kSmem = Layout<D, kQT>::kAlloc;
     if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
