@@ -10,11 +10,13 @@
 //
 // Dense mode: one CTA = 256 compacted active queries of one head, as two
 // 128-row tiles (t = 0, 1) that share every K/V tile. Block mode (a mask is
-// given): tile t of CTA x holds the active rows of original query block
+// given), d = 64: tile t of CTA x holds the active rows of original query block
 // 2x + t (at most 128; the rest of the tile is padding) and streams only the
 // key tiles that block keeps, so every loaded key tile is work for every row
 // of its tile; the two tiles' loads interleave in one K ring and one V ring.
-// In both modes the two tiles take turns on the tensor cores:
+// Block mode, d = 128: attn_blkt_kernel below, with the products transposed
+// (keys as the MMA's M, at most 64 active rows of one query block as its N).
+// In the dense and the d = 64 block kernel the two tiles take turns on the tensor cores:
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r of
 //              its tile (= TMEM lane r). Loads S from TMEM, online softmax in
 //              the log2 domain, writes P (bf16) back over the first half of
