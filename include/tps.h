@@ -291,7 +291,12 @@ TPS_API int kv_rerotate(const tps_bf16* k_cache, const int32_t* idx, const int32
  * distributed shared memory (no workspace): either the whole grid, or only
  * the query tiles left after the grid's full waves, in a second launch on the
  * same stream (tps_attn_plan reports which). Results agree with the unsplit
- * kernel within the attention tolerance. */
+ * kernel within the attention tolerance.
+ * With a mask, the active rows of each original query block (its run of the
+ * ascending idx) are computed together against only the key blocks that query
+ * block keeps: for d = 128 in units of at most 64 rows with the products
+ * transposed (the 128 keys of a key tile as the MMA's M, the unit's rows as
+ * N), for d = 64 in one 128-row tile per query block. */
 TPS_API int pruned_attn(const tps_bf16* q_act, const tps_bf16* k, const tps_bf16* v,
                 const int32_t* idx, const int32_t* count, int64_t cap, int64_t N, int H, int d,
                 float scale, const uint8_t* blockmask, int block, tps_bf16* o_act, float* lse,

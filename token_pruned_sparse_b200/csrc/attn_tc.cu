@@ -1471,19 +1471,21 @@ int launch(const AttnArgs& a, cudaStream_t st, int nsplit = 1, float* o_part = n
   if (int e = make_map(enc, &mk, a.k, a.N, a.H, a.d)) return e;
   if (int e = make_map(enc, &mv, a.v, a.N, a.H, a.d)) return e;
   TcParams prm{a, a.scale * kLog2e, status, nsplit, o_part, lse_part, 1, static_cast<int>(tile0)};
-  if (a.bm && D == 128) {
-    // transposed products: units of at most 64 rows of one query block, z = which 64 rows
-    CUtensorMap mq64;
-    if (int e = make_map(enc, &mq64, a.q, a.cap, a.H, a.d, blkt::kUR)) return e;
-    constexpr int kSmem = blkt::LayoutT::kAlloc;
-    if (int e = smem_attribute<attn_blkt_kernel>(kSmem)) return e;
-    dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), kBM / blkt::kUR);
-    attn_blkt_kernel<<<grid, blkt::kThreadsT, kSmem, st>>>(mq64, mk, mv, prm);
-  } else if (a.bm) {
-    constexpr int kSmem = Layout<D, kQT>::kAlloc;
-    if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
-    dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
-    attn_blk_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+  if (a.bm) {
+    if constexpr (D == 128) {
+      // transposed products: units of at most 64 rows of one query block, z = which 64 rows
+      CUtensorMap mq64;
+      if (int e = make_map(enc, &mq64, a.q, a.cap, a.H, a.d, blkt::kUR)) return e;
+      constexpr int kSmem = blkt::LayoutT::kAlloc;
+      if (int e = smem_attribute<attn_blkt_kernel>(kSmem)) return e;
+      dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), kBM / blkt::kUR);
+      attn_blkt_kernel<<<grid, blkt::kThreadsT, kSmem, st>>>(mq64, mk, mv, prm);
+    } else {
+      constexpr int kSmem = Layout<D, kQT>::kAlloc;
+      if (int e = smem_attribute<attn_blk_kernel<D>>(kSmem)) return e;
+      dim3 grid(static_cast<unsigned int>((a.nb + kQT - 1) / kQT), static_cast<unsigned int>(a.H), 1u);
+      attn_blk_kernel<D><<<grid, kThreads, kSmem, st>>>(mq, mk, mv, prm);
+    }
   } else {
     constexpr int kSmem = Layout<D, 1>::kAlloc;
     if (int e = smem_attribute<attn_tc_kernel<D, false>>(kSmem)) return e;
