@@ -175,6 +175,36 @@ def test_attn_blockmask_query_block_edges(impl, d):
 
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("d", [64, 128])
+def test_attn_blockmask_unit_edges_and_rescales(impl, d):
+    """Masked mode at the row counts where a query block's run splits into
+    units of 64 (d = 128: 63, 64, 65 and 128 active rows, one row, none, and
+    17 in the ragged last block), with keys that grow block by block (x(1 + 4 kb))
+    so that later key tiles push the exponent arguments past the running
+    references again and again (the rescale path, repeatedly, in both kernels)."""
+    nb_full, tail = 6, 40
+    N, H = 128 * nb_full + tail, 2
+    rng = np.random.default_rng(70 + d)
+    runs = {0: 64, 1: 65, 2: 63, 3: 128, 4: 1, 5: 0, 6: 17}
+    idx = np.concatenate([np.sort(rng.choice(np.arange(128 * b, min(N, 128 * b + 128)), n, replace=False))
+                          for b, n in runs.items() if n > 0])
+    A = len(idx)
+    q = synth.gaussian_bf16((A, H, d), 71)
+    k = synth.gaussian_bf16((N, H, d), 72).double()
+    ramp = 1.0 + 4.0 * (np.arange(N) // 128)
+    k = (k * torch.from_numpy(ramp)[:, None, None]).to(torch.bfloat16)
+    v = synth.gaussian_bf16((N, H, d), 73)
+    nb = -(-N // 128)
+    bm = torch.from_numpy((rng.random((nb, nb)) < 0.5).astype(np.uint8))
+    bm[np.arange(nb), np.arange(nb)] = 1
+    bm[3] = 1                                                   # the 128-row block keeps every key block
+    vmax = v.double().abs().amax(dim=(0, 2)).numpy()
+    o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm)
+    o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm)
+    _check(o, lse, o_ref, lse_ref, v_absmax=vmax)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("d", [64, 128])
 def test_attn_count_below_cap_leaves_tail(impl, d):
     N, A, H = 700, 300, 2
     q = synth.gaussian_bf16((A, H, d), 20)
