@@ -201,6 +201,8 @@ def test_attn_blockmask_unit_edges_and_rescales(impl, d):
     o, lse = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm)
     o_ref, lse_ref = O.pruned_attn(q, k, v, idx, 1 / math.sqrt(d), blockmask=bm)
     _check(o, lse, o_ref, lse_ref, v_absmax=vmax)
+    o2, _ = _run(impl, q, k, v, idx, 1 / math.sqrt(d), bm=bm, with_lse=False)   # no log-sum-exp output
+    assert torch.equal(o2, o)
 
 
 @pytest.mark.parametrize("impl", IMPLS)
