@@ -841,9 +841,18 @@ def config_sweep(dev, peak_tflops, hbm_gbs, stages_once=False):
     alg = 4.0 * d * H * 128 * float(bm_h[bidx_h // 128].sum())
     alg -= 4.0 * d * H * float(np.sum(bm_h[bidx_h // 128][:, -1])) * (128 - (N - (bm_h.shape[0] - 1) * 128))
     exe = executed_flops(bidx_h, N, H, d, bm_h)
+    # the transposed block kernel is bound by the shared-memory port: per (unit of <= 64 rows, key
+    # tile) it moves 176 KB (TMA writes of K and V 64 KB; MMA operand reads of K 32, Q 16, V 32 and
+    # P^T 16 KB; P^T stores 16 KB) against 128 bytes a clock per SM
+    blocks, rows_b = np.unique(bidx_h // 128, return_counts=True)
+    unit_tiles = float(np.sum(-(-rows_b // 64) * bm_h[blocks].astype(np.int64).sum(axis=1))) * H
+    smem_bytes = unit_tiles * 176 * 1024
+    smem_peak = 128.0 * torch.cuda.get_device_properties(dev).multi_processor_count * 1965e6   # B/s at the max clock
     att["block_sparse"] = {"ms": round(t, 3), "tflops_alg": round(alg / t / 1e9, 1),
                            "tflops_exec": round(exe / t / 1e9, 1), "frac_peak_exec": round(exe / t / 1e9 / peak_tflops, 3),
-                           "exec_over_alg": round(exe / alg, 2)}
+                           "exec_over_alg": round(exe / alg, 2),
+                           "smem_TBps": round(smem_bytes / t / 1e9, 2),
+                           "smem_frac": round(smem_bytes / (t * 1e-3) / smem_peak, 3)}
     out["attention"] = att
     return out
 
